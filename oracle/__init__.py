@@ -1,0 +1,240 @@
+"""CPU oracle (test infrastructure only).
+
+Loads fp8_oracle.c (plain C, built with gcc here) through ctypes.  Only the
+test suite, the smoke check and the benchmark's CPU-baseline leg may import
+this package; the GPU library never does.  The wrappers only marshal numpy
+arrays and split independent scale groups across threads (ctypes releases the
+GIL during a foreign call); all arithmetic happens in the C file.
+
+Every function cites the page passage it follows in fp8_oracle.c; the pins
+that check it against the pages live in tests/test_oracle_*.py.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "fp8_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+E4M3, E5M2 = 0, 1
+PER_TENSOR, GROUP_1x128, BLOCK_128x128 = 0, 1, 2
+KV_PER_TENSOR, KV_PER_HEAD, KV_PER_HEAD_TOK128 = 0, 1, 2
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc: IEEE float, no FMA contraction, no fast-math."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+                               "-fno-fast-math", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            i32, i64, f32, f64, u8 = ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_double, ctypes.c_uint8
+            vp = ctypes.c_void_p
+            lib.orc_fmax.argtypes = [i32]
+            lib.orc_fmax.restype = f32
+            lib.orc_encode.argtypes = [i32, f32]
+            lib.orc_encode.restype = u8
+            lib.orc_encode_nearest.argtypes = [i32, f32]
+            lib.orc_encode_nearest.restype = u8
+            lib.orc_scale.argtypes = [i32, f32]
+            lib.orc_scale.restype = f32
+            lib.orc_decode_array.argtypes = [i32, vp, i64, vp]
+            lib.orc_encode_array.argtypes = [i32, vp, i64, vp]
+            lib.orc_encode_nearest_array.argtypes = [i32, vp, i64, vp]
+            lib.orc_quantize.argtypes = [vp, i64, i64, i32, i32, vp, vp]
+            lib.orc_quantize.restype = i32
+            lib.orc_dequantize.argtypes = [vp, vp, i64, i64, i32, i32, vp]
+            lib.orc_dequantize.restype = i32
+            lib.orc_kv_quantize.argtypes = [vp, vp, i64, i64, i64, i32, i32, vp, vp, vp, vp]
+            lib.orc_kv_quantize.restype = i32
+            lib.orc_gemm_rows.argtypes = [vp, vp, i32, vp, vp, i32, i32, i32, i64, i64, i64, vp, i64, vp]
+            lib.orc_gemm_rows.restype = i32
+            lib.orc_int8_level.argtypes = [f64, f64]
+            lib.orc_int8_level.restype = i32
+            _lib = lib
+    return _lib
+
+
+def _p(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def _threads(threads: int | None) -> int:
+    return max(1, threads if threads else min(32, os.cpu_count() or 1))
+
+
+def _parallel(n: int, fn, threads: int | None, min_chunk: int) -> None:
+    nt = _threads(threads)
+    if nt == 1 or n <= min_chunk:
+        fn(0, n)
+        return
+    chunk = max(min_chunk, -(-n // (nt * 4)))
+    with ThreadPoolExecutor(nt) as ex:
+        list(ex.map(lambda s: fn(s, min(chunk, n - s)), range(0, n, chunk)))
+
+
+def cdiv(a: int, b: int) -> int:
+    return -(-a // b)
+
+
+# ---------------------------------------------------------------- codec
+
+def fmax(fmt: int) -> float:
+    return float(_load().orc_fmax(fmt))
+
+
+def decode(codes: np.ndarray, fmt: int) -> np.ndarray:
+    """uint8 codes -> exact float32 values (NaN codes keep their mantissa as payload)."""
+    c = np.ascontiguousarray(codes, np.uint8)
+    out = np.empty(c.shape, np.float32)
+    _load().orc_decode_array(fmt, _p(c), c.size, _p(out))
+    return out
+
+
+def encode(q: np.ndarray, fmt: int, threads: int | None = None) -> np.ndarray:
+    """float32 -> codes, bit-level round-to-nearest-even with saturation."""
+    q = np.ascontiguousarray(q, np.float32)
+    out = np.empty(q.shape, np.uint8)
+    qf, of = q.reshape(-1), out.reshape(-1)
+    lib = _load()
+    _parallel(qf.size, lambda s, c: lib.orc_encode_array(fmt, _p(qf[s:s + c]), c, _p(of[s:s + c])),
+              threads, 1 << 22)
+    return out
+
+
+def encode_nearest(q: np.ndarray, fmt: int, threads: int | None = None) -> np.ndarray:
+    """float32 -> codes by brute-force nearest-value search (independent encoder)."""
+    q = np.ascontiguousarray(q, np.float32)
+    out = np.empty(q.shape, np.uint8)
+    qf, of = q.reshape(-1), out.reshape(-1)
+    lib = _load()
+    _parallel(qf.size, lambda s, c: lib.orc_encode_nearest_array(fmt, _p(qf[s:s + c]), c, _p(of[s:s + c])),
+              threads, 1 << 18)
+    return out
+
+
+def scale(amax: float, fmt: int) -> float:
+    return float(_load().orc_scale(fmt, amax))
+
+
+def int8_level(x: float, amax: float) -> int:
+    return int(_load().orc_int8_level(x, amax))
+
+
+# ---------------------------------------------------------------- quantize / dequantize
+
+def num_scales(rows: int, cols: int, gran: int) -> int:
+    if gran == PER_TENSOR:
+        return 1
+    if gran == GROUP_1x128:
+        return cdiv(cols, 128) * rows
+    return cdiv(rows, 128) * cdiv(cols, 128)
+
+
+def scale_shape(rows: int, cols: int, gran: int):
+    if gran == PER_TENSOR:
+        return (1,)
+    if gran == GROUP_1x128:
+        return (cdiv(cols, 128), rows)
+    return (cdiv(rows, 128), cdiv(cols, 128))
+
+
+def quantize(x_bf16: np.ndarray, fmt: int, gran: int, threads: int | None = None):
+    """bf16 bits [rows][cols] -> (codes uint8 [rows][cols], scales float32 in the library layout)."""
+    x = np.ascontiguousarray(x_bf16, np.uint16)
+    rows, cols = x.shape
+    codes = np.empty((rows, cols), np.uint8)
+    scales = np.empty(scale_shape(rows, cols, gran), np.float32)
+    lib = _load()
+    if gran == PER_TENSOR:
+        rc = lib.orc_quantize(_p(x), rows, cols, fmt, gran, _p(codes), _p(scales))
+        assert rc == 0
+    elif gran == GROUP_1x128:
+        def run(r0, n):
+            s = np.empty((cdiv(cols, 128), n), np.float32)
+            assert lib.orc_quantize(_p(x[r0:r0 + n]), n, cols, fmt, gran, _p(codes[r0:r0 + n]), _p(s)) == 0
+            scales[:, r0:r0 + n] = s
+        _parallel(rows, run, threads, 64)
+    elif gran == BLOCK_128x128:
+        nbr = cdiv(rows, 128)
+
+        def run(b0, nb):
+            r0, r1 = b0 * 128, min(rows, (b0 + nb) * 128)
+            assert lib.orc_quantize(_p(x[r0:r1]), r1 - r0, cols, fmt, gran, _p(codes[r0:r1]),
+                                    _p(scales[b0:b0 + nb])) == 0
+        _parallel(nbr, run, threads, 1)
+    else:
+        raise ValueError(gran)
+    return codes, scales
+
+
+def dequantize(codes: np.ndarray, scales: np.ndarray, fmt: int, gran: int) -> np.ndarray:
+    """codes [rows][cols] + scales -> bf16 bits [rows][cols]."""
+    c = np.ascontiguousarray(codes, np.uint8)
+    s = np.ascontiguousarray(scales, np.float32)
+    rows, cols = c.shape
+    y = np.empty((rows, cols), np.uint16)
+    assert _load().orc_dequantize(_p(c), _p(s), rows, cols, fmt, gran, _p(y)) == 0
+    return y
+
+
+def kv_scale_shape(tokens: int, heads: int, gran: int):
+    if gran == KV_PER_TENSOR:
+        return (1,)
+    if gran == KV_PER_HEAD:
+        return (heads,)
+    return (cdiv(tokens, 128), heads)
+
+
+def kv_quantize(k_bf16: np.ndarray, v_bf16: np.ndarray, fmt: int, gran: int):
+    """K, V [tokens][heads][head_dim] bf16 bits -> (k_codes, v_codes, k_scales, v_scales)."""
+    k = np.ascontiguousarray(k_bf16, np.uint16)
+    v = np.ascontiguousarray(v_bf16, np.uint16)
+    T, H, D = k.shape
+    kc, vc = np.empty(k.shape, np.uint8), np.empty(v.shape, np.uint8)
+    ks = np.empty(kv_scale_shape(T, H, gran), np.float32)
+    vs = np.empty(kv_scale_shape(T, H, gran), np.float32)
+    rc = _load().orc_kv_quantize(_p(k), _p(v), T, H, D, fmt, gran, _p(kc), _p(vc), _p(ks), _p(vs))
+    assert rc == 0
+    return kc, vc, ks, vs
+
+
+# ---------------------------------------------------------------- GEMM
+
+def gemm_rows(a_codes, sa, ga, b_codes, sb, gb, rows, fmt_a: int = E4M3, fmt_b: int = E4M3,
+              threads: int | None = None) -> np.ndarray:
+    """fp64 rows of C = dequant(A) @ dequant(B)^T for the listed row indices -> [len(rows)][N]."""
+    A = np.ascontiguousarray(a_codes, np.uint8)
+    B = np.ascontiguousarray(b_codes, np.uint8)
+    sA = np.ascontiguousarray(sa, np.float32)
+    sB = np.ascontiguousarray(sb, np.float32)
+    M, K = A.shape
+    N, K2 = B.shape
+    assert K == K2
+    rows = np.ascontiguousarray(rows, np.int64)
+    out = np.empty((rows.size, N), np.float64)
+    lib = _load()
+
+    def run(i0, n):
+        assert lib.orc_gemm_rows(_p(A), _p(sA), ga, _p(B), _p(sB), gb, fmt_a, fmt_b, M, N, K,
+                                 _p(rows[i0:i0 + n]), n, _p(out[i0:i0 + n])) == 0
+    _parallel(rows.size, run, threads, 4)
+    return out
