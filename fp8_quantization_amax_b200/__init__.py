@@ -1,0 +1,263 @@
+"""FP8 (E4M3 / E5M2) scaled quantization, KV-cache quantization, dequantization and the
+block-scaled FP8 GEMM on B200 (sm_100a).
+
+A thin ctypes binding over the C ABI in include/fp8q.h (libfp8q.so, built in-tree by
+``python -m fp8_quantization_amax_b200.build``).  The binding only checks and marshals
+arguments: every step runs in the library's CUDA kernels on the caller's current torch
+stream.  torch supplies device memory and streams; outputs that are not passed in are
+allocated with torch.empty.  There is no CPU path: CPU tensors and a missing library raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = [
+    "E4M3", "E5M2", "PER_TENSOR", "GROUP_1x128", "BLOCK_128x128",
+    "KV_PER_TENSOR", "KV_PER_HEAD", "KV_PER_HEAD_TOK128",
+    "Fp8qError", "lib", "library_path", "num_scales", "workspace_bytes", "kv_num_scales",
+    "kv_workspace_bytes", "gemm_workspace_bytes", "scale_shape", "kv_scale_shape",
+    "fp8_encode", "fp8_decode", "fp8_quantize", "fp8_dequantize", "fp8_kv_quantize",
+    "fp8_gemm_blockscaled",
+]
+
+E4M3, E5M2 = 0, 1
+PER_TENSOR, GROUP_1x128, BLOCK_128x128 = 0, 1, 2
+KV_PER_TENSOR, KV_PER_HEAD, KV_PER_HEAD_TOK128 = 0, 1, 2
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libfp8q.so")
+_lock = threading.Lock()
+_lib = None
+
+
+class Fp8qError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {_status_string(status)} ({status})")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libfp8q.so with argument types set.  Raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise ImportError(f"{_LIB_PATH} is missing; build it with "
+                                  "`python -m fp8_quantization_amax_b200.build`")
+            L = ctypes.CDLL(_LIB_PATH)
+            i32, i64, sz, vp = ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p
+            L.fp8q_status_string.argtypes = [i32]
+            L.fp8q_status_string.restype = ctypes.c_char_p
+            L.fp8q_version.restype = i32
+            L.fp8q_num_scales.argtypes = [i64, i64, i32]
+            L.fp8q_num_scales.restype = sz
+            L.fp8q_workspace_bytes.argtypes = [i64, i64, i32]
+            L.fp8q_workspace_bytes.restype = sz
+            L.fp8q_kv_num_scales.argtypes = [i64, i64, i32]
+            L.fp8q_kv_num_scales.restype = sz
+            L.fp8q_kv_workspace_bytes.argtypes = [i64, i64, i64, i32]
+            L.fp8q_kv_workspace_bytes.restype = sz
+            L.fp8q_gemm_workspace_bytes.argtypes = [i64, i64, i64]
+            L.fp8q_gemm_workspace_bytes.restype = sz
+            L.fp8_encode.argtypes = [vp, i64, i32, vp, vp]
+            L.fp8_decode.argtypes = [vp, i64, i32, vp, vp]
+            L.fp8_quantize.argtypes = [vp, i64, i64, i32, i32, vp, vp, vp, sz, vp]
+            L.fp8_dequantize.argtypes = [vp, vp, i64, i64, i32, i32, vp, vp]
+            L.fp8_kv_quantize.argtypes = [vp, vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, sz, vp]
+            L.fp8_gemm_blockscaled.argtypes = [vp, vp, i32, vp, vp, i32, i64, i64, i64, vp, vp, sz, vp]
+            for fn in ("fp8_encode", "fp8_decode", "fp8_quantize", "fp8_dequantize", "fp8_kv_quantize",
+                       "fp8_gemm_blockscaled"):
+                getattr(L, fn).restype = i32
+            _lib = L
+    return _lib
+
+
+def _status_string(status: int) -> str:
+    try:
+        return lib().fp8q_status_string(status).decode()
+    except Exception:  # pragma: no cover - only while reporting another error
+        return "unknown"
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise Fp8qError(fn, status)
+
+
+def _cdiv(a: int, b: int) -> int:
+    return -(-a // b)
+
+
+# ------------------------------------------------------------------ sizes
+
+def num_scales(rows: int, cols: int, gran: int) -> int:
+    return int(lib().fp8q_num_scales(rows, cols, gran))
+
+
+def workspace_bytes(rows: int, cols: int, gran: int) -> int:
+    return int(lib().fp8q_workspace_bytes(rows, cols, gran))
+
+
+def kv_num_scales(tokens: int, heads: int, gran: int) -> int:
+    return int(lib().fp8q_kv_num_scales(tokens, heads, gran))
+
+
+def kv_workspace_bytes(tokens: int, heads: int, head_dim: int, gran: int) -> int:
+    return int(lib().fp8q_kv_workspace_bytes(tokens, heads, head_dim, gran))
+
+
+def gemm_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib().fp8q_gemm_workspace_bytes(M, N, K))
+
+
+def scale_shape(rows: int, cols: int, gran: int) -> tuple:
+    if gran == PER_TENSOR:
+        return (1,)
+    if gran == GROUP_1x128:
+        return (_cdiv(cols, 128), rows)
+    return (_cdiv(rows, 128), _cdiv(cols, 128))
+
+
+def kv_scale_shape(tokens: int, heads: int, gran: int) -> tuple:
+    if gran == KV_PER_TENSOR:
+        return (1,)
+    if gran == KV_PER_HEAD:
+        return (heads,)
+    return (_cdiv(tokens, 128), heads)
+
+
+# ------------------------------------------------------------------ marshalling helpers
+
+def _dev(t: torch.Tensor, name: str, dtype=None) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (this library has no CPU path)")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _workspace(nbytes: int, device, ws: torch.Tensor | None) -> torch.Tensor | None:
+    if nbytes == 0:
+        return ws
+    if ws is None:
+        return torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return ws
+
+
+# ------------------------------------------------------------------ codec
+
+def fp8_encode(q: torch.Tensor, fmt: int = E4M3, out: torch.Tensor | None = None) -> torch.Tensor:
+    """fp32 values -> FP8 codes (uint8), round to nearest even, saturating."""
+    _dev(q, "q", torch.float32)
+    out = torch.empty(q.shape, dtype=torch.uint8, device=q.device) if out is None else _dev(out, "out", torch.uint8)
+    _check("fp8_encode", lib().fp8_encode(_ptr(q), q.numel(), fmt, _ptr(out), _stream(q.device)))
+    return out
+
+
+def fp8_decode(codes: torch.Tensor, fmt: int = E4M3, out: torch.Tensor | None = None) -> torch.Tensor:
+    """FP8 codes (uint8) -> exact fp32 values."""
+    _dev(codes, "codes", torch.uint8)
+    out = torch.empty(codes.shape, dtype=torch.float32, device=codes.device) if out is None else \
+        _dev(out, "out", torch.float32)
+    _check("fp8_decode", lib().fp8_decode(_ptr(codes), codes.numel(), fmt, _ptr(out), _stream(codes.device)))
+    return out
+
+
+# ------------------------------------------------------------------ quantize / dequantize
+
+def fp8_quantize(x: torch.Tensor, fmt: int = E4M3, gran: int = GROUP_1x128, codes: torch.Tensor | None = None,
+                 scales: torch.Tensor | None = None, ws: torch.Tensor | None = None):
+    """bf16 [rows][cols] -> (codes uint8 [rows][cols], fp32 scales in the library layout)."""
+    _dev(x, "x", torch.bfloat16)
+    if x.dim() != 2:
+        raise ValueError("x must be 2-D [rows][cols]")
+    rows, cols = x.shape
+    codes = torch.empty((rows, cols), dtype=torch.uint8, device=x.device) if codes is None else \
+        _dev(codes, "codes", torch.uint8)
+    scales = torch.empty(scale_shape(rows, cols, gran), dtype=torch.float32, device=x.device) if scales is None \
+        else _dev(scales, "scales", torch.float32)
+    nws = workspace_bytes(rows, cols, gran)
+    ws = _workspace(nws, x.device, ws)
+    st = lib().fp8_quantize(_ptr(x), rows, cols, fmt, gran, _ptr(codes), _ptr(scales), _ptr(ws),
+                            0 if ws is None else ws.numel() * ws.element_size(), _stream(x.device))
+    _check("fp8_quantize", st)
+    return codes, scales
+
+
+def fp8_dequantize(codes: torch.Tensor, scales: torch.Tensor, fmt: int = E4M3, gran: int = GROUP_1x128,
+                   out: torch.Tensor | None = None) -> torch.Tensor:
+    """codes + scales -> bf16 [rows][cols], y = bf16(decode(code) * s)."""
+    _dev(codes, "codes", torch.uint8)
+    _dev(scales, "scales", torch.float32)
+    if codes.dim() != 2:
+        raise ValueError("codes must be 2-D [rows][cols]")
+    rows, cols = codes.shape
+    out = torch.empty((rows, cols), dtype=torch.bfloat16, device=codes.device) if out is None else \
+        _dev(out, "out", torch.bfloat16)
+    st = lib().fp8_dequantize(_ptr(codes), _ptr(scales), rows, cols, fmt, gran, _ptr(out), _stream(codes.device))
+    _check("fp8_dequantize", st)
+    return out
+
+
+def fp8_kv_quantize(k: torch.Tensor, v: torch.Tensor, fmt: int = E4M3, gran: int = KV_PER_HEAD,
+                    k_codes=None, v_codes=None, k_scales=None, v_scales=None, ws=None):
+    """K, V bf16 [tokens][heads][head_dim] -> (k_codes, v_codes, k_scales, v_scales)."""
+    _dev(k, "k", torch.bfloat16)
+    _dev(v, "v", torch.bfloat16)
+    if k.dim() != 3 or k.shape != v.shape:
+        raise ValueError("k and v must both be [tokens][heads][head_dim]")
+    T, H, D = k.shape
+    dev = k.device
+    k_codes = torch.empty(k.shape, dtype=torch.uint8, device=dev) if k_codes is None else _dev(k_codes, "k_codes", torch.uint8)
+    v_codes = torch.empty(v.shape, dtype=torch.uint8, device=dev) if v_codes is None else _dev(v_codes, "v_codes", torch.uint8)
+    shp = kv_scale_shape(T, H, gran)
+    k_scales = torch.empty(shp, dtype=torch.float32, device=dev) if k_scales is None else _dev(k_scales, "k_scales", torch.float32)
+    v_scales = torch.empty(shp, dtype=torch.float32, device=dev) if v_scales is None else _dev(v_scales, "v_scales", torch.float32)
+    ws = _workspace(kv_workspace_bytes(T, H, D, gran), dev, ws)
+    st = lib().fp8_kv_quantize(_ptr(k), _ptr(v), T, H, D, fmt, gran, _ptr(k_codes), _ptr(v_codes), _ptr(k_scales),
+                               _ptr(v_scales), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+                               _stream(dev))
+    _check("fp8_kv_quantize", st)
+    return k_codes, v_codes, k_scales, v_scales
+
+
+# ------------------------------------------------------------------ GEMM
+
+def fp8_gemm_blockscaled(a: torch.Tensor, sa: torch.Tensor, b: torch.Tensor, sb: torch.Tensor,
+                         ga: int = GROUP_1x128, gb: int = BLOCK_128x128, out: torch.Tensor | None = None,
+                         ws: torch.Tensor | None = None) -> torch.Tensor:
+    """C[M][N] (bf16) = block-scaled FP8 product of A [M][K] and B [N][K] (E4M3 codes, K-major)."""
+    _dev(a, "a", torch.uint8)
+    _dev(b, "b", torch.uint8)
+    _dev(sa, "sa", torch.float32)
+    _dev(sb, "sb", torch.float32)
+    M, K = a.shape
+    N, K2 = b.shape
+    if K != K2:
+        raise ValueError("a and b disagree on K")
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device) if out is None else _dev(out, "out", torch.bfloat16)
+    ws = _workspace(gemm_workspace_bytes(M, N, K), a.device, ws)
+    st = lib().fp8_gemm_blockscaled(_ptr(a), _ptr(sa), ga, _ptr(b), _ptr(sb), gb, M, N, K, _ptr(out), _ptr(ws),
+                                    0 if ws is None else ws.numel() * ws.element_size(), _stream(a.device))
+    _check("fp8_gemm_blockscaled", st)
+    return out

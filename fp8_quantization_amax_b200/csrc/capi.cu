@@ -1,0 +1,181 @@
+// C-ABI entry points declared in include/fp8q.h: argument validation, sizes and dispatch.
+// Every check happens on the host before anything is launched.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "fp8q.h"
+#include "internal.h"
+
+namespace {
+
+constexpr int64_t kMaxElems = int64_t(1) << 33;   // 32-bit indexing of 16-byte pieces of two tensors
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+bool valid_fmt(int f) { return f == FP8Q_E4M3 || f == FP8Q_E5M2; }
+bool valid_gran(int g) { return g == FP8Q_PER_TENSOR || g == FP8Q_GROUP_1x128 || g == FP8Q_BLOCK_128x128; }
+bool valid_kv_gran(int g) {
+  return g == FP8Q_KV_PER_TENSOR || g == FP8Q_KV_PER_HEAD || g == FP8Q_KV_PER_HEAD_TOK128;
+}
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// rows * cols without overflow; -1 when it does not fit the library's indexing
+int64_t checked_elems(int64_t a, int64_t b) {
+  if (a < 0 || b < 0) return -1;
+  if (a == 0 || b == 0) return 0;
+  if (a > kMaxElems / b) return -1;
+  return a * b;
+}
+
+fp8q_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* fp8q_status_string(fp8q_status status) {
+  switch (status) {
+    case FP8Q_OK: return "ok";
+    case FP8Q_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case FP8Q_ERR_UNSUPPORTED: return "unsupported";
+    case FP8Q_ERR_WORKSPACE: return "workspace missing or too small";
+    case FP8Q_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+int fp8q_version(void) { return 100; }
+
+size_t fp8q_num_scales(int64_t rows, int64_t cols, fp8q_granularity g) {
+  if (rows < 0 || cols < 0 || !valid_gran(g)) return 0;
+  if (g == FP8Q_PER_TENSOR) return 1;
+  if (g == FP8Q_GROUP_1x128) return (size_t)(cdiv(cols, 128) * rows);
+  return (size_t)(cdiv(rows, 128) * cdiv(cols, 128));
+}
+
+size_t fp8q_workspace_bytes(int64_t rows, int64_t cols, fp8q_granularity g) {
+  if (rows < 0 || cols < 0 || !valid_gran(g)) return 0;
+  return g == FP8Q_PER_TENSOR ? fp8q::two_pass_workspace_bytes(1, 1) : 0;
+}
+
+size_t fp8q_kv_num_scales(int64_t tokens, int64_t heads, fp8q_kv_granularity g) {
+  if (tokens < 0 || heads < 0 || !valid_kv_gran(g)) return 0;
+  if (g == FP8Q_KV_PER_TENSOR) return 1;
+  if (g == FP8Q_KV_PER_HEAD) return (size_t)heads;
+  return (size_t)(cdiv(tokens, 128) * heads);
+}
+
+size_t fp8q_kv_workspace_bytes(int64_t tokens, int64_t heads, int64_t head_dim, fp8q_kv_granularity g) {
+  if (tokens < 0 || heads < 0 || head_dim < 0 || !valid_kv_gran(g)) return 0;
+  if (g == FP8Q_KV_PER_TENSOR) return fp8q::two_pass_workspace_bytes(2, 1);
+  if (g == FP8Q_KV_PER_HEAD) return fp8q::two_pass_workspace_bytes(2, heads);
+  return 0;
+}
+
+size_t fp8q_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || N < 0 || K < 0) return 0;
+  return fp8q::gemm_workspace_bytes(M, N, K);
+}
+
+fp8q_status fp8_encode(const float* q, int64_t n, fp8q_format f, uint8_t* codes, fp8q_stream_t stream) {
+  if (n < 0 || n > kMaxElems || !valid_fmt(f)) return FP8Q_ERR_INVALID_ARGUMENT;
+  if (n == 0) return FP8Q_OK;
+  if (!q || !codes || !aligned(q, 16) || !aligned(codes, 16)) return FP8Q_ERR_INVALID_ARGUMENT;
+  return from_cuda(fp8q::launch_encode(q, n, f, codes, (cudaStream_t)stream));
+}
+
+fp8q_status fp8_decode(const uint8_t* codes, int64_t n, fp8q_format f, float* out, fp8q_stream_t stream) {
+  if (n < 0 || n > kMaxElems || !valid_fmt(f)) return FP8Q_ERR_INVALID_ARGUMENT;
+  if (n == 0) return FP8Q_OK;
+  if (!codes || !out || !aligned(codes, 16) || !aligned(out, 16)) return FP8Q_ERR_INVALID_ARGUMENT;
+  return from_cuda(fp8q::launch_decode(codes, n, f, out, (cudaStream_t)stream));
+}
+
+fp8q_status fp8_quantize(const void* x, int64_t rows, int64_t cols, fp8q_format f, fp8q_granularity g,
+                         uint8_t* codes, float* scales, void* ws, size_t ws_bytes, fp8q_stream_t stream) {
+  const int64_t n = checked_elems(rows, cols);
+  if (rows < 0 || cols < 0 || !valid_fmt(f) || !valid_gran(g) || cols % 8 != 0) return FP8Q_ERR_INVALID_ARGUMENT;
+  if (n < 0) return FP8Q_ERR_UNSUPPORTED;
+  if (n > 0 && (!x || !codes || !aligned(x, 16) || !aligned(codes, 16))) return FP8Q_ERR_INVALID_ARGUMENT;
+  if ((n > 0 || g == FP8Q_PER_TENSOR) && (!scales || !aligned(scales, 4))) return FP8Q_ERR_INVALID_ARGUMENT;
+  const cudaStream_t st = (cudaStream_t)stream;
+  const uint16_t* xs = static_cast<const uint16_t*>(x);
+  if (g == FP8Q_PER_TENSOR) {
+    const size_t need = fp8q_workspace_bytes(rows, cols, g);
+    if (!ws || ws_bytes < need || !aligned(ws, 4)) return FP8Q_ERR_WORKSPACE;
+    return from_cuda(fp8q::launch_quant_two_pass(xs, nullptr, codes, nullptr, scales, nullptr, 1, rows, 1, cols, f,
+                                                 static_cast<float*>(ws), st));
+  }
+  if (n == 0) return FP8Q_OK;
+  if (g == FP8Q_GROUP_1x128) return from_cuda(fp8q::launch_quant_1x128(xs, rows, cols, f, codes, scales, st));
+  return from_cuda(
+      fp8q::launch_quant_tiles(xs, nullptr, codes, nullptr, scales, nullptr, 1, rows, cols, cols, 128, f, st));
+}
+
+fp8q_status fp8_dequantize(const uint8_t* codes, const float* scales, int64_t rows, int64_t cols, fp8q_format f,
+                           fp8q_granularity g, void* y, fp8q_stream_t stream) {
+  const int64_t n = checked_elems(rows, cols);
+  if (rows < 0 || cols < 0 || !valid_fmt(f) || !valid_gran(g) || cols % 8 != 0) return FP8Q_ERR_INVALID_ARGUMENT;
+  if (n < 0) return FP8Q_ERR_UNSUPPORTED;
+  if (n == 0) return FP8Q_OK;
+  if (!codes || !scales || !y || !aligned(codes, 16) || !aligned(y, 16) || !aligned(scales, 4))
+    return FP8Q_ERR_INVALID_ARGUMENT;
+  return from_cuda(fp8q::launch_dequant(codes, scales, rows, cols, f, g, static_cast<uint16_t*>(y),
+                                        (cudaStream_t)stream));
+}
+
+fp8q_status fp8_kv_quantize(const void* k, const void* v, int64_t tokens, int64_t heads, int64_t head_dim,
+                            fp8q_format f, fp8q_kv_granularity g, uint8_t* k_codes, uint8_t* v_codes,
+                            float* k_scales, float* v_scales, void* ws, size_t ws_bytes, fp8q_stream_t stream) {
+  if (tokens < 0 || heads < 0 || head_dim < 0 || !valid_fmt(f) || !valid_kv_gran(g) || head_dim % 8 != 0)
+    return FP8Q_ERR_INVALID_ARGUMENT;
+  const int64_t row = checked_elems(heads, head_dim);
+  const int64_t n = row < 0 ? -1 : checked_elems(tokens, row);
+  if (n < 0) return FP8Q_ERR_UNSUPPORTED;
+  if (g == FP8Q_KV_PER_HEAD_TOK128 && head_dim > 256) return FP8Q_ERR_UNSUPPORTED;
+  if (g == FP8Q_KV_PER_HEAD && heads > 128) return FP8Q_ERR_UNSUPPORTED;
+  const size_t nsc = fp8q_kv_num_scales(tokens, heads, g);
+  if (n > 0 && (!k || !v || !k_codes || !v_codes || !aligned(k, 16) || !aligned(v, 16) || !aligned(k_codes, 16) ||
+                !aligned(v_codes, 16)))
+    return FP8Q_ERR_INVALID_ARGUMENT;
+  if (nsc > 0 && (!k_scales || !v_scales || !aligned(k_scales, 4) || !aligned(v_scales, 4)))
+    return FP8Q_ERR_INVALID_ARGUMENT;
+  const cudaStream_t st = (cudaStream_t)stream;
+  const uint16_t* ks = static_cast<const uint16_t*>(k);
+  const uint16_t* vs = static_cast<const uint16_t*>(v);
+  if (g == FP8Q_KV_PER_HEAD_TOK128) {
+    if (n == 0) return FP8Q_OK;
+    return from_cuda(fp8q::launch_quant_tiles(ks, vs, k_codes, v_codes, k_scales, v_scales, 2, tokens, row, row,
+                                              (int)head_dim, f, st));
+  }
+  if (nsc == 0) return FP8Q_OK;   // no heads: nothing to write
+  const size_t need = fp8q_kv_workspace_bytes(tokens, heads, head_dim, g);
+  if (!ws || ws_bytes < need || !aligned(ws, 4)) return FP8Q_ERR_WORKSPACE;
+  const int64_t h = g == FP8Q_KV_PER_TENSOR ? 1 : heads;
+  const int64_t d = g == FP8Q_KV_PER_TENSOR ? row : head_dim;
+  return from_cuda(fp8q::launch_quant_two_pass(ks, vs, k_codes, v_codes, k_scales, v_scales, 2, tokens, h, d, f,
+                                               static_cast<float*>(ws), st));
+}
+
+fp8q_status fp8_gemm_blockscaled(const uint8_t* A, const float* sA, fp8q_granularity gA, const uint8_t* B,
+                                 const float* sB, fp8q_granularity gB, int64_t M, int64_t N, int64_t K, void* C,
+                                 void* ws, size_t ws_bytes, fp8q_stream_t stream) {
+  if (M < 0 || N < 0 || K < 0) return FP8Q_ERR_INVALID_ARGUMENT;
+  if (!(gA == FP8Q_GROUP_1x128 || gA == FP8Q_PER_TENSOR)) return FP8Q_ERR_INVALID_ARGUMENT;
+  if (!(gB == FP8Q_BLOCK_128x128 || gB == FP8Q_PER_TENSOR)) return FP8Q_ERR_INVALID_ARGUMENT;
+  if (M == 0 || N == 0) return FP8Q_OK;
+  if (N % 128 != 0 || K % 128 != 0 || K == 0) return FP8Q_ERR_UNSUPPORTED;
+  if (checked_elems(M, K) < 0 || checked_elems(N, K) < 0 || checked_elems(M, N) < 0) return FP8Q_ERR_UNSUPPORTED;
+  if (M > (int64_t(1) << 31) - 1 || N > (int64_t(1) << 31) - 1) return FP8Q_ERR_UNSUPPORTED;
+  if (!A || !B || !C || !sA || !sB || !aligned(A, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(sA, 4) ||
+      !aligned(sB, 4))
+    return FP8Q_ERR_INVALID_ARGUMENT;
+  const size_t need = fp8q::gemm_workspace_bytes(M, N, K);
+  if (need > 0 && (!ws || ws_bytes < need || !aligned(ws, 16))) return FP8Q_ERR_WORKSPACE;
+  const cudaError_t e = fp8q::launch_gemm(A, sA, gA, B, sB, gB, M, N, K, static_cast<uint16_t*>(C), ws, ws_bytes,
+                                          (cudaStream_t)stream);
+  if (e == cudaErrorNotSupported) return FP8Q_ERR_UNSUPPORTED;
+  return from_cuda(e);
+}
+
+}  // extern "C"

@@ -1,0 +1,52 @@
+// Launchers shared between the C-ABI entry points and the kernel files.  Host-side only.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace fp8q {
+
+// number of SMs of the current device (queried once per device)
+int device_sm_count();
+
+// largest number of first-pass partial maxima any two-pass launch writes, per scale group
+constexpr int kMaxPartials = 1024;
+
+// 32-bit unsigned division by an invariant divisor (T. Granlund, P. Montgomery, "Division by
+// invariant integers using multiplication", PLDI 1994): q = (umulhi(n, m) + n) >> s.
+struct FastDiv {
+  uint32_t d, m, s;
+};
+FastDiv make_fastdiv(uint32_t d);
+
+cudaError_t launch_encode(const float* q, int64_t n, int fmt, uint8_t* codes, cudaStream_t st);
+cudaError_t launch_decode(const uint8_t* codes, int64_t n, int fmt, float* out, cudaStream_t st);
+
+// one scale per (row, 128 consecutive columns); scales laid out [ceil(cols/128)][rows]
+cudaError_t launch_quant_1x128(const uint16_t* x, int64_t rows, int64_t cols, int fmt, uint8_t* codes,
+                               float* scales, cudaStream_t st);
+
+// one scale per tile of 128 rows x gw columns of a [rows][ld] matrix (cols valid columns);
+// up to two tensors in one launch; scales [ceil(rows/128)][nbc]
+cudaError_t launch_quant_tiles(const uint16_t* x0, const uint16_t* x1, uint8_t* c0, uint8_t* c1, float* s0,
+                               float* s1, int ntens, int64_t rows, int64_t cols, int64_t ld, int gw, int fmt,
+                               cudaStream_t st);
+
+// two passes: amax per (tensor, head) over all rows, then the cast.  Each tensor is
+// [rows][heads * head_dim]; per-tensor quantization is heads = 1, head_dim = cols.
+size_t two_pass_workspace_bytes(int ntens, int64_t heads);
+cudaError_t launch_quant_two_pass(const uint16_t* x0, const uint16_t* x1, uint8_t* c0, uint8_t* c1, float* s0,
+                                  float* s1, int ntens, int64_t rows, int64_t heads, int64_t head_dim, int fmt,
+                                  float* ws, cudaStream_t st);
+
+// y = bf16(decode(code) * s) under a granularity (0 tensor, 1 1x128, 2 128x128)
+cudaError_t launch_dequant(const uint8_t* codes, const float* scales, int64_t rows, int64_t cols, int fmt,
+                           int gran, uint16_t* y, cudaStream_t st);
+
+// block-scaled / per-tensor FP8 GEMM on tcgen05
+cudaError_t launch_gemm(const uint8_t* A, const float* sA, int gA, const uint8_t* B, const float* sB, int gB,
+                        int64_t M, int64_t N, int64_t K, uint16_t* C, void* ws, size_t ws_bytes,
+                        cudaStream_t st);
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+}  // namespace fp8q

@@ -1,0 +1,202 @@
+/*
+ * fp8q — FP8 (E4M3 / E5M2) scaled quantization, dequantization, KV-cache
+ * quantization and block-scaled FP8 GEMM on NVIDIA B200 (sm_100a).
+ *
+ * C ABI.  Every pointer argument named as a tensor is a DEVICE pointer owned
+ * by the caller; the library allocates no memory.  Every compute call is
+ * asynchronous on the caller's stream (NULL = the legacy default stream) and
+ * never synchronizes the host.  Argument errors are reported before anything
+ * is launched; a launch failure returns FP8Q_ERR_CUDA; faults inside a kernel
+ * surface at the caller's next synchronization.  No C++ exception crosses
+ * this interface.
+ *
+ * Method (web pages the definitions come from, cited by title and section):
+ *   [W] wangyu.me, "大语言模型量化技术（五）：FP8" — format table and step
+ *       sizes ("FP8 是什么"); quantization steps s = amax/448, x/s, round to
+ *       nearest, saturate ("什么是 FP8 量化"); 128x128 weight blocks and the
+ *       weight_scale_inv layout ("权重量化：128x128 分块 FP8"); dynamic
+ *       per-token / per-128-group activation scales and the GEMM identity
+ *       ("激活动态量化"); fp32 accumulation with scales applied on
+ *       accumulation ("FP8 矩阵乘").
+ *   [C] charles2530.github.io, "量化：FP8 与混合精度推理" — x_fp8 =
+ *       FP8Cast(x/s), x_hat = s * x_fp8.
+ *   [P] pwwt.cn, "从权重到激活：FP8 量化到底动了哪些东西" — separate K and V
+ *       scales, per-head keys (section 1); per-head x per-128-token KV blocks
+ *       (section 3).
+ *   [M] api.makesence.top, "LLM推理量化:FP8 versus INT8" — W8A8 E4M3 with
+ *       an E5M2 KV cache (section 二).
+ *
+ * Arithmetic, per scale group G (bit-exact contract):
+ *   amax = max over G of |x|        (x is bf16, widened exactly to fp32;
+ *                                    a NaN anywhere in G makes amax NaN)
+ *   s    = amax / FMAX              (one IEEE fp32 division; FMAX = 448 for
+ *                                    E4M3, 57344 for E5M2; stored as the
+ *                                    group's fp32 scale, a dequant multiplier)
+ *   code = FP8_RNE_SAT(x / s)       (the quotient is the IEEE fp32
+ *                                    round-to-nearest-even quotient; it is
+ *                                    then rounded to nearest-even on the FP8
+ *                                    grid, subnormals included, saturating to
+ *                                    +-FMAX; Inf saturates too)
+ *   amax == 0 gives s = 0 and signed-zero codes (no division).
+ *   dequant: y = bf16_rne( fp32( decode(code) * s ) ).
+ *
+ * Layouts (row-major, contiguous):
+ *   tensors, codes, outputs   [rows][cols]
+ *   FP8Q_PER_TENSOR scales    [1]
+ *   FP8Q_GROUP_1x128 scales   [ceil(cols/128)][rows]   (group-major: the 128
+ *                             row scales of one K-block are contiguous)
+ *   FP8Q_BLOCK_128x128 scales [ceil(rows/128)][ceil(cols/128)]
+ *                             (the weight_scale_inv layout of [W])
+ *   KV caches                 [tokens][heads][head_dim]
+ *   KV scales                 per-tensor [1]; per-head [heads];
+ *                             per-head x 128-token [ceil(tokens/128)][heads]
+ *   GEMM                      C[M][N] = A[M][K] . B[N][K]^T, A and B K-major.
+ *
+ * Alignment: tensor, code and output pointers 16-byte aligned; scale
+ * pointers 4-byte aligned; cols (and head_dim) a multiple of 8.
+ */
+#ifndef FP8Q_H
+#define FP8Q_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FP8Q_API __attribute__((visibility("default")))
+#else
+#define FP8Q_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; declared here so this header needs no CUDA headers. */
+typedef struct CUstream_st *fp8q_stream_t;
+
+typedef enum {
+    FP8Q_OK = 0,
+    FP8Q_ERR_INVALID_ARGUMENT = 1, /* null pointer, negative size, misalignment, bad enum  */
+    FP8Q_ERR_UNSUPPORTED = 2,      /* valid request outside what this build implements     */
+    FP8Q_ERR_WORKSPACE = 3,        /* workspace missing or smaller than *_workspace_bytes() */
+    FP8Q_ERR_CUDA = 4              /* a CUDA call or launch failed                          */
+} fp8q_status;
+
+typedef enum { FP8Q_E4M3 = 0, FP8Q_E5M2 = 1 } fp8q_format;
+
+typedef enum {
+    FP8Q_PER_TENSOR = 0,    /* one scale for the whole tensor                             */
+    FP8Q_GROUP_1x128 = 1,   /* one scale per row and 128 consecutive columns ([W] 激活动态量化) */
+    FP8Q_BLOCK_128x128 = 2  /* one scale per 128x128 block ([W] 权重量化)                  */
+} fp8q_granularity;
+
+typedef enum {
+    FP8Q_KV_PER_TENSOR = 0,      /* one scale for K, one for V ([M] section 二)           */
+    FP8Q_KV_PER_HEAD = 1,        /* one scale per head, separately for K and V ([P] 1)    */
+    FP8Q_KV_PER_HEAD_TOK128 = 2  /* one per head and 128-token block ([P] section 3)       */
+} fp8q_kv_granularity;
+
+/* Human-readable name of a status code (static storage; never NULL). */
+FP8Q_API const char *fp8q_status_string(fp8q_status status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+FP8Q_API int fp8q_version(void);
+
+/* ---------------------------------------------------------------- sizes */
+
+/* Number of fp32 scales fp8_quantize writes for a [rows][cols] tensor; 0 on a bad argument. */
+FP8Q_API size_t fp8q_num_scales(int64_t rows, int64_t cols, fp8q_granularity g);
+
+/* Device workspace bytes fp8_quantize needs (per-tensor partial maxima; 0 for one-pass granularities). */
+FP8Q_API size_t fp8q_workspace_bytes(int64_t rows, int64_t cols, fp8q_granularity g);
+
+/* Number of fp32 scales fp8_kv_quantize writes into EACH of k_scales and v_scales. */
+FP8Q_API size_t fp8q_kv_num_scales(int64_t tokens, int64_t heads, fp8q_kv_granularity g);
+
+/* Device workspace bytes fp8_kv_quantize needs (0 for the one-pass per-head x 128-token case). */
+FP8Q_API size_t fp8q_kv_workspace_bytes(int64_t tokens, int64_t heads, int64_t head_dim, fp8q_kv_granularity g);
+
+/* Device workspace bytes fp8_gemm_blockscaled needs for this shape (0 when none is needed). */
+FP8Q_API size_t fp8q_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/* ---------------------------------------------------------------- codec */
+
+/*
+ * Element-wise FP8 encode: codes[i] = FP8_RNE_SAT(q[i]) ([W] "FP8 是什么": round to
+ * the nearest representable value, ties to even, out-of-range values saturate to
+ * +-max; NaN stays NaN).  q: fp32 [n]; codes: uint8 [n].  Both 16-byte aligned.
+ * n == 0 is a no-op.
+ */
+FP8Q_API fp8q_status fp8_encode(const float *q, int64_t n, fp8q_format f, uint8_t *codes, fp8q_stream_t stream);
+
+/*
+ * Element-wise FP8 decode to the exact fp32 value ([W] format table).  codes: uint8 [n];
+ * out: fp32 [n].  Both 16-byte aligned.  E4M3 has no Inf; S.1111.111 decodes to NaN.
+ */
+FP8Q_API fp8q_status fp8_decode(const uint8_t *codes, int64_t n, fp8q_format f, float *out, fp8q_stream_t stream);
+
+/* ---------------------------------------------------------------- quantize */
+
+/*
+ * Scaled FP8 quantization of one bf16 tensor ([W] "什么是 FP8 量化", "权重量化",
+ * "激活动态量化"; [C] x_fp8 = FP8Cast(x/s)).
+ *   x       bf16 [rows][cols] (device)
+ *   codes   uint8 [rows][cols] (device, written)
+ *   scales  fp32, fp8q_num_scales(rows, cols, g) entries in the layout above (device, written)
+ *   ws      device workspace of at least fp8q_workspace_bytes(rows, cols, g) bytes
+ *           (may be NULL when that is 0); its contents need no initialisation
+ * Per-tensor runs two kernels (the whole tensor's amax must be known before any
+ * element is cast); the 1x128 and 128x128 granularities run one fused kernel.
+ * rows == 0 or cols == 0 writes nothing, except that a per-tensor call writes s = 0.
+ */
+FP8Q_API fp8q_status fp8_quantize(const void *x, int64_t rows, int64_t cols, fp8q_format f, fp8q_granularity g,
+                         uint8_t *codes, float *scales, void *ws, size_t ws_bytes, fp8q_stream_t stream);
+
+/*
+ * Dequantization x_hat = s * x_fp8 ([C]; [W] "什么是 FP8 量化", restore x ~ x_hat * s),
+ * computed as y = bf16_rne(fp32(decode(code) * s)).
+ *   codes   uint8 [rows][cols] (device);  scales as written by fp8_quantize (device)
+ *   y       bf16 [rows][cols] (device, written)
+ */
+FP8Q_API fp8q_status fp8_dequantize(const uint8_t *codes, const float *scales, int64_t rows, int64_t cols,
+                           fp8q_format f, fp8q_granularity g, void *y, fp8q_stream_t stream);
+
+/*
+ * KV-cache quantization with separate K and V scales ([P] sections 1 and 3; [M] 二).
+ *   k, v                 bf16 [tokens][heads][head_dim] (device); head_dim % 8 == 0, head_dim <= 256
+ *   k_codes, v_codes     uint8, same shape (device, written)
+ *   k_scales, v_scales   fp32, fp8q_kv_num_scales(tokens, heads, g) entries each (device, written)
+ *   ws                   at least fp8q_kv_workspace_bytes(...) bytes (device), may be NULL when 0
+ * Per-tensor and per-head run two kernels; per-head x 128-token runs one.
+ */
+FP8Q_API fp8q_status fp8_kv_quantize(const void *k, const void *v, int64_t tokens, int64_t heads, int64_t head_dim,
+                            fp8q_format f, fp8q_kv_granularity g, uint8_t *k_codes, uint8_t *v_codes,
+                            float *k_scales, float *v_scales, void *ws, size_t ws_bytes,
+                            fp8q_stream_t stream);
+
+/* ---------------------------------------------------------------- GEMM */
+
+/*
+ * Block-scaled FP8 GEMM ([W] "激活动态量化", "FP8 矩阵乘"):
+ *   C[m][n] = bf16_rne( sum_kb sA(m,kb) * sB(n,kb) * P_kb[m][n] ),
+ *   P_kb[m][n] = sum over k in K-block kb (128 wide) of decode(A[m][k]) * decode(B[n][k]),
+ * with P_kb from the FP8 tensor cores and all accumulation in fp32.
+ *   A   E4M3 codes [M][K] (K-major);  sA: gA = FP8Q_GROUP_1x128 ([K/128][M]) or FP8Q_PER_TENSOR ([1])
+ *   B   E4M3 codes [N][K] (K-major, W in R^{N x K});
+ *       sB: gB = FP8Q_BLOCK_128x128 ([N/128][K/128]) or FP8Q_PER_TENSOR ([1])
+ *   C   bf16 [M][N] (device, written)
+ * When both are per-tensor the product is accumulated over all of K and scaled once
+ * at the end: C = bf16(sA * sB * sum_k a*b).
+ * Requirements: M >= 1; N % 128 == 0; K % 128 == 0 (else FP8Q_ERR_UNSUPPORTED);
+ * A, B, C 16-byte aligned.  ws may be NULL when fp8q_gemm_workspace_bytes() is 0.
+ */
+FP8Q_API fp8q_status fp8_gemm_blockscaled(const uint8_t *A, const float *sA, fp8q_granularity gA,
+                                 const uint8_t *B, const float *sB, fp8q_granularity gB,
+                                 int64_t M, int64_t N, int64_t K, void *C,
+                                 void *ws, size_t ws_bytes, fp8q_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8Q_H */

@@ -124,6 +124,8 @@ def normal_bf16(k: int, shape, std: float, row_gain: np.ndarray | None = None,
 
 def distinct_indices(k: int, count: int, bound: int) -> np.ndarray:
     """`count` distinct indices in [0, bound): successive outputs mod bound, repeats skipped."""
+    if count > bound:
+        raise ValueError(f"cannot draw {count} distinct indices from {bound}")
     seen: dict[int, None] = {}
     i = 0
     while len(seen) < count:
@@ -149,9 +151,12 @@ def scale_points(out: np.ndarray, k: int, std: float, idx: np.ndarray, gain: flo
 
 def per_tensor_1024(seed: int = 0, rows: int = 1024, cols: int = 1024) -> np.ndarray:
     """1024x1024 bf16: every entry ~ U(-0.1, 0.1), then 64 distinct positions overwritten
-    with outliers of magnitude ~ U(5, 10) and a random sign."""
+    with outliers of magnitude ~ U(5, 10) and a random sign (smaller shapes: one outlier per
+    16 elements at most)."""
     x = uniform_bf16(key(seed, 0), (rows, cols), -0.1, 0.1)
-    n_out = 64
+    n_out = min(64, rows * cols // 16)
+    if n_out == 0:
+        return x
     pos = distinct_indices(key(seed, 1), n_out, rows * cols)
     mag = uniform_f64(key(seed, 2), n_out, 5.0, 10.0)
     sgn = np.where(u64(key(seed, 3), n_out) & np.uint64(1), -1.0, 1.0)

@@ -1,0 +1,115 @@
+"""The C-ABI library loads, exports every function include/fp8q.h declares, and rejects bad
+arguments before launching anything.  No call here reaches a kernel: these run without a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import fp8_quantization_amax_b200 as fq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp8q.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from fp8_quantization_amax_b200 import build
+    build.build()
+    return fq.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"FP8Q_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for fn in ["fp8_quantize", "fp8_dequantize", "fp8_kv_quantize", "fp8_gemm_blockscaled", "fp8_encode",
+               "fp8_decode", "fp8q_num_scales", "fp8q_workspace_bytes", "fp8q_status_string"]:
+        assert fn in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for fn in declared_functions():
+        assert hasattr(L, fn), fn
+        assert ctypes.cast(getattr(L, fn), ctypes.c_void_p).value
+
+
+def test_status_strings(L):
+    for code in range(5):
+        assert L.fp8q_status_string(code)
+    assert L.fp8q_status_string(99) == b"unknown status"
+    assert L.fp8q_version() >= 100
+
+
+def test_sizes(L):
+    assert fq.num_scales(8192, 4096, fq.GROUP_1x128) == 32 * 8192
+    assert fq.num_scales(14336, 4096, fq.BLOCK_128x128) == 112 * 32
+    assert fq.num_scales(129, 257, fq.BLOCK_128x128) == 2 * 3
+    assert fq.num_scales(5, 5, fq.PER_TENSOR) == 1
+    assert fq.num_scales(-1, 5, fq.PER_TENSOR) == 0
+    assert fq.num_scales(5, 5, 7) == 0
+    assert fq.workspace_bytes(10, 16, fq.PER_TENSOR) > 0
+    assert fq.workspace_bytes(10, 16, fq.GROUP_1x128) == 0
+    assert fq.kv_num_scales(131072, 8, fq.KV_PER_HEAD_TOK128) == 1024 * 8
+    assert fq.kv_num_scales(131072, 8, fq.KV_PER_HEAD) == 8
+    assert fq.kv_num_scales(131072, 8, fq.KV_PER_TENSOR) == 1
+    assert fq.kv_workspace_bytes(131072, 8, 128, fq.KV_PER_HEAD_TOK128) == 0
+    assert fq.kv_workspace_bytes(131072, 8, 128, fq.KV_PER_HEAD) >= fq.kv_workspace_bytes(131072, 8, 128, fq.KV_PER_TENSOR)
+
+
+P = ctypes.c_void_p
+ALIGNED = P(1 << 20)          # never dereferenced: every call below fails validation first
+MISALIGNED = P((1 << 20) + 4)
+
+
+@pytest.mark.parametrize("args,status", [
+    ((ALIGNED, -1, 8, 0, 1, ALIGNED, ALIGNED, None, 0, None), 1),        # negative rows
+    ((ALIGNED, 4, 12, 0, 1, ALIGNED, ALIGNED, None, 0, None), 1),        # cols % 8
+    ((ALIGNED, 4, 8, 2, 1, ALIGNED, ALIGNED, None, 0, None), 1),         # bad format
+    ((ALIGNED, 4, 8, 0, 3, ALIGNED, ALIGNED, None, 0, None), 1),         # bad granularity
+    ((None, 4, 8, 0, 1, ALIGNED, ALIGNED, None, 0, None), 1),            # null input
+    ((MISALIGNED, 4, 8, 0, 1, ALIGNED, ALIGNED, None, 0, None), 1),      # misaligned input
+    ((ALIGNED, 4, 8, 0, 1, MISALIGNED, ALIGNED, None, 0, None), 1),      # misaligned codes
+    ((ALIGNED, 4, 8, 0, 1, ALIGNED, None, None, 0, None), 1),            # null scales
+    ((ALIGNED, 4, 8, 0, 0, ALIGNED, ALIGNED, None, 0, None), 3),         # per-tensor without workspace
+    ((ALIGNED, 4, 8, 0, 0, ALIGNED, ALIGNED, ALIGNED, 16, None), 3),     # workspace too small
+    ((ALIGNED, 1 << 40, 1 << 8, 0, 1, ALIGNED, ALIGNED, None, 0, None), 2),  # too large
+    ((None, 0, 8, 0, 1, None, None, None, 0, None), 0),                  # empty: nothing to do
+])
+def test_quantize_rejects(L, args, status):
+    assert L.fp8_quantize(*args) == status
+
+
+def test_dequantize_rejects(L):
+    assert L.fp8_dequantize(ALIGNED, ALIGNED, 4, 12, 0, 1, ALIGNED, None) == 1
+    assert L.fp8_dequantize(ALIGNED, None, 4, 8, 0, 1, ALIGNED, None) == 1
+    assert L.fp8_dequantize(ALIGNED, ALIGNED, 4, 8, 0, 1, MISALIGNED, None) == 1
+    assert L.fp8_dequantize(None, None, 0, 8, 0, 1, None, None) == 0
+
+
+def test_kv_rejects(L):
+    k = ALIGNED
+    assert L.fp8_kv_quantize(k, k, 16, 8, 12, 0, 1, k, k, k, k, k, 1 << 20, None) == 1        # head_dim % 8
+    assert L.fp8_kv_quantize(k, k, 16, 8, 128, 0, 5, k, k, k, k, k, 1 << 20, None) == 1       # bad granularity
+    assert L.fp8_kv_quantize(k, k, 16, 8, 128, 0, 1, k, k, k, k, None, 0, None) == 3          # no workspace
+    assert L.fp8_kv_quantize(k, k, 16, 8, 512, 0, 2, k, k, k, k, None, 0, None) == 2          # head_dim > 256
+    assert L.fp8_kv_quantize(k, None, 16, 8, 128, 0, 2, k, k, k, k, None, 0, None) == 1       # null v
+
+
+def test_gemm_rejects(L):
+    a = ALIGNED
+    assert L.fp8_gemm_blockscaled(a, a, 1, a, a, 2, 128, 100, 128, a, None, 0, None) == 2      # N % 128
+    assert L.fp8_gemm_blockscaled(a, a, 1, a, a, 2, 128, 128, 96, a, None, 0, None) == 2       # K % 128
+    assert L.fp8_gemm_blockscaled(a, a, 2, a, a, 2, 128, 128, 128, a, None, 0, None) == 1      # gA
+    assert L.fp8_gemm_blockscaled(a, a, 1, a, a, 1, 128, 128, 128, a, None, 0, None) == 1      # gB
+    assert L.fp8_gemm_blockscaled(MISALIGNED, a, 1, a, a, 2, 128, 128, 128, a, None, 0, None) == 1
+    assert L.fp8_gemm_blockscaled(a, a, 1, a, a, 2, 0, 128, 128, a, None, 0, None) == 0
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        fq.fp8_quantize(torch.zeros(4, 8, dtype=torch.bfloat16))
