@@ -403,6 +403,16 @@ def our_arm(args):
     x_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_x[:used])
     clocks = sampler.summary(wall0, wall1)
 
+    if args.skip_extras:
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+                              "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+                              "note": "profiling run: steps only", "kernels_us": [round(w_ms * 1e3, 2),
+                                                                                  round(x_ms * 1e3, 2)]}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+
     # end to end through the binding, pinned host buffers, copies inside the timed region
     hw = torch.from_numpy(w_np.view(np.int16)).view(torch.bfloat16).pin_memory()
     hx = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -486,6 +496,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-supplementary", action="store_true")
+    ap.add_argument("--skip-extras", action="store_true",
+                    help="time the steps only: no e2e, CPU baseline or supplementary kernels (for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

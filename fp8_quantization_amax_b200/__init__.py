@@ -18,7 +18,7 @@ import torch
 __all__ = [
     "E4M3", "E5M2", "PER_TENSOR", "GROUP_1x128", "BLOCK_128x128",
     "KV_PER_TENSOR", "KV_PER_HEAD", "KV_PER_HEAD_TOK128",
-    "Fp8qError", "lib", "library_path", "num_scales", "workspace_bytes", "kv_num_scales",
+    "Fp8qError", "lib", "library_path", "device_status", "num_scales", "workspace_bytes", "kv_num_scales",
     "kv_workspace_bytes", "gemm_workspace_bytes", "scale_shape", "kv_scale_shape",
     "fp8_encode", "fp8_decode", "fp8_quantize", "fp8_dequantize", "fp8_kv_quantize",
     "fp8_gemm_blockscaled",
@@ -57,6 +57,7 @@ def lib() -> ctypes.CDLL:
             L.fp8q_status_string.argtypes = [i32]
             L.fp8q_status_string.restype = ctypes.c_char_p
             L.fp8q_version.restype = i32
+            L.fp8q_device_status.restype = ctypes.c_uint32
             L.fp8q_num_scales.argtypes = [i64, i64, i32]
             L.fp8q_num_scales.restype = sz
             L.fp8q_workspace_bytes.argtypes = [i64, i64, i32]
@@ -78,6 +79,11 @@ def lib() -> ctypes.CDLL:
                 getattr(L, fn).restype = i32
             _lib = L
     return _lib
+
+
+def device_status() -> int:
+    """Synchronize the device; return and clear the kernels' error bits (0 = none)."""
+    return int(lib().fp8q_device_status())
 
 
 def _status_string(status: int) -> str:

@@ -46,6 +46,8 @@ const char* fp8q_status_string(fp8q_status status) {
 
 int fp8q_version(void) { return 100; }
 
+uint32_t fp8q_device_status(void) { return fp8q::read_and_clear_device_error(); }
+
 size_t fp8q_num_scales(int64_t rows, int64_t cols, fp8q_granularity g) {
   if (rows < 0 || cols < 0 || !valid_gran(g)) return 0;
   if (g == FP8Q_PER_TENSOR) return 1;
@@ -133,7 +135,7 @@ fp8q_status fp8_kv_quantize(const void* k, const void* v, int64_t tokens, int64_
   const int64_t n = row < 0 ? -1 : checked_elems(tokens, row);
   if (n < 0) return FP8Q_ERR_UNSUPPORTED;
   if (g == FP8Q_KV_PER_HEAD_TOK128 && head_dim > 256) return FP8Q_ERR_UNSUPPORTED;
-  if (g == FP8Q_KV_PER_HEAD && heads > 128) return FP8Q_ERR_UNSUPPORTED;
+  if (g == FP8Q_KV_PER_HEAD && (heads > 128 || head_dim > 256)) return FP8Q_ERR_UNSUPPORTED;
   const size_t nsc = fp8q_kv_num_scales(tokens, heads, g);
   if (n > 0 && (!k || !v || !k_codes || !v_codes || !aligned(k, 16) || !aligned(v, 16) || !aligned(k_codes, 16) ||
                 !aligned(v_codes, 16)))

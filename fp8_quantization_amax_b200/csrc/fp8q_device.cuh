@@ -26,7 +26,7 @@ struct Fmt<kE5M2> {
   static constexpr float kMax = 57344.0f;
 };
 
-// ---------------------------------------------------------------- memory
+// ---------------------------------------------------------------- global memory
 
 __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
   uint4 v;
@@ -54,73 +54,74 @@ __device__ __forceinline__ void st_stream_v4(void* p, uint4 v) {
 
 // ---------------------------------------------------------------- amax on packed bf16
 //
-// |x| of a bf16 is its bit pattern with the sign cleared; for non-negative bf16 values the
-// unsigned integer order of the 16-bit patterns is the numeric order, with Inf above every
-// finite value and every NaN above Inf.  So a packed unsigned 16x2 max of the sign-cleared
-// words is an exact amax in which any NaN dominates.
+// max.NaN.xorsign.abs.bf16x2 keeps the larger magnitude of each half (the result's sign is the
+// xor of the inputs' signs, which never matters: every use takes magnitudes again) and
+// propagates NaN.  bf16 comparison is exact, so the group amax is exact and order-free.
 
-__device__ __forceinline__ uint32_t umax16x2(uint32_t a, uint32_t b) {
+__device__ __forceinline__ uint32_t absmax2(uint32_t a, uint32_t b) {
   uint32_t d;
-  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
   return d;
 }
 
 __device__ __forceinline__ uint32_t absmax_v4(uint32_t m, uint4 v) {
-  m = umax16x2(m, v.x & 0x7FFF7FFFu);
-  m = umax16x2(m, v.y & 0x7FFF7FFFu);
-  m = umax16x2(m, v.z & 0x7FFF7FFFu);
-  m = umax16x2(m, v.w & 0x7FFF7FFFu);
-  return m;
+  return absmax2(absmax2(m, v.x), absmax2(absmax2(v.y, v.z), v.w));
 }
 
-// packed pair max -> fp32 amax
+// packed pair -> fp32 amax of the two halves (any NaN gives NaN)
 __device__ __forceinline__ float packed_amax_to_f32(uint32_t m) {
-  uint32_t lo = m & 0xFFFFu, hi = m >> 16;
-  return __uint_as_float((lo > hi ? lo : hi) << 16);
+  const uint32_t r = absmax2(m, m >> 16) & 0x7FFFu;
+  return __uint_as_float(r << 16);
 }
 
 // ---------------------------------------------------------------- scale and quotient
 //
-// The scale is s = amax / FMAX (one IEEE division) and every element's quotient must be the
-// IEEE round-to-nearest fp32 value of x / s.  A per-element division is too slow for an HBM
-// bound kernel, so groups whose scale is a comfortably normal number use the reciprocal
-// r = RN(1/s) once per group and Markstein's correction per element:
-//   q0 = RN(x * r);  e = x - q0 * s (exact, one FMA);  q = RN(q0 + e * r)
-// (P. Markstein, "Computation of elementary functions on the IBM RISC System/6000
-// processor", IBM J. Res. Dev. 34(1), 1990), which yields RN(x / s) when r is the correctly
-// rounded reciprocal and nothing underflows.  The sign of a zero quotient is restored from x
-// (the correction adds +0 to -0).  Groups with tiny, zero, infinite or NaN scales fall back
-// to the IEEE division per element; an all-zero group keeps the sign of each zero.
-// Exactness of the fast path is verified exhaustively over every (bf16 x, bf16 amax) pair
-// by the GPU parity tests.
+// Every element's quotient must be the IEEE round-to-nearest fp32 value of x / s.  A division
+// per element is far too slow for an HBM-bound kernel, so groups whose amax is an ordinary
+// normal number use Markstein's correction (P. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990): with
+// r = RN(1/d) and q0 = RN(x * r), the residual e = x - q0 * d is exact in one FMA and
+// RN(q0 + e * r) = RN(x / d) when nothing overflows or underflows.  The same step with the
+// constant RN(1/FMAX) gives the scale s = RN(amax / FMAX).  Groups with a tiny, infinite or
+// NaN amax take IEEE divisions instead.  An all-zero group has s = 0 and divides by 1 (every x
+// is +-0).  The Markstein step maps x = -0 to +0, so the inputs' sign bits are OR-ed back into
+// the codes.  The fast path is checked against the oracle for every (bf16 x, bf16 amax) pair.
 
 struct GroupScale {
   float s;     // stored scale
-  float sd;    // divisor used for the quotient
-  float r;     // RN(1 / sd) for the fast path
-  bool fast;   // Markstein path valid for this group
+  float d;     // divisor used for the quotients
+  float r;     // RN(1 / d) (fast path)
+  bool fast;
 };
+
+__device__ __forceinline__ float markstein_div(float x, float d, float r) {
+  const float q0 = __fmul_rn(x, r);
+  const float e = __fmaf_rn(-q0, d, x);
+  return __fmaf_rn(e, r, q0);
+}
 
 template <int FMT>
 __device__ __forceinline__ GroupScale make_group_scale(float amax) {
+  constexpr float kMax = Fmt<FMT>::kMax;
+  constexpr float kInvMax = 1.0f / Fmt<FMT>::kMax;            // RN(1 / FMAX)
   GroupScale g;
-  g.s = __fdiv_rn(amax, Fmt<FMT>::kMax);
-  // fast path: s in [2^-80, FLT_MAX]; s == 0 (all-zero group) uses divisor 1: q = x exactly
-  const bool normal_s = g.s >= 0x1.0p-80f && g.s <= 3.4028234663852886e38f;
-  g.sd = (g.s == 0.0f) ? 1.0f : g.s;
-  g.fast = normal_s || g.s == 0.0f;
-  g.r = g.fast ? __frcp_rn(g.sd) : 0.0f;
-  return g;
-}
-
-__device__ __forceinline__ float quotient(float x, const GroupScale& g) {
-  if (g.fast) {
-    float q0 = __fmul_rn(x, g.r);
-    float e = __fmaf_rn(-q0, g.sd, x);
-    float q = __fmaf_rn(e, g.r, q0);
-    return __uint_as_float((__float_as_uint(q) & 0x7FFFFFFFu) | (__float_as_uint(x) & 0x80000000u));
+  if (amax >= 0x1.0p-60f && amax <= 3.4028234663852886e38f) {
+    g.s = markstein_div(amax, kMax, kInvMax);
+    g.d = g.s;
+    g.r = __frcp_rn(g.s);
+    g.fast = true;
+  } else if (amax == 0.0f) {
+    g.s = 0.0f;
+    g.d = 1.0f;
+    g.r = 1.0f;
+    g.fast = true;
+  } else {
+    g.s = __fdiv_rn(amax, kMax);
+    g.d = g.s;
+    g.r = 0.0f;
+    g.fast = false;
   }
-  return __fdiv_rn(x, g.sd);
+  return g;
 }
 
 // ---------------------------------------------------------------- FP8 conversions
@@ -172,18 +173,42 @@ __device__ __forceinline__ uint32_t f32x2_to_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// quantize four bf16 (two words) into four codes packed in a 32-bit word
-template <int FMT>
-__device__ __forceinline__ uint32_t quant4(uint32_t w0, uint32_t w1, const GroupScale& g) {
-  uint32_t a = cvt2<FMT>(quotient(bf16_lo(w0), g), quotient(bf16_hi(w0), g));
-  uint32_t b = cvt2<FMT>(quotient(bf16_lo(w1), g), quotient(bf16_hi(w1), g));
-  return a | (b << 16);
+// sign bits of four bf16 (two words) placed on bit 7 of four code bytes
+__device__ __forceinline__ uint32_t signs4(uint32_t w0, uint32_t w1) {
+  return __byte_perm(w0, w1, 0x7531) & 0x80808080u;
 }
 
-// quantize eight bf16 (16 bytes) into eight codes (8 bytes)
+// four bf16 (two words) -> four codes, fast path
+template <int FMT>
+__device__ __forceinline__ uint32_t quant4_fast(uint32_t w0, uint32_t w1, float d, float r) {
+  const uint32_t a = cvt2<FMT>(markstein_div(bf16_lo(w0), d, r), markstein_div(bf16_hi(w0), d, r));
+  const uint32_t b = cvt2<FMT>(markstein_div(bf16_lo(w1), d, r), markstein_div(bf16_hi(w1), d, r));
+  return __byte_perm(a, b, 0x5410) | signs4(w0, w1);
+}
+
+// eight bf16 (16 bytes) -> eight codes (8 bytes), fast path
+template <int FMT>
+__device__ __forceinline__ uint2 quant8_fast(uint4 v, float d, float r) {
+  return make_uint2(quant4_fast<FMT>(v.x, v.y, d, r), quant4_fast<FMT>(v.z, v.w, d, r));
+}
+
+// eight bf16 -> eight codes with IEEE divisions (groups with tiny, infinite or NaN amax)
+template <int FMT>
+__device__ __noinline__ uint2 quant8_slow(uint4 v, float d) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t c[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const uint32_t a = cvt2<FMT>(__fdiv_rn(bf16_lo(w[2 * i]), d), __fdiv_rn(bf16_hi(w[2 * i]), d));
+    const uint32_t b = cvt2<FMT>(__fdiv_rn(bf16_lo(w[2 * i + 1]), d), __fdiv_rn(bf16_hi(w[2 * i + 1]), d));
+    c[i] = __byte_perm(a, b, 0x5410) | signs4(w[2 * i], w[2 * i + 1]);
+  }
+  return make_uint2(c[0], c[1]);
+}
+
 template <int FMT>
 __device__ __forceinline__ uint2 quant8(uint4 v, const GroupScale& g) {
-  return make_uint2(quant4<FMT>(v.x, v.y, g), quant4<FMT>(v.z, v.w, g));
+  return g.fast ? quant8_fast<FMT>(v, g.d, g.r) : quant8_slow<FMT>(v, g.d);
 }
 
 }  // namespace fp8q

@@ -2,12 +2,23 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace fp8q {
 
 // number of SMs of the current device (queried once per device)
 int device_sm_count();
+
+// device address of the library's error word on the current device (kernels set bits in it
+// when a bounded wait gives up); read_and_clear_device_error() synchronizes the device first
+uint32_t* device_error_word();
+uint32_t read_and_clear_device_error();
+
+// 2-D TMA descriptor for a row-major [outer][inner] tensor of 1-, 2- or 4-byte elements with the
+// given row stride; box = box_outer rows x box_inner elements
+bool make_tmap_2d(CUtensorMap* map, int elem_bytes, const void* base, uint64_t inner, uint64_t outer,
+                  uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, int swizzle_128b);
 
 // largest number of first-pass partial maxima any two-pass launch writes, per scale group
 constexpr int kMaxPartials = 1024;

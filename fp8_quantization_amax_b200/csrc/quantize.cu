@@ -8,16 +8,22 @@
 // per head x 128 tokens); api.makesence.top "LLM推理量化:FP8 versus INT8", section 二 (E5M2
 // KV cache).
 //
-// All kernels are HBM-bound streams: 16-byte loads that bypass L1, group reductions in
-// registers and warp shuffles, and the cast done on the registers already loaded, so a
-// one-pass granularity reads each element once.
+// Structure (all kernels): a persistent CTA of nine warps.  Warp 8 is the producer: one lane
+// streams 2-D TMA boxes of the bf16 input into a ring of shared-memory stages (mbarrier
+// full/empty pipeline).  Warps 0-7 consume: each thread reads its 16-byte pieces of a stage,
+// frees the stage, reduces the group amax (warp shuffles, plus a named barrier when a group
+// spans the whole box), computes the scale and writes the FP8 codes straight to global memory.
+// Loads stay in flight several stages ahead regardless of the consumers' progress.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
 #include <cstdint>
+#include <cstring>
 
 #include "fp8q_device.cuh"
 #include "internal.h"
+#include "sm100.cuh"
 
 namespace fp8q {
 
@@ -47,334 +53,504 @@ __device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
   return (uint32_t)(((uint64_t)__umulhi(n, f.m) + n) >> f.s);
 }
 
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumers = 32 * kConsumerWarps;
+constexpr int kThreads = kConsumers + 32;          // + the producer warp
+constexpr int kMaxStages = 8;
+constexpr uint32_t kStageBudget = 96 * 1024;        // ring bytes per CTA (two CTAs per SM)
+
+// Producer side of the ring: issue TMA box loads for this CTA's items in `item_at(k)` order,
+// each into the next stage once the consumers have freed it; finally wait until every issued
+// copy has landed (they have, unless the consumers gave up), so no copy outlives the CTA.
+template <class ItemFn, class IssueFn>
+__device__ __forceinline__ void run_producer(uint64_t* full, uint64_t* empty, int S, uint32_t nk, uint32_t bytes,
+                                             uint32_t* err, ItemFn item_at, IssueFn issue) {
+  int s = 0;
+  uint32_t ph = 0, k = 0;
+  for (; k < nk; ++k) {
+    if (k >= (uint32_t)S && !mbar_wait(&empty[s], ph ^ 1u, err)) break;
+    mbar_arrive_expect_tx(&full[s], bytes);
+    issue(item_at(k), s, &full[s]);
+    if (++s == S) {
+      s = 0;
+      ph ^= 1u;
+    }
+  }
+  const uint32_t last = k;
+  for (uint32_t j = 0; j < (uint32_t)S && j < last; ++j) {
+    const uint32_t kk = last - 1 - j;
+    mbar_wait(&full[kk % S], (kk / S) & 1u, err);
+  }
+}
+
+// number of items of this CTA under a grid-stride assignment
+__device__ __forceinline__ uint32_t items_of_cta(uint32_t nitems) {
+  return nitems > blockIdx.x ? (nitems - blockIdx.x + gridDim.x - 1) / gridDim.x : 0u;
+}
+
+static uint32_t ring_stages(uint32_t stage_bytes) {
+  return std::max<uint32_t>(2, std::min<uint32_t>(kMaxStages, kStageBudget / stage_bytes));
+}
+
+static size_t ring_smem(uint32_t stages, uint32_t stage_bytes) {
+  return 1024 + (size_t)stages * stage_bytes + 2 * kMaxStages * sizeof(uint64_t);   // + alignment slack
+}
+
+// dynamic shared memory starts after the static arrays; TMA boxes land on 1024-byte boundaries
+__device__ __forceinline__ uint8_t* ring_base(uint8_t* raw) {
+  const uint32_t a = smem_u32(raw);
+  return raw + (((a + 1023u) & ~1023u) - a);
+}
+
+template <class K>
+static int grid_for(K kernel, size_t smem, uint32_t nitems) {
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kThreads, smem) != cudaSuccess || occ <= 0)
+    occ = 1;
+  return (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)nitems, (int64_t)device_sm_count() * occ));
+}
+
 // ============================================================================ 1 x 128 groups
 //
-// A warp quantizes four groups at a time: rows 4q .. 4q+3 of one 128-column group.  Eight
-// lanes own one group, each lane 16 elements in two 16-byte pieces 64 columns apart, so each
-// load instruction reads four fully used 128-byte lines.  The group amax is reduced across
-// the eight lanes with three xor-shuffles.  The scales of consecutive rows of one group are
-// contiguous in memory, so the four scales of a warp form one 16-byte run.
+// Box = 64 rows x 128 columns (16 KB): 64 groups.  Four consecutive threads own one group
+// (32 elements each, four 16-byte pieces), reduce it with two xor-shuffles, and store 32 codes.
+// The 64 scales of a box are 64 consecutive rows of one group column: one 256-byte run.
 
-template <int FMT, int UNROLL>
-__global__ void __launch_bounds__(256) k_quant_1x128(const uint16_t* __restrict__ x, uint8_t* __restrict__ codes,
-                                                     float* __restrict__ scales, int64_t rows, int64_t cols,
-                                                     uint32_t nrq, uint32_t units) {
-  const uint32_t lane = threadIdx.x & 31u, sub = lane >> 3, l8 = lane & 7u;
-  const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
-  for (uint32_t u0 = warp; u0 < units; u0 += nwarps * UNROLL) {
-    uint4 a[UNROLL], b[UNROLL];
-    int64_t row[UNROLL], col[UNROLL];
-    bool rv[UNROLL], v0[UNROLL], v1[UNROLL];
-#pragma unroll
-    for (int j = 0; j < UNROLL; ++j) {
-      const uint32_t u = u0 + j * nwarps;
-      const bool live = u < units;                     // warp-uniform
-      const uint32_t g = live ? u / nrq : 0u;
-      const uint32_t rq = live ? u - g * nrq : 0u;
-      row[j] = (int64_t)rq * 4 + sub;
-      col[j] = (int64_t)g * 128 + l8 * 8;
-      rv[j] = live && row[j] < rows;
-      v0[j] = rv[j] && col[j] < cols;
-      v1[j] = rv[j] && col[j] + 64 < cols;
-      const uint16_t* p = x + row[j] * cols + col[j];
-      a[j] = v0[j] ? ld_stream_v4(p) : make_uint4(0u, 0u, 0u, 0u);
-      b[j] = v1[j] ? ld_stream_v4(p + 64) : make_uint4(0u, 0u, 0u, 0u);
+constexpr uint32_t kGroupBoxRows = 64;
+constexpr uint32_t kGroupStage = kGroupBoxRows * 128 * 2;
+
+struct GroupParams {
+  uint8_t* codes;
+  float* scales;
+  int64_t rows, cols;
+  uint32_t nitems;
+  FastDiv ngc;        // 128-column groups per row
+  int stages;
+  int wide_stores;    // cols % 32 == 0: 16-byte code stores
+  uint32_t* err;
+};
+
+template <int FMT>
+__global__ void __launch_bounds__(kThreads, 2) k_group128(const __grid_constant__ CUtensorMap tx, GroupParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = ring_base(smem_raw);
+  const int S = p.stages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * kGroupStage);
+  uint64_t* empty = full + kMaxStages;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
     }
-#pragma unroll
-    for (int j = 0; j < UNROLL; ++j) {
-      uint32_t m = absmax_v4(absmax_v4(0u, a[j]), b[j]);
-      m = umax16x2(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-      m = umax16x2(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-      m = umax16x2(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
-      const GroupScale gs = make_group_scale<FMT>(packed_amax_to_f32(m));
-      uint8_t* cp = codes + row[j] * cols + col[j];
-      if (v0[j]) st_stream_v2(cp, quant8<FMT>(a[j], gs));
-      if (v1[j]) st_stream_v2(cp + 64, quant8<FMT>(b[j], gs));
-      if (l8 == 0 && rv[j]) scales[(col[j] >> 7) * rows + row[j]] = gs.s;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const uint32_t nk = items_of_cta(p.nitems);
+  if (warp == kConsumerWarps) {
+    if (lane == 0 && nk > 0) {
+      tma_prefetch_desc(&tx);
+      run_producer(
+          full, empty, S, nk, kGroupStage, p.err, [&](uint32_t k) { return blockIdx.x + k * gridDim.x; },
+          [&](uint32_t i, int s, uint64_t* bar) {
+            const uint32_t rb = fdiv(i, p.ngc), g = i - rb * p.ngc.d;
+            tma_load_2d(smem + s * kGroupStage, &tx, (int32_t)(g * 128), (int32_t)(rb * kGroupBoxRows), bar);
+          });
     }
+    return;
+  }
+  const int t = threadIdx.x, grp = t >> 2, q = t & 3;
+  int s = 0;
+  uint32_t ph = 0;
+  for (uint32_t k = 0; k < nk; ++k) {
+    const uint32_t i = blockIdx.x + k * gridDim.x;
+    if (!mbar_wait(&full[s], ph, p.err)) break;
+    const uint8_t* src = smem + s * kGroupStage + grp * 256 + q * 64;
+    const uint4 v0 = ld_shared_v4(src), v1 = ld_shared_v4(src + 16), v2 = ld_shared_v4(src + 32),
+                v3 = ld_shared_v4(src + 48);
+    uint32_t m = absmax_v4(absmax_v4(absmax_v4(absmax_v4(0u, v0), v1), v2), v3);   // consumes every load
+    release_stage(&empty[s], lane);
+    if (++s == S) {
+      s = 0;
+      ph ^= 1u;
+    }
+    m = absmax2(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+    m = absmax2(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+    const GroupScale gs = make_group_scale<FMT>(packed_amax_to_f32(m));
+    const uint32_t rb = fdiv(i, p.ngc), g = i - rb * p.ngc.d;
+    const int64_t row = (int64_t)rb * kGroupBoxRows + grp;
+    const int64_t col = (int64_t)g * 128 + q * 32;
+    if (row >= p.rows) continue;
+    uint2 c0, c1, c2, c3;
+    if (gs.fast) {
+      c0 = quant8_fast<FMT>(v0, gs.d, gs.r);
+      c1 = quant8_fast<FMT>(v1, gs.d, gs.r);
+      c2 = quant8_fast<FMT>(v2, gs.d, gs.r);
+      c3 = quant8_fast<FMT>(v3, gs.d, gs.r);
+    } else {
+      c0 = quant8_slow<FMT>(v0, gs.d);
+      c1 = quant8_slow<FMT>(v1, gs.d);
+      c2 = quant8_slow<FMT>(v2, gs.d);
+      c3 = quant8_slow<FMT>(v3, gs.d);
+    }
+    uint8_t* dst = p.codes + row * p.cols + col;
+    if (p.wide_stores && col + 32 <= p.cols) {
+      st_stream_v4(dst, make_uint4(c0.x, c0.y, c1.x, c1.y));
+      st_stream_v4(dst + 16, make_uint4(c2.x, c2.y, c3.x, c3.y));
+    } else {
+      if (col < p.cols) st_stream_v2(dst, c0);
+      if (col + 8 < p.cols) st_stream_v2(dst + 8, c1);
+      if (col + 16 < p.cols) st_stream_v2(dst + 16, c2);
+      if (col + 24 < p.cols) st_stream_v2(dst + 24, c3);
+    }
+    if (q == 0) p.scales[(int64_t)g * p.rows + row] = gs.s;
   }
 }
 
 template <int FMT>
-static cudaError_t launch_1x128_fmt(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* codes, float* scales,
-                                    cudaStream_t st) {
-  const int64_t ngc = (cols + 127) / 128, nrq = (rows + 3) / 4;
-  const int64_t units = ngc * nrq;
-  if (units == 0) return cudaSuccess;
-  constexpr int kUnroll = 2;
-  static int occ = 0;
-  if (occ == 0) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_quant_1x128<FMT, kUnroll>, 256, 0) != cudaSuccess ||
-        occ <= 0)
-      occ = 4;
+static cudaError_t launch_group128_fmt(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* codes,
+                                       float* scales, cudaStream_t st) {
+  const int64_t ngc = (cols + 127) / 128, nrb = (rows + kGroupBoxRows - 1) / kGroupBoxRows;
+  const int64_t nitems = ngc * nrb;
+  if (nitems == 0) return cudaSuccess;
+  CUtensorMap map;
+  std::memset(&map, 0, sizeof(map));
+  if (!make_tmap_2d(&map, 2, x, (uint64_t)cols, (uint64_t)rows, (uint64_t)cols * 2, 128, kGroupBoxRows, 0))
+    return cudaErrorInvalidValue;
+  GroupParams p;
+  p.codes = codes;
+  p.scales = scales;
+  p.rows = rows;
+  p.cols = cols;
+  p.nitems = (uint32_t)nitems;
+  p.ngc = make_fastdiv((uint32_t)ngc);
+  p.stages = (int)ring_stages(kGroupStage);
+  p.wide_stores = cols % 32 == 0;
+  p.err = device_error_word();
+  const size_t smem = ring_smem(p.stages, kGroupStage);
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(k_group128<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    attr = true;
   }
-  const int64_t need = (units + 8 * kUnroll - 1) / (8 * kUnroll);   // 8 warps per block
-  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(need, (int64_t)device_sm_count() * occ));
-  k_quant_1x128<FMT, kUnroll><<<grid, 256, 0, st>>>(x, codes, scales, rows, cols, (uint32_t)nrq, (uint32_t)units);
+  const int grid = grid_for(k_group128<FMT>, smem, p.nitems);
+  k_group128<FMT><<<grid, kThreads, smem, st>>>(map, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_quant_1x128(const uint16_t* x, int64_t rows, int64_t cols, int fmt, uint8_t* codes,
                                float* scales, cudaStream_t st) {
-  return fmt == kE4M3 ? launch_1x128_fmt<kE4M3>(x, rows, cols, codes, scales, st)
-                      : launch_1x128_fmt<kE5M2>(x, rows, cols, codes, scales, st);
+  return fmt == kE4M3 ? launch_group128_fmt<kE4M3>(x, rows, cols, codes, scales, st)
+                      : launch_group128_fmt<kE5M2>(x, rows, cols, codes, scales, st);
 }
 
 // ============================================================================ 128-row tiles
 //
-// One CTA of 256 threads quantizes one tile of 128 rows x gw columns: 128 x 128 weight
-// blocks (gw = 128, row stride = cols) and 128-token x head_dim KV blocks (gw = head_dim,
-// row stride = heads * head_dim).  The whole tile (32 KB for 128 x 128) sits in registers,
-// eight 16-byte pieces per thread, so the amax and the cast see each element exactly once.
-// A warp loads two 256-byte row segments per instruction.  The CTA loops over tiles; several
-// CTAs per SM keep loads of one tile in flight while another reduces and stores.
+// Box = 128 rows x bc columns of a [rows][ld] bf16 matrix (bc = 128 for weight blocks and
+// per-tensor passes, bc = head_dim for the KV cache).  Thread t owns the 16-byte pieces
+// t, t + 256, ... of the box (a warp reads 512 contiguous bytes of shared memory).
+//   kOnePass: the box is one scale group (128x128 weight block, 128-token x head KV block):
+//             amax over the CTA (shuffles + named barrier), scale, cast, store.
+//   kAmax:    pass 1 of per-tensor / per-head: fold the box amax into this CTA's running
+//             maximum for the box's group; write them out at the end.
+//   kCast:    pass 2: fold all CTAs' partial maxima into the group scales, then cast every
+//             box, walking the boxes in the reverse of pass 1's order so the boxes pass 1
+//             read last, the likeliest to still be in L2, come first.
 
-template <int FMT, int CPR_T, int MAXC>
-__global__ void __launch_bounds__(256) k_quant_tiles(const uint16_t* __restrict__ x0, const uint16_t* __restrict__ x1,
-                                                     uint8_t* __restrict__ c0, uint8_t* __restrict__ c1,
-                                                     float* __restrict__ s0, float* __restrict__ s1, int64_t rows,
-                                                     int64_t cols, int64_t ld, int gw, int nbr, int nbc,
-                                                     int ntiles) {
-  __shared__ uint32_t red[8];
-  const int cpr = CPR_T > 0 ? CPR_T : gw / 8;   // 16-byte pieces per tile row
-  const int nchunks = 128 * cpr;
-  const int per_tensor = nbr * nbc;
-  for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
-    const int tens = t / per_tensor;
-    const int rem = t - tens * per_tensor;
-    const int bi = rem / nbc, bj = rem - bi * nbc;
-    const uint16_t* x = tens ? x1 : x0;
-    uint8_t* c = tens ? c1 : c0;
-    uint4 v[MAXC];
-    int64_t off[MAXC];
-    bool ok[MAXC];
-    uint32_t m = 0;
-#pragma unroll
-    for (int k = 0; k < MAXC; ++k) {
-      const int i = threadIdx.x + 256 * k;
-      const int r = i / cpr, cc = i - r * cpr;
-      const int64_t row = (int64_t)bi * 128 + r;
-      const int64_t col = (int64_t)bj * gw + cc * 8;
-      ok[k] = i < nchunks && row < rows && col < cols && cc * 8 < gw;
-      off[k] = row * ld + col;
-      v[k] = ok[k] ? ld_stream_v4(x + off[k]) : make_uint4(0u, 0u, 0u, 0u);
-      m = absmax_v4(m, v[k]);
+constexpr int kOnePass = 0;
+constexpr int kAmax = 1;
+constexpr int kCast = 2;
+constexpr int kMaxGroups = 256;
+
+struct TileParams {
+  uint8_t* c0;
+  uint8_t* c1;
+  float* s0;
+  float* s1;
+  float* partials;       // kAmax: written [grid][ngroups]; kCast: read [nparts][ngroups]
+  int nparts;
+  int64_t rows, cols, ld;
+  int bc, cpr;           // box columns, 16-byte pieces per box row
+  FastDiv nbc;           // boxes across
+  FastDiv per_tensor;    // boxes per tensor
+  uint32_t nitems;
+  int head_groups;       // kAmax / kCast: the group follows the box column (one per head)
+  int heads;             // groups per tensor
+  int ngroups;
+  int stages;
+  uint32_t stage_bytes;
+  uint32_t* err;
+};
+
+struct TileItem {
+  uint32_t tens, bi, bj;
+};
+
+__device__ __forceinline__ TileItem tile_item(uint32_t i, const TileParams& p) {
+  TileItem it;
+  it.tens = fdiv(i, p.per_tensor);
+  const uint32_t rem = i - it.tens * p.per_tensor.d;
+  it.bi = fdiv(rem, p.nbc);
+  it.bj = rem - it.bi * p.nbc.d;
+  return it;
+}
+
+template <int MODE>
+__device__ __forceinline__ uint32_t tile_item_index(uint32_t k, uint32_t nitems) {
+  const uint32_t fwd = blockIdx.x + k * gridDim.x;
+  return MODE == kCast ? nitems - 1 - fwd : fwd;
+}
+
+template <int FMT, int MODE, int CPR, int MAXC>
+__global__ void __launch_bounds__(kThreads, 2) k_tile128(const __grid_constant__ CUtensorMap t0,
+                                                          const __grid_constant__ CUtensorMap t1, TileParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = ring_base(smem_raw);
+  __shared__ uint32_t red[2][kConsumerWarps];
+  __shared__ uint32_t wmax[MODE == kAmax ? kConsumerWarps : 1][MODE == kAmax ? kMaxGroups : 1];
+  __shared__ uint32_t fold[MODE == kCast ? kMaxGroups : 1];
+  __shared__ GroupScale table[MODE == kCast ? kMaxGroups : 1];
+  const int S = p.stages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * p.stage_bytes);
+  uint64_t* empty = full + kMaxStages;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
     }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const uint32_t nk = items_of_cta(p.nitems);
+  if (warp == kConsumerWarps) {
+    if (lane == 0 && nk > 0) {
+      tma_prefetch_desc(&t0);
+      tma_prefetch_desc(&t1);
+      run_producer(
+          full, empty, S, nk, p.stage_bytes, p.err, [&](uint32_t k) { return tile_item_index<MODE>(k, p.nitems); },
+          [&](uint32_t i, int s, uint64_t* bar) {
+            const TileItem it = tile_item(i, p);
+            tma_load_2d(smem + s * p.stage_bytes, it.tens ? &t1 : &t0, (int32_t)(it.bj * p.bc),
+                        (int32_t)(it.bi * 128), bar);
+          });
+    }
+    return;
+  }
+  const int t = threadIdx.x;
+  const int cpr = CPR > 0 ? CPR : p.cpr;
+  const int nchunks = 128 * cpr;
+
+  if (MODE == kAmax) {
+    for (int g = lane; g < kMaxGroups; g += 32) wmax[warp][g] = 0u;
+  }
+  if (MODE == kCast) {
+    // fold the partial maxima: non-negative floats (or NaN) order like their bit patterns
+    for (int g = t; g < p.ngroups; g += kConsumers) fold[g] = 0u;
+    named_barrier(1, kConsumers);
+    const int nitems_p = p.nparts * p.ngroups;
+    for (int it = t; it < nitems_p; it += kConsumers)
+      atomicMax(&fold[it % p.ngroups], __float_as_uint(p.partials[it]));
+    named_barrier(1, kConsumers);
+    for (int g = t; g < p.ngroups; g += kConsumers) {
+      table[g] = make_group_scale<FMT>(__uint_as_float(fold[g]));
+      if (blockIdx.x == 0) {
+        const int tens = g / p.heads;
+        (tens ? p.s1 : p.s0)[g - tens * p.heads] = table[g].s;
+      }
+    }
+    named_barrier(1, kConsumers);
+  }
+
+  int s = 0;
+  uint32_t ph = 0;
+  for (uint32_t k = 0; k < nk; ++k) {
+    const uint32_t i = tile_item_index<MODE>(k, p.nitems);
+    if (!mbar_wait(&full[s], ph, p.err)) break;
+    const uint8_t* stage = smem + s * p.stage_bytes;
+    uint4 v[MAXC];
+    uint32_t m = 0u;
 #pragma unroll
-    for (int d = 16; d >= 1; d >>= 1) m = umax16x2(m, __shfl_xor_sync(0xFFFFFFFFu, m, d));
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
-    __syncthreads();
-    uint32_t mm = red[0];
+    for (int j = 0; j < MAXC; ++j) {
+      const int c = t + kConsumers * j;
+      v[j] = (CPR > 0 || c < nchunks) ? ld_shared_v4(stage + c * 16) : make_uint4(0u, 0u, 0u, 0u);
+      if (MODE != kCast) m = absmax_v4(m, v[j]);
+    }
+    // the amax consumed every load; the cast pass releases the stage after the cast instead
+    uint64_t* release = &empty[s];
+    if (MODE != kCast) release_stage(release, lane);
+    if (++s == S) {
+      s = 0;
+      ph ^= 1u;
+    }
+    const TileItem it = tile_item(i, p);
+    if (MODE != kCast) {
 #pragma unroll
-    for (int w = 1; w < 8; ++w) mm = umax16x2(mm, red[w]);
-    const GroupScale gs = make_group_scale<FMT>(packed_amax_to_f32(mm));
-    if (threadIdx.x == 0) (tens ? s1 : s0)[bi * nbc + bj] = gs.s;
+      for (int d = 16; d >= 1; d >>= 1) m = absmax2(m, __shfl_xor_sync(0xFFFFFFFFu, m, d));
+    }
+    if (MODE == kAmax) {
+      if (lane == 0) {
+        const int g = (int)it.tens * p.heads + (p.head_groups ? (int)it.bj : 0);
+        const uint32_t a = __float_as_uint(packed_amax_to_f32(m));
+        wmax[warp][g] = max(wmax[warp][g], a);
+      }
+      continue;
+    }
+    GroupScale gs;
+    if (MODE == kOnePass) {
+      if (lane == 0) red[k & 1][warp] = m;
+      named_barrier(1, kConsumers);
+      uint32_t mm = red[k & 1][0];
 #pragma unroll
-    for (int k = 0; k < MAXC; ++k)
-      if (ok[k]) st_stream_v2(c + off[k], quant8<FMT>(v[k], gs));
-    __syncthreads();   // red[] is rewritten by the next tile
+      for (int w = 1; w < kConsumerWarps; ++w) mm = absmax2(mm, red[k & 1][w]);
+      gs = make_group_scale<FMT>(packed_amax_to_f32(mm));
+      if (t == 0) (it.tens ? p.s1 : p.s0)[it.bi * p.nbc.d + it.bj] = gs.s;
+    } else {
+      gs = table[(int)it.tens * p.heads + (p.head_groups ? (int)it.bj : 0)];
+    }
+    uint8_t* codes = it.tens ? p.c1 : p.c0;
+#pragma unroll
+    for (int j = 0; j < MAXC; ++j) {
+      const int c = t + kConsumers * j;
+      const int r = c / cpr, cc = c - r * cpr;
+      const int64_t row = (int64_t)it.bi * 128 + r;
+      const int64_t col = (int64_t)it.bj * p.bc + cc * 8;
+      const uint2 q = gs.fast ? quant8_fast<FMT>(v[j], gs.d, gs.r) : quant8_slow<FMT>(v[j], gs.d);
+      if ((CPR > 0 || c < nchunks) && row < p.rows && col < p.cols) st_stream_v2(codes + row * p.ld + col, q);
+    }
+    if (MODE == kCast) release_stage(release, lane);
+  }
+  if (MODE == kAmax) {
+    named_barrier(1, kConsumers);
+    for (int g = t; g < p.ngroups; g += kConsumers) {
+      uint32_t mx = wmax[0][g];
+#pragma unroll
+      for (int w = 1; w < kConsumerWarps; ++w) mx = max(mx, wmax[w][g]);
+      p.partials[(size_t)blockIdx.x * p.ngroups + g] = __uint_as_float(mx);
+    }
   }
 }
 
-template <int FMT, int CPR_T, int MAXC>
-static cudaError_t launch_tiles_impl(const uint16_t* x0, const uint16_t* x1, uint8_t* c0, uint8_t* c1, float* s0,
-                                     float* s1, int ntens, int64_t rows, int64_t cols, int64_t ld, int gw,
-                                     cudaStream_t st) {
-  const int nbr = (int)((rows + 127) / 128);
-  const int nbc = (int)((cols + gw - 1) / gw);
-  const int64_t ntiles = (int64_t)ntens * nbr * nbc;
-  if (ntiles == 0) return cudaSuccess;
-  static int occ = 0;
-  if (occ == 0) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_quant_tiles<FMT, CPR_T, MAXC>, 256, 0) !=
-            cudaSuccess ||
-        occ <= 0)
-      occ = 2;
+template <int FMT, int MODE, int CPR, int MAXC>
+static cudaError_t launch_tile_impl(const CUtensorMap& m0, const CUtensorMap& m1, TileParams& p, int max_grid,
+                                    cudaStream_t st, int* grid_used) {
+  const size_t smem = ring_smem(p.stages, p.stage_bytes);
+  static size_t attr = 0;
+  if (attr < smem) {
+    cudaFuncSetAttribute(k_tile128<FMT, MODE, CPR, MAXC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    attr = smem;
   }
-  const int grid = (int)std::min<int64_t>(ntiles, (int64_t)device_sm_count() * occ);
-  k_quant_tiles<FMT, CPR_T, MAXC><<<grid, 256, 0, st>>>(x0, x1, c0, c1, s0, s1, rows, cols, ld, gw, nbr, nbc,
-                                                         (int)ntiles);
+  int grid = grid_for(k_tile128<FMT, MODE, CPR, MAXC>, smem, std::max<uint32_t>(p.nitems, 1));
+  if (max_grid > 0) grid = std::min(grid, max_grid);
+  if (grid_used) *grid_used = grid;
+  k_tile128<FMT, MODE, CPR, MAXC><<<grid, kThreads, smem, st>>>(m0, m1, p);
   return cudaGetLastError();
 }
 
-template <int FMT>
-static cudaError_t launch_tiles_fmt(const uint16_t* x0, const uint16_t* x1, uint8_t* c0, uint8_t* c1, float* s0,
-                                    float* s1, int ntens, int64_t rows, int64_t cols, int64_t ld, int gw,
-                                    cudaStream_t st) {
-  if (gw == 128) return launch_tiles_impl<FMT, 16, 8>(x0, x1, c0, c1, s0, s1, ntens, rows, cols, ld, gw, st);
-  if (gw <= 128) return launch_tiles_impl<FMT, 0, 8>(x0, x1, c0, c1, s0, s1, ntens, rows, cols, ld, gw, st);
-  return launch_tiles_impl<FMT, 0, 16>(x0, x1, c0, c1, s0, s1, ntens, rows, cols, ld, gw, st);
+template <int FMT, int MODE>
+static cudaError_t launch_tile_fmt(const CUtensorMap& m0, const CUtensorMap& m1, TileParams& p, int max_grid,
+                                   cudaStream_t st, int* grid_used) {
+  if (p.bc == 128) return launch_tile_impl<FMT, MODE, 16, 8>(m0, m1, p, max_grid, st, grid_used);
+  if (p.bc == 64) return launch_tile_impl<FMT, MODE, 8, 4>(m0, m1, p, max_grid, st, grid_used);
+  if (p.bc == 256) return launch_tile_impl<FMT, MODE, 32, 16>(m0, m1, p, max_grid, st, grid_used);
+  if (p.bc < 128) return launch_tile_impl<FMT, MODE, 0, 8>(m0, m1, p, max_grid, st, grid_used);
+  return launch_tile_impl<FMT, MODE, 0, 16>(m0, m1, p, max_grid, st, grid_used);
+}
+
+template <int MODE>
+static cudaError_t launch_tile(int fmt, const CUtensorMap& m0, const CUtensorMap& m1, TileParams& p, int max_grid,
+                               cudaStream_t st, int* grid_used = nullptr) {
+  return fmt == kE4M3 ? launch_tile_fmt<kE4M3, MODE>(m0, m1, p, max_grid, st, grid_used)
+                      : launch_tile_fmt<kE5M2, MODE>(m0, m1, p, max_grid, st, grid_used);
+}
+
+// common set-up of a tile launch over ntens tensors of [rows][cols] (row stride ld) with
+// boxes of 128 x bc
+static bool tile_setup(TileParams& p, CUtensorMap& m0, CUtensorMap& m1, const uint16_t* x0, const uint16_t* x1,
+                       int ntens, int64_t rows, int64_t cols, int64_t ld, int bc) {
+  std::memset(&m0, 0, sizeof(m0));
+  std::memset(&m1, 0, sizeof(m1));
+  p.rows = rows;
+  p.cols = cols;
+  p.ld = ld;
+  p.bc = bc;
+  p.cpr = bc / 8;
+  const int64_t nbr = (rows + 127) / 128, nbc = (cols + bc - 1) / bc;
+  p.nbc = make_fastdiv((uint32_t)std::max<int64_t>(nbc, 1));
+  p.per_tensor = make_fastdiv((uint32_t)std::max<int64_t>(nbr * nbc, 1));
+  p.nitems = (uint32_t)(ntens * nbr * nbc);
+  p.stage_bytes = (uint32_t)(128 * bc * 2);
+  p.stages = (int)ring_stages(p.stage_bytes);
+  p.err = device_error_word();
+  p.partials = nullptr;
+  p.nparts = 0;
+  p.head_groups = 0;
+  p.heads = 1;
+  p.ngroups = ntens;
+  if (p.nitems == 0) return true;
+  if (!make_tmap_2d(&m0, 2, x0, (uint64_t)cols, (uint64_t)rows, (uint64_t)ld * 2, (uint32_t)bc, 128, 0)) return false;
+  if (!make_tmap_2d(&m1, 2, ntens > 1 ? x1 : x0, (uint64_t)cols, (uint64_t)rows, (uint64_t)ld * 2, (uint32_t)bc, 128,
+                    0))
+    return false;
+  return true;
 }
 
 cudaError_t launch_quant_tiles(const uint16_t* x0, const uint16_t* x1, uint8_t* c0, uint8_t* c1, float* s0,
                                float* s1, int ntens, int64_t rows, int64_t cols, int64_t ld, int gw, int fmt,
                                cudaStream_t st) {
-  return fmt == kE4M3 ? launch_tiles_fmt<kE4M3>(x0, x1, c0, c1, s0, s1, ntens, rows, cols, ld, gw, st)
-                      : launch_tiles_fmt<kE5M2>(x0, x1, c0, c1, s0, s1, ntens, rows, cols, ld, gw, st);
+  TileParams p;
+  CUtensorMap m0, m1;
+  if (!tile_setup(p, m0, m1, x0, x1, ntens, rows, cols, ld, gw)) return cudaErrorInvalidValue;
+  if (p.nitems == 0) return cudaSuccess;
+  p.c0 = c0;
+  p.c1 = ntens > 1 ? c1 : c0;
+  p.s0 = s0;
+  p.s1 = ntens > 1 ? s1 : s0;
+  return launch_tile<kOnePass>(fmt, m0, m1, p, 0, st);
 }
 
 // ============================================================================ two passes
 //
-// Per-tensor and per-head scales need the amax of a group that spans the whole tensor (or
-// all tokens of a head) before its first element can be cast, so they take two kernels.
-// Pass 1: CTA b reduces a contiguous range of 16-byte pieces into per-group maxima (shared
-// memory atomics on the 16-bit magnitude patterns) and writes them to partials[b][group].
-// Pass 2: each CTA folds the partials into the group scales, CTA 0 stores them, and the CTA
-// casts the same range it covered in pass 1, walking it backwards so that the tail it read
-// last, which is the part most likely still in L2, is consumed first.
-
-constexpr int kTwoPassThreads = 256;
-constexpr int kTwoPassUnroll = 8;
+// Per-tensor and per-head scales need the amax of a group spanning a whole tensor (or all
+// tokens of a head) before any of its elements can be cast: pass 1 (kAmax) writes per-CTA
+// partial maxima to the workspace, pass 2 (kCast) folds them and casts.
 
 size_t two_pass_workspace_bytes(int ntens, int64_t heads) {
-  return (size_t)kMaxPartials * (size_t)ntens * (size_t)heads * sizeof(float);
-}
-
-struct TwoPassShape {
-  const uint16_t* x0;
-  const uint16_t* x1;
-  uint8_t* c0;
-  uint8_t* c1;
-  float* s0;
-  float* s1;
-  uint32_t chunks;      // 16-byte pieces per tensor
-  FastDiv cpr;          // pieces per row
-  FastDiv cpg;          // pieces per head
-  uint32_t heads;
-  uint32_t ngroups;     // ntens * heads
-  uint32_t per_cta;     // pieces per CTA range (multiple of the thread count)
-  uint32_t total;       // ntens * chunks
-};
-
-__device__ __forceinline__ uint32_t group_of(const TwoPassShape& sh, uint32_t i, uint32_t* tens, uint32_t* w) {
-  const uint32_t t = i >= sh.chunks ? 1u : 0u;
-  const uint32_t wi = i - t * sh.chunks;
-  *tens = t;
-  *w = wi;
-  if (sh.heads == 1) return t;
-  const uint32_t col_piece = wi - fdiv(wi, sh.cpr) * sh.cpr.d;
-  return t * sh.heads + fdiv(col_piece, sh.cpg);
-}
-
-__global__ void __launch_bounds__(kTwoPassThreads) k_two_pass_amax(TwoPassShape sh, float* __restrict__ partials) {
-  __shared__ uint32_t smax[256];
-  for (uint32_t g = threadIdx.x; g < sh.ngroups; g += kTwoPassThreads) smax[g] = 0u;
-  __syncthreads();
-  const uint32_t beg = blockIdx.x * sh.per_cta;
-  const uint32_t end = min(sh.total, beg + sh.per_cta);
-  uint32_t cur = 0xFFFFFFFFu, m = 0u;
-  for (uint32_t i0 = beg + threadIdx.x; i0 < end; i0 += kTwoPassThreads * kTwoPassUnroll) {
-    uint4 v[kTwoPassUnroll];
-#pragma unroll
-    for (int k = 0; k < kTwoPassUnroll; ++k) {
-      const uint32_t i = i0 + k * kTwoPassThreads;
-      uint32_t t = 0, w = 0;
-      if (i < end) group_of(sh, i, &t, &w);
-      v[k] = i < end ? ld_stream_v4((t ? sh.x1 : sh.x0) + (size_t)w * 8) : make_uint4(0u, 0u, 0u, 0u);
-    }
-#pragma unroll
-    for (int k = 0; k < kTwoPassUnroll; ++k) {
-      const uint32_t i = i0 + k * kTwoPassThreads;
-      if (i >= end) break;
-      uint32_t t, w;
-      const uint32_t g = group_of(sh, i, &t, &w);
-      if (g != cur) {
-        if (cur != 0xFFFFFFFFu) atomicMax(&smax[cur], max(m & 0xFFFFu, m >> 16));
-        cur = g;
-        m = 0u;
-      }
-      m = absmax_v4(m, v[k]);
-    }
-  }
-  if (cur != 0xFFFFFFFFu) atomicMax(&smax[cur], max(m & 0xFFFFu, m >> 16));
-  __syncthreads();
-  for (uint32_t g = threadIdx.x; g < sh.ngroups; g += kTwoPassThreads)
-    partials[(size_t)blockIdx.x * sh.ngroups + g] = __uint_as_float(smax[g] << 16);
-}
-
-template <int FMT>
-__global__ void __launch_bounds__(kTwoPassThreads) k_two_pass_cast(TwoPassShape sh, const float* __restrict__ partials,
-                                                                 int nparts) {
-  __shared__ uint32_t sred[256];
-  __shared__ GroupScale sg[256];
-  for (uint32_t g = threadIdx.x; g < sh.ngroups; g += kTwoPassThreads) sred[g] = 0u;
-  __syncthreads();
-  // fold partials: amax values are non-negative floats (or NaN), whose bit patterns order
-  // like their values with NaN on top, so an integer max is exact
-  const uint32_t nitems = (uint32_t)nparts * sh.ngroups;
-  for (uint32_t it = threadIdx.x; it < nitems; it += kTwoPassThreads) {
-    const uint32_t g = it % sh.ngroups;
-    atomicMax(&sred[g], __float_as_uint(partials[it]));
-  }
-  __syncthreads();
-  for (uint32_t g = threadIdx.x; g < sh.ngroups; g += kTwoPassThreads) {
-    sg[g] = make_group_scale<FMT>(__uint_as_float(sred[g]));
-    if (blockIdx.x == 0) {
-      const uint32_t t = g / sh.heads;
-      (t ? sh.s1 : sh.s0)[g - t * sh.heads] = sg[g].s;
-    }
-  }
-  __syncthreads();
-  const uint32_t beg = blockIdx.x * sh.per_cta;
-  const uint32_t end = min(sh.total, beg + sh.per_cta);
-  if (beg >= end) return;
-  // walk the range backwards in steps of the CTA width
-  const uint32_t span = end - beg;
-  const uint32_t nsteps = (span + kTwoPassThreads - 1) / kTwoPassThreads;
-  for (int64_t step = (int64_t)nsteps - 1; step >= 0; step -= 4) {
-    uint4 v[4];
-    uint32_t ii[4], tt[4], ww[4], gg[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int64_t sidx = step - k;
-      const uint32_t i = sidx >= 0 ? beg + (uint32_t)sidx * kTwoPassThreads + threadIdx.x : end;
-      ii[k] = i;
-      tt[k] = 0;
-      ww[k] = 0;
-      gg[k] = i < end ? group_of(sh, i, &tt[k], &ww[k]) : 0u;
-      v[k] = i < end ? ld_stream_v4((tt[k] ? sh.x1 : sh.x0) + (size_t)ww[k] * 8) : make_uint4(0u, 0u, 0u, 0u);
-    }
-#pragma unroll
-    for (int k = 0; k < 4; ++k)
-      if (ii[k] < end) st_stream_v2((tt[k] ? sh.c1 : sh.c0) + (size_t)ww[k] * 8, quant8<FMT>(v[k], sg[gg[k]]));
-  }
+  return (size_t)kMaxPartials * (size_t)ntens * (size_t)std::max<int64_t>(heads, 1) * sizeof(float);
 }
 
 cudaError_t launch_quant_two_pass(const uint16_t* x0, const uint16_t* x1, uint8_t* c0, uint8_t* c1, float* s0,
                                   float* s1, int ntens, int64_t rows, int64_t heads, int64_t head_dim, int fmt,
                                   float* ws, cudaStream_t st) {
-  TwoPassShape sh;
-  sh.x0 = x0;
-  sh.x1 = ntens > 1 ? x1 : x0;
-  sh.c0 = c0;
-  sh.c1 = ntens > 1 ? c1 : c0;
-  sh.s0 = s0;
-  sh.s1 = ntens > 1 ? s1 : s0;
-  const int64_t cpr = heads * head_dim / 8;
-  sh.chunks = (uint32_t)(rows * cpr);
-  sh.cpr = make_fastdiv((uint32_t)std::max<int64_t>(cpr, 1));
-  sh.cpg = make_fastdiv((uint32_t)std::max<int64_t>(head_dim / 8, 1));
-  sh.heads = (uint32_t)heads;
-  sh.ngroups = (uint32_t)(ntens * heads);
-  sh.total = (uint32_t)ntens * sh.chunks;
-  const int sms = device_sm_count();
-  // pass-1 CTAs: two per SM for large tensors, fewer for small ones (at least 8 KB each)
-  const int64_t want = std::min<int64_t>((int64_t)2 * sms, kMaxPartials);
-  const int64_t min_per = 512;   // pieces (8 KB of bf16)
-  int64_t nparts = std::max<int64_t>(1, std::min<int64_t>(want, ((int64_t)sh.total + min_per - 1) / min_per));
-  int64_t per = ((int64_t)sh.total + nparts - 1) / nparts;
-  per = std::max<int64_t>(kTwoPassThreads, (per + kTwoPassThreads - 1) / kTwoPassThreads * kTwoPassThreads);
-  nparts = std::max<int64_t>(1, ((int64_t)sh.total + per - 1) / per);
-  sh.per_cta = (uint32_t)per;
-  k_two_pass_amax<<<(int)nparts, kTwoPassThreads, 0, st>>>(sh, ws);
-  cudaError_t e = cudaGetLastError();
+  // per-tensor: boxes of 128 x 128 over [rows][heads * head_dim]; per-head: boxes of
+  // 128 tokens x head_dim, one group per (tensor, head)
+  const int64_t cols = heads * head_dim;
+  const bool per_head = heads > 1;
+  const int bc = per_head ? (int)head_dim : 128;
+  if (ntens * (per_head ? heads : 1) > kMaxGroups) return cudaErrorInvalidValue;
+  TileParams p;
+  CUtensorMap m0, m1;
+  if (!tile_setup(p, m0, m1, x0, x1, ntens, rows, cols, cols, bc)) return cudaErrorInvalidValue;
+  p.c0 = c0;
+  p.c1 = ntens > 1 ? c1 : c0;
+  p.s0 = s0;
+  p.s1 = ntens > 1 ? s1 : s0;
+  p.head_groups = per_head ? 1 : 0;
+  p.heads = per_head ? (int)heads : 1;
+  p.ngroups = ntens * p.heads;
+  p.partials = ws;
+  if (p.nitems == 0) {
+    // empty tensors: amax = 0 for every group, so pass 2 alone writes s = 0
+    p.nparts = 0;
+    return launch_tile<kCast>(fmt, m0, m1, p, 1, st);
+  }
+  const int grid1 = (int)std::min<int64_t>((int64_t)p.nitems, std::min<int64_t>(kMaxPartials, 2 * device_sm_count()));
+  p.nparts = 0;
+  int written = 0;
+  cudaError_t e = launch_tile<kAmax>(fmt, m0, m1, p, grid1, st, &written);
   if (e != cudaSuccess) return e;
-  if (fmt == kE4M3)
-    k_two_pass_cast<kE4M3><<<(int)nparts, kTwoPassThreads, 0, st>>>(sh, ws, (int)nparts);
-  else
-    k_two_pass_cast<kE5M2><<<(int)nparts, kTwoPassThreads, 0, st>>>(sh, ws, (int)nparts);
-  return cudaGetLastError();
+  p.nparts = written;   // partial rows pass 1 wrote (its grid size)
+  return launch_tile<kCast>(fmt, m0, m1, p, written, st);
 }
 
 }  // namespace fp8q

@@ -102,6 +102,14 @@ FP8Q_API const char *fp8q_status_string(fp8q_status status);
 /* Library version as major*10000 + minor*100 + patch. */
 FP8Q_API int fp8q_version(void);
 
+/*
+ * Synchronizes the current device, returns the library's device error bits and clears them.
+ * 0: no error.  Bit 0: a bounded wait inside a kernel (a pipeline barrier that never completed)
+ * gave up after its time limit, so that kernel's outputs are incomplete.  0xFFFFFFFF: the
+ * device could not be queried (e.g. an earlier fault).
+ */
+FP8Q_API uint32_t fp8q_device_status(void);
+
 /* ---------------------------------------------------------------- sizes */
 
 /* Number of fp32 scales fp8_quantize writes for a [rows][cols] tensor; 0 on a bad argument. */

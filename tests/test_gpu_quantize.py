@@ -21,6 +21,9 @@ pytestmark = pytest.mark.gpu
 def _cuda():
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
     fq.lib()
+    assert fq.device_status() == 0
+    yield
+    assert fq.device_status() == 0, "a kernel's bounded wait gave up"
 
 
 def quant_gpu(x, fmt, gran):
