@@ -80,12 +80,14 @@ __device__ __forceinline__ float packed_amax_to_f32(uint32_t m) {
 // per element is far too slow for an HBM-bound kernel, so groups whose amax is an ordinary
 // normal number use Markstein's correction (P. Markstein, "Computation of elementary
 // functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990): with
-// r = RN(1/d) and q0 = RN(x * r), the residual e = x - q0 * d is exact in one FMA and
-// RN(q0 + e * r) = RN(x / d) when nothing overflows or underflows.  The same step with the
-// constant RN(1/FMAX) gives the scale s = RN(amax / FMAX).  Groups with a tiny, infinite or
-// NaN amax take IEEE divisions instead.  An all-zero group has s = 0 and divides by 1 (every x
-// is +-0).  The Markstein step maps x = -0 to +0, so the inputs' sign bits are OR-ed back into
-// the codes.  The fast path is checked against the oracle for every (bf16 x, bf16 amax) pair.
+// r = RN(1/d) and q0 = RN(x * r), the residual x - q0 * d is exact in one FMA and
+// RN(q0 + (x - q0 * d) * r) = RN(x / d) when nothing overflows or underflows.  The residual is
+// formed negated, e' = q0 * d - x, and applied as q = q0 - e' * r: the same value for x != 0,
+// and for x = -0 it yields -0 (q0 = -0, e' = +0, -0 + -0 = -0), so zero signs need no fix-up.
+// The same step with the constant RN(1/FMAX) gives the scale s = RN(amax / FMAX).  Groups with
+// a tiny, infinite or NaN amax take IEEE divisions instead.  An all-zero group has s = 0 and
+// divides by 1 (every x is +-0).  The fast path is checked against the oracle for every
+// (bf16 x, bf16 amax) pair.
 
 struct GroupScale {
   float s;     // stored scale
@@ -96,8 +98,8 @@ struct GroupScale {
 
 __device__ __forceinline__ float markstein_div(float x, float d, float r) {
   const float q0 = __fmul_rn(x, r);
-  const float e = __fmaf_rn(-q0, d, x);
-  return __fmaf_rn(e, r, q0);
+  const float en = __fmaf_rn(q0, d, -x);     // -(x - q0 * d), exact
+  return __fmaf_rn(-en, r, q0);
 }
 
 template <int FMT>
@@ -173,23 +175,25 @@ __device__ __forceinline__ uint32_t f32x2_to_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// sign bits of four bf16 (two words) placed on bit 7 of four code bytes
-__device__ __forceinline__ uint32_t signs4(uint32_t w0, uint32_t w1) {
-  return __byte_perm(w0, w1, 0x7531) & 0x80808080u;
-}
-
 // four bf16 (two words) -> four codes, fast path
 template <int FMT>
 __device__ __forceinline__ uint32_t quant4_fast(uint32_t w0, uint32_t w1, float d, float r) {
   const uint32_t a = cvt2<FMT>(markstein_div(bf16_lo(w0), d, r), markstein_div(bf16_hi(w0), d, r));
   const uint32_t b = cvt2<FMT>(markstein_div(bf16_lo(w1), d, r), markstein_div(bf16_hi(w1), d, r));
-  return __byte_perm(a, b, 0x5410) | signs4(w0, w1);
+  return __byte_perm(a, b, 0x5410);
 }
 
 // eight bf16 (16 bytes) -> eight codes (8 bytes), fast path
 template <int FMT>
 __device__ __forceinline__ uint2 quant8_fast(uint4 v, float d, float r) {
   return make_uint2(quant4_fast<FMT>(v.x, v.y, d, r), quant4_fast<FMT>(v.z, v.w, d, r));
+}
+
+// sixteen bf16 (two 16-byte pieces) -> sixteen codes (16 bytes), fast path
+template <int FMT>
+__device__ __forceinline__ uint4 quant16_fast(uint4 a, uint4 b, float d, float r) {
+  return make_uint4(quant4_fast<FMT>(a.x, a.y, d, r), quant4_fast<FMT>(a.z, a.w, d, r),
+                    quant4_fast<FMT>(b.x, b.y, d, r), quant4_fast<FMT>(b.z, b.w, d, r));
 }
 
 // eight bf16 -> eight codes with IEEE divisions (groups with tiny, infinite or NaN amax)
@@ -201,7 +205,7 @@ __device__ __noinline__ uint2 quant8_slow(uint4 v, float d) {
   for (int i = 0; i < 2; ++i) {
     const uint32_t a = cvt2<FMT>(__fdiv_rn(bf16_lo(w[2 * i]), d), __fdiv_rn(bf16_hi(w[2 * i]), d));
     const uint32_t b = cvt2<FMT>(__fdiv_rn(bf16_lo(w[2 * i + 1]), d), __fdiv_rn(bf16_hi(w[2 * i + 1]), d));
-    c[i] = __byte_perm(a, b, 0x5410) | signs4(w[2 * i], w[2 * i + 1]);
+    c[i] = __byte_perm(a, b, 0x5410);
   }
   return make_uint2(c[0], c[1]);
 }

@@ -126,7 +126,7 @@ struct GroupParams {
   uint32_t nitems;
   FastDiv ngc;        // 128-column groups per row
   int stages;
-  int wide_stores;    // cols % 32 == 0: 16-byte code stores
+  int wide_stores;    // cols % 16 == 0: rows start 16-byte aligned, 16-byte code stores
   uint32_t* err;
 };
 
@@ -159,15 +159,17 @@ __global__ void __launch_bounds__(kThreads, 2) k_group128(const __grid_constant_
     }
     return;
   }
+  // thread (grp, q) owns chunk pairs q and q + 4 of box row grp: 32 elements, two 16-byte stores
   const int t = threadIdx.x, grp = t >> 2, q = t & 3;
+  const uint32_t soff = grp * 256 + q * 32;
   int s = 0;
   uint32_t ph = 0;
   for (uint32_t k = 0; k < nk; ++k) {
     const uint32_t i = blockIdx.x + k * gridDim.x;
     if (!mbar_wait(&full[s], ph, p.err)) break;
-    const uint8_t* src = smem + s * kGroupStage + grp * 256 + q * 64;
-    const uint4 v0 = ld_shared_v4(src), v1 = ld_shared_v4(src + 16), v2 = ld_shared_v4(src + 32),
-                v3 = ld_shared_v4(src + 48);
+    const uint8_t* src = smem + s * kGroupStage + soff;
+    const uint4 v0 = ld_shared_v4(src), v1 = ld_shared_v4(src + 16), v2 = ld_shared_v4(src + 128),
+                v3 = ld_shared_v4(src + 144);
     uint32_t m = absmax_v4(absmax_v4(absmax_v4(absmax_v4(0u, v0), v1), v2), v3);   // consumes every load
     release_stage(&empty[s], lane);
     if (++s == S) {
@@ -179,29 +181,17 @@ __global__ void __launch_bounds__(kThreads, 2) k_group128(const __grid_constant_
     const GroupScale gs = make_group_scale<FMT>(packed_amax_to_f32(m));
     const uint32_t rb = fdiv(i, p.ngc), g = i - rb * p.ngc.d;
     const int64_t row = (int64_t)rb * kGroupBoxRows + grp;
-    const int64_t col = (int64_t)g * 128 + q * 32;
     if (row >= p.rows) continue;
-    uint2 c0, c1, c2, c3;
-    if (gs.fast) {
-      c0 = quant8_fast<FMT>(v0, gs.d, gs.r);
-      c1 = quant8_fast<FMT>(v1, gs.d, gs.r);
-      c2 = quant8_fast<FMT>(v2, gs.d, gs.r);
-      c3 = quant8_fast<FMT>(v3, gs.d, gs.r);
+    const int64_t col0 = (int64_t)g * 128 + q * 16, col1 = col0 + 64;
+    uint8_t* dst = p.codes + row * p.cols;
+    if (gs.fast && p.wide_stores && (int64_t)g * 128 + 128 <= p.cols) {
+      st_stream_v4(dst + col0, quant16_fast<FMT>(v0, v1, gs.d, gs.r));
+      st_stream_v4(dst + col1, quant16_fast<FMT>(v2, v3, gs.d, gs.r));
     } else {
-      c0 = quant8_slow<FMT>(v0, gs.d);
-      c1 = quant8_slow<FMT>(v1, gs.d);
-      c2 = quant8_slow<FMT>(v2, gs.d);
-      c3 = quant8_slow<FMT>(v3, gs.d);
-    }
-    uint8_t* dst = p.codes + row * p.cols + col;
-    if (p.wide_stores && col + 32 <= p.cols) {
-      st_stream_v4(dst, make_uint4(c0.x, c0.y, c1.x, c1.y));
-      st_stream_v4(dst + 16, make_uint4(c2.x, c2.y, c3.x, c3.y));
-    } else {
-      if (col < p.cols) st_stream_v2(dst, c0);
-      if (col + 8 < p.cols) st_stream_v2(dst + 8, c1);
-      if (col + 16 < p.cols) st_stream_v2(dst + 16, c2);
-      if (col + 24 < p.cols) st_stream_v2(dst + 24, c3);
+      if (col0 < p.cols) st_stream_v2(dst + col0, quant8<FMT>(v0, gs));
+      if (col0 + 8 < p.cols) st_stream_v2(dst + col0 + 8, quant8<FMT>(v1, gs));
+      if (col1 < p.cols) st_stream_v2(dst + col1, quant8<FMT>(v2, gs));
+      if (col1 + 8 < p.cols) st_stream_v2(dst + col1 + 8, quant8<FMT>(v3, gs));
     }
     if (q == 0) p.scales[(int64_t)g * p.rows + row] = gs.s;
   }
@@ -225,7 +215,7 @@ static cudaError_t launch_group128_fmt(const uint16_t* x, int64_t rows, int64_t 
   p.nitems = (uint32_t)nitems;
   p.ngc = make_fastdiv((uint32_t)ngc);
   p.stages = (int)ring_stages(kGroupStage);
-  p.wide_stores = cols % 32 == 0;
+  p.wide_stores = cols % 16 == 0;
   p.err = device_error_word();
   const size_t smem = ring_smem(p.stages, kGroupStage);
   static bool attr = false;
@@ -362,19 +352,37 @@ __global__ void __launch_bounds__(kThreads, 2) k_tile128(const __grid_constant__
     named_barrier(1, kConsumers);
   }
 
+  // CPR > 0: thread t owns chunk pairs t + 256 * jp (32 smem bytes each; pair q of the box sits
+  // at row q / PPR, 16-column block q % PPR); interior boxes with a fast scale take 16-byte
+  // stores with no per-chunk checks.  CPR == 0 (unusual head sizes): single chunks, all checked.
+  constexpr int PPR = CPR / 2;
+  constexpr int MAXP = CPR > 0 ? CPR / 4 : 1;
+  constexpr int ROWSTEP = CPR > 0 ? kConsumers / PPR : 1;
+  const int r0 = CPR > 0 ? t / PPR : 0, cp = CPR > 0 ? t % PPR : 0;
+  const bool wide = (p.ld % 16) == 0;
   int s = 0;
   uint32_t ph = 0;
   for (uint32_t k = 0; k < nk; ++k) {
     const uint32_t i = tile_item_index<MODE>(k, p.nitems);
     if (!mbar_wait(&full[s], ph, p.err)) break;
     const uint8_t* stage = smem + s * p.stage_bytes;
-    uint4 v[MAXC];
+    uint4 va[CPR > 0 ? MAXP : MAXC], vb[CPR > 0 ? MAXP : 1];
     uint32_t m = 0u;
+    if constexpr (CPR > 0) {
 #pragma unroll
-    for (int j = 0; j < MAXC; ++j) {
-      const int c = t + kConsumers * j;
-      v[j] = (CPR > 0 || c < nchunks) ? ld_shared_v4(stage + c * 16) : make_uint4(0u, 0u, 0u, 0u);
-      if (MODE != kCast) m = absmax_v4(m, v[j]);
+      for (int jp = 0; jp < MAXP; ++jp) {
+        const uint8_t* src = stage + (t + kConsumers * jp) * 32;
+        va[jp] = ld_shared_v4(src);
+        vb[jp] = ld_shared_v4(src + 16);
+        if (MODE != kCast) m = absmax_v4(absmax_v4(m, va[jp]), vb[jp]);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < MAXC; ++j) {
+        const int c = t + kConsumers * j;
+        va[j] = c < nchunks ? ld_shared_v4(stage + c * 16) : make_uint4(0u, 0u, 0u, 0u);
+        if (MODE != kCast) m = absmax_v4(m, va[j]);
+      }
     }
     // the amax consumed every load; the cast pass releases the stage after the cast instead
     uint64_t* release = &empty[s];
@@ -409,14 +417,34 @@ __global__ void __launch_bounds__(kThreads, 2) k_tile128(const __grid_constant__
       gs = table[(int)it.tens * p.heads + (p.head_groups ? (int)it.bj : 0)];
     }
     uint8_t* codes = it.tens ? p.c1 : p.c0;
+    const int64_t row_base = (int64_t)it.bi * 128, col_base = (int64_t)it.bj * p.bc;
+    if constexpr (CPR > 0) {
+      const bool interior = row_base + 128 <= p.rows && col_base + p.bc <= p.cols;
+      if (gs.fast && interior && wide) {
+        uint8_t* dst = codes + (row_base + r0) * p.ld + col_base + cp * 16;
+        const int64_t step = (int64_t)ROWSTEP * p.ld;
 #pragma unroll
-    for (int j = 0; j < MAXC; ++j) {
-      const int c = t + kConsumers * j;
-      const int r = c / cpr, cc = c - r * cpr;
-      const int64_t row = (int64_t)it.bi * 128 + r;
-      const int64_t col = (int64_t)it.bj * p.bc + cc * 8;
-      const uint2 q = gs.fast ? quant8_fast<FMT>(v[j], gs.d, gs.r) : quant8_slow<FMT>(v[j], gs.d);
-      if ((CPR > 0 || c < nchunks) && row < p.rows && col < p.cols) st_stream_v2(codes + row * p.ld + col, q);
+        for (int jp = 0; jp < MAXP; ++jp) st_stream_v4(dst + jp * step, quant16_fast<FMT>(va[jp], vb[jp], gs.d, gs.r));
+      } else {
+#pragma unroll
+        for (int jp = 0; jp < MAXP; ++jp) {
+          const int64_t row = row_base + r0 + jp * ROWSTEP;
+          const int64_t col = col_base + cp * 16;
+          uint8_t* dst = codes + row * p.ld + col;
+          if (row < p.rows && col < p.cols) st_stream_v2(dst, quant8<FMT>(va[jp], gs));
+          if (row < p.rows && col + 8 < p.cols) st_stream_v2(dst + 8, quant8<FMT>(vb[jp], gs));
+        }
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < MAXC; ++j) {
+        const int c = t + kConsumers * j;
+        const int r = c / cpr, cc = c - r * cpr;
+        const int64_t row = row_base + r;
+        const int64_t col = col_base + cc * 8;
+        const uint2 q = quant8<FMT>(va[j], gs);
+        if (c < nchunks && row < p.rows && col < p.cols) st_stream_v2(codes + row * p.ld + col, q);
+      }
     }
     if (MODE == kCast) release_stage(release, lane);
   }
