@@ -1,0 +1,152 @@
+"""GPU parity for the block-scaled FP8 GEMM against the oracle's fp64 product.
+
+Operands are quantized by the oracle on the CPU and the same codes and scales go to both
+sides.  Tolerance (bf16 output vs the fp64 product of the dequantized operands):
+relative Frobenius error <= 5e-3 and every element within 1e-2 * max(|ref|, 1e-2).
+Small shapes cover partial M tiles, N not a multiple of the 256-column tile and every scale
+combination; the configuration shapes are checked on sampled rows (one per 128-row M tile at
+varying offsets, plus the first and last row), which touch every output tile.
+"""
+import numpy as np
+import pytest
+import torch
+
+import fp8_quantization_amax_b200 as fq
+import synth
+from helpers import dev, host
+
+pytestmark = pytest.mark.gpu
+
+REL_FRO = 5e-3
+ELEM = 1e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    fq.lib()
+    assert fq.device_status() == 0
+    yield
+    assert fq.device_status() == 0, "a kernel's bounded wait gave up"
+
+
+def bf16_to_f64(bits):
+    return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def check_tolerance(got_bits, ref, what=""):
+    got = bf16_to_f64(got_bits)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    rel = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300)
+    bound = ELEM * np.maximum(np.abs(ref), 1e-2)
+    bad = np.abs(got - ref) > bound
+    assert rel <= REL_FRO, f"{what}: relative Frobenius error {rel:.3e}"
+    assert not bad.any(), f"{what}: {bad.sum()} elements out of bound, e.g. got {got[bad][:4]} ref {ref[bad][:4]}"
+    return rel
+
+
+def operands(orc, M, N, K, ga, gb, seed, x=None, w=None):
+    if x is None:
+        x = synth.activations(seed=seed, m=M, k=K)
+    if w is None:
+        w = synth.weight_8b(seed=seed, n=N, k=K)
+    a, sa = orc.quantize(x, orc.E4M3, orc.GROUP_1x128 if ga == 1 else orc.PER_TENSOR)
+    b, sb = orc.quantize(w, orc.E4M3, orc.BLOCK_128x128 if gb == 2 else orc.PER_TENSOR)
+    return a, sa, b, sb
+
+
+def run_gpu(a, sa, b, sb, ga, gb):
+    c = fq.fp8_gemm_blockscaled(dev(a), dev(sa), dev(b), dev(sb), ga, gb)
+    torch.cuda.synchronize()
+    return host(c)
+
+
+def sample_rows(M, seed=0):
+    rng = np.random.default_rng(seed)
+    rows = [0, M - 1] + [t * 128 + int(rng.integers(0, min(128, M - t * 128))) for t in range((M + 127) // 128)]
+    return np.unique(np.array(rows, np.int64))
+
+
+@pytest.mark.parametrize("ga,gb", [(1, 2), (0, 0), (1, 0), (0, 2)])
+@pytest.mark.parametrize("shape", [(1, 128, 128), (16, 256, 256), (128, 256, 128), (130, 384, 512),
+                                   (300, 512, 384), (257, 128, 1024)])
+def test_gemm_small(orc, ga, gb, shape):
+    M, N, K = shape
+    a, sa, b, sb = operands(orc, M, N, K, ga, gb, seed=M + N + K)
+    got = run_gpu(a, sa, b, sb, ga, gb)
+    ref = orc.gemm_rows(a, sa, ga, b, sb, gb, np.arange(M))
+    check_tolerance(got, ref, f"{shape} gA={ga} gB={gb}")
+
+
+def test_gemm_exact_small_integers(orc):
+    """Codes of small integers with unit scales: fp32 accumulation is exact, the output is the
+    integer product rounded once to bf16."""
+    rng = np.random.default_rng(3)
+    M, N, K = 64, 256, 256
+    vals = np.array([0.0, 1.0, -1.0, 2.0, -2.0, 3.0, -4.0], np.float32)
+    A = orc.encode(vals[rng.integers(0, vals.size, (M, K))], orc.E4M3)
+    B = orc.encode(vals[rng.integers(0, vals.size, (N, K))], orc.E4M3)
+    one = np.ones(1, np.float32)
+    got = run_gpu(A, one, B, one, fq.PER_TENSOR, fq.PER_TENSOR)
+    ref = orc.gemm_rows(A, one, 0, B, one, 0, np.arange(M))
+    want = (ref.astype(np.float32).view(np.uint32) + 0x7FFF + ((ref.astype(np.float32).view(np.uint32) >> 16) & 1)) >> 16
+    assert np.array_equal(got.astype(np.uint32), want)
+
+
+def test_gemm_block_scale_selection(orc):
+    """A single nonzero K block: the output must carry exactly that block's scales."""
+    M, N, K = 128, 256, 512
+    A = np.zeros((M, K), np.uint8)
+    B = np.zeros((N, K), np.uint8)
+    A[:, 256:384] = 0x38      # 1.0 in K block 2
+    B[:, 256:384] = 0x38
+    sa = (np.arange(4 * M, dtype=np.float32).reshape(4, M) % 7 + 1) / 8
+    sb = (np.arange(2 * 4, dtype=np.float32).reshape(2, 4) + 1) / 4
+    got = run_gpu(A, sa, B, sb, fq.GROUP_1x128, fq.BLOCK_128x128)
+    ref = orc.gemm_rows(A, sa, 1, B, sb, 2, np.arange(M))
+    check_tolerance(got, ref, "single block")
+
+
+def test_gemm_config2_prefill_8b(orc):
+    M, N, K = 8192, 14336, 4096
+    x = synth.activations(seed=1)
+    w = synth.weight_8b(seed=1)
+    a, sa, b, sb = operands(orc, M, N, K, 1, 2, 1, x=x, w=w)
+    got = run_gpu(a, sa, b, sb, 1, 2)
+    rows = sample_rows(M)
+    ref = orc.gemm_rows(a, sa, 1, b, sb, 2, rows)
+    check_tolerance(got[rows], ref, "config 2 M=8192")
+
+
+def test_gemm_config2_decode_8b(orc):
+    M, N, K = 16, 14336, 4096
+    x = synth.activations(seed=1)[:M]
+    w = synth.weight_8b(seed=1)
+    a, sa, b, sb = operands(orc, M, N, K, 1, 2, 1, x=x, w=w)
+    got = run_gpu(a, sa, b, sb, 1, 2)
+    ref = orc.gemm_rows(a, sa, 1, b, sb, 2, np.arange(M))
+    check_tolerance(got, ref, "config 2 M=16")
+
+
+@pytest.mark.parametrize("which", ["up", "down"])
+@pytest.mark.parametrize("M", [16384, 64])
+def test_gemm_config4_70b(orc, which, M):
+    w = synth.weight_70b(seed=4, which=which)
+    x = synth.activations_70b(seed=4, m=M, which=which)
+    N, K = w.shape
+    a, sa, b, sb = operands(orc, M, N, K, 1, 2, 4, x=x, w=w)
+    got = run_gpu(a, sa, b, sb, 1, 2)
+    rows = sample_rows(M)[:40] if M > 64 else np.arange(M)
+    ref = orc.gemm_rows(a, sa, 1, b, sb, 2, rows)
+    check_tolerance(got[rows], ref, f"config 4 {which} M={M}")
+
+
+def test_gemm_config4_per_tensor_variant(orc):
+    w = synth.weight_70b(seed=4, which="up")
+    x = synth.activations_70b(seed=4, m=1024, which="up")
+    N, K = w.shape
+    a, sa, b, sb = operands(orc, 1024, N, K, 0, 0, 4, x=x, w=w)
+    got = run_gpu(a, sa, b, sb, 0, 0)
+    rows = sample_rows(1024)
+    ref = orc.gemm_rows(a, sa, 0, b, sb, 0, rows)
+    check_tolerance(got[rows], ref, "config 4 per-tensor")
