@@ -489,6 +489,47 @@ def our_arm(args):
     return 0
 
 
+def profile_target(name, reps):
+    """Set up one workload, run it `reps` times (after two warm-up runs) and print the mean time."""
+    import torch
+
+    import fp8_quantization_amax_b200 as fq
+    import synth
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        if name.startswith("gemm"):
+            if name == "gemm_70b_up_m16384":
+                w = dev_bf16(synth.weight_70b(seed=4, which="up"), device)
+                x = dev_bf16(synth.activations_70b(seed=4, m=16384, which="up"), device)
+            else:
+                w = dev_bf16(synth.weight_8b(seed=1), device)
+                x = dev_bf16(synth.activations(seed=1), device)
+                if name == "gemm_8b_m16":
+                    x = x[:16].contiguous()
+            a, sa = fq.fp8_quantize(x, fq.E4M3, fq.GROUP_1x128)
+            b, sb = fq.fp8_quantize(w, fq.E4M3, fq.BLOCK_128x128)
+            c = torch.empty((a.shape[0], b.shape[0]), dtype=torch.bfloat16, device=device)
+            fn = lambda: fq.fp8_gemm_blockscaled(a, sa, b, sb, out=c)  # noqa: E731
+        elif name.startswith("kv"):
+            k, v = synth.kv_70b(seed=3)
+            kd, vd = dev_bf16(k, device), dev_bf16(v, device)
+            gran = fq.KV_PER_HEAD_TOK128 if name == "kv_tok128" else fq.KV_PER_HEAD
+            r = fq.fp8_kv_quantize(kd, vd, fq.E4M3, gran)
+            fn = lambda: fq.fp8_kv_quantize(kd, vd, fq.E4M3, gran, *r)  # noqa: E731
+        else:
+            w = dev_bf16(synth.weight_8b(seed=1), device)
+            wc, ws = fq.fp8_quantize(w, fq.E4M3, fq.BLOCK_128x128)
+            y = torch.empty_like(w)
+            fn = lambda: fq.fp8_dequantize(wc, ws, fq.E4M3, fq.BLOCK_128x128, out=y)  # noqa: E731
+        for _ in range(2):
+            fn()
+        ms = timed(fn, max(reps, 1), stream)
+    print(json.dumps({"profile_target": name, "reps": reps, "ms": round(ms, 4)}), flush=True)
+    return 0 if fq.device_status() == 0 else 1
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -498,11 +539,17 @@ def main():
     ap.add_argument("--no-supplementary", action="store_true")
     ap.add_argument("--skip-extras", action="store_true",
                     help="time the steps only: no e2e, CPU baseline or supplementary kernels (for profiling)")
+    ap.add_argument("--profile-target", default=None,
+                    choices=["gemm_8b_m8192", "gemm_8b_m16", "gemm_70b_up_m16384", "kv_tok128", "kv_head",
+                             "dequant_8b"],
+                    help="run one workload a few times and exit (a small target for ncu)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         return reference_arm(args)
+    if args.profile_target:
+        return profile_target(args.profile_target, args.steps)
     return our_arm(args)
 
 

@@ -10,6 +10,7 @@ from __future__ import annotations
 
 import glob
 import os
+import re
 import subprocess
 import sys
 from concurrent.futures import ThreadPoolExecutor
@@ -40,6 +41,25 @@ def _headers() -> list[str]:
         glob.glob(os.path.join(INCLUDE, "*.h"))
 
 
+# The GEMM kernels hand registers between warpgroups with setmaxnreg; the split is only valid
+# for the launch register count it was computed for (see gemm_sm100.cu), so the build refuses
+# any other count rather than produce a kernel whose setmaxnreg.inc could wait forever.
+GEMM_LAUNCH_REGS = 168
+
+
+def _check_register_split(ptxas_report: str) -> None:
+    entry = None
+    for line in ptxas_report.splitlines():
+        m = re.search(r"Compiling entry function '([^']+)'", line)
+        if m:
+            entry = m.group(1)
+            continue
+        m = re.search(r"Used (\d+) registers", line)
+        if m and entry and "k_gemm" in entry and int(m.group(1)) != GEMM_LAUNCH_REGS:
+            raise RuntimeError(f"{entry}: ptxas allocated {m.group(1)} registers, the warpgroup register "
+                               f"split needs exactly {GEMM_LAUNCH_REGS}")
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
     sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
@@ -50,15 +70,20 @@ def build(force: bool = False, verbose: bool = False) -> str:
         obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
         stale = force or not os.path.exists(obj) or os.path.getmtime(obj) < max(os.path.getmtime(src), newest_header)
         if stale:
-            cmd = [nvcc, *NVCC_FLAGS, "-c", src, "-o", obj]
+            cmd = [nvcc, "-Xptxas=-v", *NVCC_FLAGS, "-c", src, "-o", obj]
             if verbose:
-                cmd.insert(1, "-Xptxas=-v")
                 print(" ".join(cmd), flush=True)
             r = subprocess.run(cmd, capture_output=True, text=True)
             if r.returncode != 0:
                 raise RuntimeError(f"nvcc failed for {src}:\n{r.stdout}\n{r.stderr}")
-            if verbose and (r.stdout or r.stderr):
-                print(r.stdout + r.stderr, flush=True)
+            report = r.stdout + r.stderr
+            if verbose and report:
+                print(report, flush=True)
+            try:
+                _check_register_split(report)
+            except RuntimeError:
+                os.remove(obj)
+                raise
         return obj
 
     with ThreadPoolExecutor(max(1, min(len(sources), os.cpu_count() or 1))) as ex:

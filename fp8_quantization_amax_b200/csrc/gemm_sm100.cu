@@ -12,7 +12,10 @@
 //               swizzle) per K block into a 4-stage shared-memory ring.
 //   warp 1      allocates all 512 TMEM columns; lane 0 issues four tcgen05.mma (M128 N256 K32,
 //               kind::f8f6f4, fp32 accumulate) per K block.
-//   warps 2-9   promotion / epilogue.  Block-scaled: each K block's partial P_kb goes to one of
+//   warp 2      block-scaled path: copies each K block's A row scales and B scales (cp.async)
+//               into an 8-slot shared-memory ring for the epilogue.
+//   warp 3      idle (completes warpgroup 0, which hands its registers to the epilogue).
+//   warps 4-11  promotion / epilogue.  Block-scaled: each K block's partial P_kb goes to one of
 //               two 256-column TMEM buffers; while the tensor cores fill the other buffer, each
 //               thread loads its row's 128 columns (tcgen05.ld) and accumulates
 //               acc += (sA * sB) * P_kb in fp32 registers; at the end of the tile the
@@ -44,8 +47,20 @@ constexpr uint32_t kStageA = BM * BK;             // 16 KB of E4M3
 constexpr uint32_t kStageB = BN * BK;             // 32 KB
 constexpr uint32_t kStageBytes = kStageA + kStageB;
 constexpr int kEpiWarps = 8;
-constexpr int kThreads = 64 + 32 * kEpiWarps;     // producer, MMA, 8 epilogue warps
+constexpr int kFirstEpiWarp = 4;                  // warpgroup 0: producer, MMA, two idle warps
+constexpr int kThreads = 128 + 32 * kEpiWarps;    // three warpgroups
 constexpr uint32_t kTmemCols = 512;               // two 128 x 256 fp32 accumulators
+
+// Register split.  The kernel is launched with kLaunchRegs registers per thread (enforced by the
+// build, which checks ptxas' report): 384 x 168 = 64512.  Warpgroup 0 gives registers back and
+// the two epilogue warpgroups take them: 128 x 40 + 256 x 232 = 64512, the launch's total, so
+// setmaxnreg.inc always finds its registers.  Per SM sub-partition (one warp of each warpgroup):
+// 40 + 232 + 232 = 504 registers x 32 lanes = 16128 <= 16384.
+constexpr int kScaleSlots = 8;                    // scale ring depth (K blocks)
+constexpr int kLaunchRegs = 168;
+constexpr int kProducerRegs = 40;
+constexpr int kEpilogueRegs = 232;
+static_assert(128 * kProducerRegs + 256 * kEpilogueRegs == kThreads * kLaunchRegs, "register split must add up");
 
 // kind::f8f6f4 instruction descriptor: D fp32, A = B = E4M3, both K-major, N = 256, M = 128
 constexpr uint32_t kIdesc = (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(BN >> 3) << 17) |
@@ -117,6 +132,11 @@ template <bool PROMOTE>
 __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ CUtensorMap tA,
                                                       const __grid_constant__ CUtensorMap tB, Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // scale ring (block-scaled path): slot r holds the 128 row scales of A and the two column-half
+  // scales of B for one (tile, K block) pair, written by warp 2 and read by the epilogue
+  __shared__ float sc_a[PROMOTE ? kScaleSlots : 1][BM];
+  __shared__ float sc_b[PROMOTE ? kScaleSlots : 1][4];
+  __shared__ uint64_t sc_full[kScaleSlots], sc_empty[kScaleSlots];
   uint8_t* smem = smem_raw + (((smem_u32(smem_raw) + 1023u) & ~1023u) - smem_u32(smem_raw));
   uint8_t* sm_a = smem;                                   // kStages x 16 KB
   uint8_t* sm_b = smem + kStages * kStageA;               // kStages x 32 KB
@@ -136,6 +156,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ CU
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], kEpiWarps);
     }
+    for (int r = 0; r < kScaleSlots; ++r) {
+      mbar_init(&sc_full[r], 32);            // one arrival per lane of warp 2, on copy completion
+      mbar_init(&sc_empty[r], kEpiWarps);
+    }
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -150,6 +174,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ CU
   const uint32_t tmem_base = *tmem_slot;
   const int my_tiles = p.tiles > (int)blockIdx.x ? (p.tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
 
+  if (warp < kFirstEpiWarp) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0 && my_tiles > 0) {
@@ -228,88 +254,157 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ CU
       // all issued MMAs must complete before TMEM is released
       if (acc_use > 0) mbar_wait(&tfull[(acc_use - 1) & 1u], ((acc_use - 1) >> 1) & 1u, p.err);
     }
+  } else if (warp == 2 && PROMOTE) {
+    // ------------------------------------------------------------ scale producer
+    // For every (tile, K block) pair, lane l copies A's row scales 4l .. 4l+3 of the tile (zero
+    // beyond M) and lanes 0-1 B's scales of the two 128-column halves, all with cp.async, then
+    // every lane arrives on the slot's barrier once its copies have landed.
+    const int nkb = p.num_kb;
+    int r = 0;
+    uint32_t ph = 0, g = 0;
+    bool ok = true;
+    for (int k = 0; k < my_tiles && ok; ++k) {
+      int m0, n0;
+      tile_coords((int)blockIdx.x + k * (int)gridDim.x, p, &m0, &n0);
+      for (int kb = 0; kb < nkb; ++kb, ++g) {
+        if (g >= (uint32_t)kScaleSlots && !mbar_wait(&sc_empty[r], ph ^ 1u, p.err)) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int row = lane * 4 + i, m = m0 + row;
+          const float* src = p.gA_group ? p.sA + (size_t)kb * p.M + (m < p.M ? m : 0) : p.sA;
+          const uint32_t nbytes = (p.gA_group && m >= p.M) ? 0u : 4u;
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(&sc_a[r][row])), "l"(src),
+                       "r"(nbytes)
+                       : "memory");
+        }
+        if (lane < 2) {
+          const int ncol0 = n0 + lane * 128;
+          const float* src = p.gB_block ? p.sB + (size_t)((ncol0 < p.N ? ncol0 : 0) >> 7) * nkb + kb : p.sB;
+          const uint32_t nbytes = (p.gB_block && ncol0 >= p.N) ? 0u : 4u;
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(&sc_b[r][lane])), "l"(src),
+                       "r"(nbytes)
+                       : "memory");
+        }
+        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&sc_full[r]))
+                     : "memory");
+        if (++r == kScaleSlots) {
+          r = 0;
+          ph ^= 1u;
+        }
+      }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kEpilogueRegs));
     // ------------------------------------------------------------ promotion / epilogue
-    const int ew = warp - 2;                 // 0..7
+    const int ew = warp - kFirstEpiWarp;     // 0..7
     const int quarter = warp & 3;            // TMEM lane quarter this warp may access
     const int half = ew >> 2;                // column half: 128 columns each
     const int row_in_tile = quarter * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
     uint32_t acc_use = 0;
-    bool ok = true;
-    for (int k = 0; k < my_tiles && ok; ++k) {
-      int m0, n0;
-      tile_coords((int)blockIdx.x + k * (int)gridDim.x, p, &m0, &n0);
-      const int m = m0 + row_in_tile;
-      const int ncol0 = n0 + half * 128;
-      const bool row_ok = m < p.M;
-      const bool cols_ok = ncol0 < p.N;
-      float acc[128];
-      if (PROMOTE) {
+    if (PROMOTE) {
+      // Scales come from the ring filled by warp 2: one wait, two shared loads per K block.
+      const int nkb = p.num_kb;
+      const int total = my_tiles * nkb;
+      int r = 0;
+      uint32_t sph = 0;
+      float2 acc[64];
+      int kb = 0, k = 0;
+      for (int g = 0; g < total; ++g) {
+        if (kb == 0) {
 #pragma unroll
-        for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
-        const int nb = ncol0 / 128;
-        const int nbk = p.num_kb;
-        auto multiplier = [&](int kb) -> float {
-          const float a = p.gA_group ? (row_ok ? __ldg(p.sA + (size_t)kb * p.M + m) : 0.0f) : __ldg(p.sA);
-          const float b = p.gB_block ? (cols_ok ? __ldg(p.sB + (size_t)nb * nbk + kb) : 0.0f) : __ldg(p.sB);
-          return a * b;
-        };
-        float mult_next = multiplier(0);
-        for (int kb = 0; kb < p.num_kb; ++kb) {
-          const float mult = mult_next;
-          if (kb + 1 < p.num_kb) mult_next = multiplier(kb + 1);
-          const uint32_t buf = acc_use & 1u;
-          if (!mbar_wait(&tfull[buf], (acc_use >> 1) & 1u, p.err)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t taddr = tmem_base + lane_addr + buf * BN + half * 128;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t v[32];
-            tmem_ld32(taddr + c * 32, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) acc[c * 32 + j] = __fmaf_rn(mult, __uint_as_float(v[j]), acc[c * 32 + j]);
-          }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[buf]);
-          ++acc_use;
+          for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
         }
-        if (!ok) break;
-      } else {
+        if (!mbar_wait(&sc_full[r], sph, p.err)) break;
+        const float mult = sc_a[r][row_in_tile] * sc_b[r][half];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sc_empty[r]);
+        if (++r == kScaleSlots) {
+          r = 0;
+          sph ^= 1u;
+        }
+        const float2 mult2 = make_float2(mult, mult);
+        const uint32_t buf = acc_use & 1u;
+        if (!mbar_wait(&tfull[buf], (acc_use >> 1) & 1u, p.err)) break;
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + lane_addr + buf * BN + half * 128;
+#pragma unroll
+        for (int c = 0; c < 4; c += 2) {
+          uint32_t v[32], w[32];
+          tmem_ld32(taddr + c * 32, v);
+          tmem_ld32(taddr + c * 32 + 32, w);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            acc[c * 16 + i] =
+                __ffma2_rn(mult2, make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), acc[c * 16 + i]);
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            acc[c * 16 + 16 + i] = __ffma2_rn(
+                mult2, make_float2(__uint_as_float(w[2 * i]), __uint_as_float(w[2 * i + 1])), acc[c * 16 + 16 + i]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[buf]);
+        ++acc_use;
+        if (++kb == nkb) {
+          // tile done: round to bf16 and store this thread's row segment (256 bytes)
+          int m0, n0;
+          tile_coords((int)blockIdx.x + k * (int)gridDim.x, p, &m0, &n0);
+          const int m = m0 + row_in_tile;
+          const int ncol0 = n0 + half * 128;
+          if (m < p.M && ncol0 < p.N) {
+            uint16_t* dst = p.C + (size_t)m * p.N + ncol0;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              uint4 wv;
+              wv.x = f32x2_to_bf16x2(acc[c * 4 + 0].x, acc[c * 4 + 0].y);
+              wv.y = f32x2_to_bf16x2(acc[c * 4 + 1].x, acc[c * 4 + 1].y);
+              wv.z = f32x2_to_bf16x2(acc[c * 4 + 2].x, acc[c * 4 + 2].y);
+              wv.w = f32x2_to_bf16x2(acc[c * 4 + 3].x, acc[c * 4 + 3].y);
+              st_stream_v4(dst + c * 8, wv);
+            }
+          }
+          kb = 0;
+          ++k;
+        }
+      }
+    } else {
+      for (int k = 0; k < my_tiles; ++k) {
+        int m0, n0;
+        tile_coords((int)blockIdx.x + k * (int)gridDim.x, p, &m0, &n0);
+        const int m = m0 + row_in_tile;
+        const int ncol0 = n0 + half * 128;
         const uint32_t buf = acc_use & 1u;
         if (!mbar_wait(&tfull[buf], (acc_use >> 1) & 1u, p.err)) break;
         tc_fence_after();
         const float mult = __ldg(p.sA) * __ldg(p.sB);
         const uint32_t taddr = tmem_base + lane_addr + buf * BN + half * 128;
+        uint32_t out[64];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t v[32];
           tmem_ld32(taddr + c * 32, v);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) acc[c * 32 + j] = __fmul_rn(mult, __uint_as_float(v[j]));
+          for (int i = 0; i < 16; ++i)
+            out[c * 16 + i] = f32x2_to_bf16x2(__fmul_rn(mult, __uint_as_float(v[2 * i])),
+                                              __fmul_rn(mult, __uint_as_float(v[2 * i + 1])));
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[buf]);
         ++acc_use;
-      }
-      // round to bf16 and store this thread's row segment (256 bytes)
-      if (row_ok && cols_ok) {
-        uint16_t* dst = p.C + (size_t)m * p.N + ncol0;
+        if (m < p.M && ncol0 < p.N) {
+          uint16_t* dst = p.C + (size_t)m * p.N + ncol0;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          uint4 w;
-          w.x = f32x2_to_bf16x2(acc[c * 8 + 0], acc[c * 8 + 1]);
-          w.y = f32x2_to_bf16x2(acc[c * 8 + 2], acc[c * 8 + 3]);
-          w.z = f32x2_to_bf16x2(acc[c * 8 + 4], acc[c * 8 + 5]);
-          w.w = f32x2_to_bf16x2(acc[c * 8 + 6], acc[c * 8 + 7]);
-          st_stream_v4(dst + c * 8, w);
+          for (int c = 0; c < 16; ++c)
+            st_stream_v4(dst + c * 8, make_uint4(out[c * 4], out[c * 4 + 1], out[c * 4 + 2], out[c * 4 + 3]));
         }
       }
     }
