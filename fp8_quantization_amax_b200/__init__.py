@@ -21,7 +21,7 @@ __all__ = [
     "Fp8qError", "lib", "library_path", "device_status", "num_scales", "workspace_bytes", "kv_num_scales",
     "kv_workspace_bytes", "gemm_workspace_bytes", "scale_shape", "kv_scale_shape",
     "fp8_encode", "fp8_decode", "fp8_quantize", "fp8_dequantize", "fp8_kv_quantize",
-    "fp8_gemm_blockscaled",
+    "fp8_kv_quantize_noalloc", "fp8_gemm_blockscaled",
 ]
 
 E4M3, E5M2 = 0, 1
@@ -74,8 +74,9 @@ def lib() -> ctypes.CDLL:
             L.fp8_dequantize.argtypes = [vp, vp, i64, i64, i32, i32, vp, vp]
             L.fp8_kv_quantize.argtypes = [vp, vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, sz, vp]
             L.fp8_gemm_blockscaled.argtypes = [vp, vp, i32, vp, vp, i32, i64, i64, i64, vp, vp, sz, vp]
+            L.fp8_kv_quantize_noalloc.argtypes = [vp, vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp]
             for fn in ("fp8_encode", "fp8_decode", "fp8_quantize", "fp8_dequantize", "fp8_kv_quantize",
-                       "fp8_gemm_blockscaled"):
+                       "fp8_gemm_blockscaled", "fp8_kv_quantize_noalloc"):
                 getattr(L, fn).restype = i32
             _lib = L
     return _lib
@@ -244,6 +245,28 @@ def fp8_kv_quantize(k: torch.Tensor, v: torch.Tensor, fmt: int = E4M3, gran: int
                                _ptr(v_scales), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
                                _stream(dev))
     _check("fp8_kv_quantize", st)
+    return k_codes, v_codes, k_scales, v_scales
+
+
+def fp8_kv_quantize_noalloc(k: torch.Tensor, v: torch.Tensor, fmt: int = E4M3, gran: int = KV_PER_HEAD,
+                            k_codes=None, v_codes=None, k_scales=None, v_scales=None):
+    """fp8_kv_quantize for callers that cannot allocate device memory: the two-pass partial maxima
+    live in a fixed array inside the library (at most 32 heads for per-head scales).  Outputs
+    not passed in are allocated here only for convenience; pass them to allocate nothing."""
+    _dev(k, "k", torch.bfloat16)
+    _dev(v, "v", torch.bfloat16)
+    if k.dim() != 3 or k.shape != v.shape:
+        raise ValueError("k and v must both be [tokens][heads][head_dim]")
+    T, H, D = k.shape
+    dev = k.device
+    k_codes = torch.empty(k.shape, dtype=torch.uint8, device=dev) if k_codes is None else _dev(k_codes, "k_codes", torch.uint8)
+    v_codes = torch.empty(v.shape, dtype=torch.uint8, device=dev) if v_codes is None else _dev(v_codes, "v_codes", torch.uint8)
+    shp = kv_scale_shape(T, H, gran)
+    k_scales = torch.empty(shp, dtype=torch.float32, device=dev) if k_scales is None else _dev(k_scales, "k_scales", torch.float32)
+    v_scales = torch.empty(shp, dtype=torch.float32, device=dev) if v_scales is None else _dev(v_scales, "v_scales", torch.float32)
+    st = lib().fp8_kv_quantize_noalloc(_ptr(k), _ptr(v), T, H, D, fmt, gran, _ptr(k_codes), _ptr(v_codes),
+                                       _ptr(k_scales), _ptr(v_scales), _stream(dev))
+    _check("fp8_kv_quantize_noalloc", st)
     return k_codes, v_codes, k_scales, v_scales
 
 

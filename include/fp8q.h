@@ -182,6 +182,24 @@ FP8Q_API fp8q_status fp8_kv_quantize(const void *k, const void *v, int64_t token
                             float *k_scales, float *v_scales, void *ws, size_t ws_bytes,
                             fp8q_stream_t stream);
 
+/*
+ * fp8_kv_quantize without a workspace, for callers that cannot allocate device memory (an
+ * engine that owns all device memory up front, a latency-critical path where an allocation may
+ * stall or fail, a plug-in that receives tensors but has no way to request scratch).  The
+ * source pages have no counterpart to this entry point: it is a deployment convenience.
+ * Arguments, layouts and results are exactly those of fp8_kv_quantize without ws / ws_bytes.
+ * The partial maxima of the two-pass granularities live in a fixed 256 KB array inside the
+ * library, one per device that loads it, kept until the process exits; per-head quantization
+ * therefore supports at most 32 heads (more returns FP8Q_ERR_WORKSPACE).  The first call on a
+ * device looks up that array's device address (cudaGetSymbolAddress) with the device current,
+ * so make that first call before any stream capture.  All calls share the array: calls whose
+ * kernels can overlap on the GPU (e.g. on unordered streams) race on it and must not be made.
+ */
+FP8Q_API fp8q_status fp8_kv_quantize_noalloc(const void *k, const void *v, int64_t tokens, int64_t heads,
+                                             int64_t head_dim, fp8q_format f, fp8q_kv_granularity g,
+                                             uint8_t *k_codes, uint8_t *v_codes, float *k_scales,
+                                             float *v_scales, fp8q_stream_t stream);
+
 /* ---------------------------------------------------------------- GEMM */
 
 /*
