@@ -153,6 +153,24 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(inside), "window": window}
 
 
+# ------------------------------------------------------------------ cross-rank aggregation
+
+def reduce_max(value: float, device) -> float:
+    """Max of a per-rank scalar over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput_gbs(bytes_per_step: int, steps: int, world: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank's steps' bytes over the slowest rank's device time."""
+    return world * bytes_per_step * steps / (ms_max * 1e-3) / 1e9
+
+
 # ------------------------------------------------------------------ helpers
 
 def dev_bf16(a, device):
@@ -392,13 +410,9 @@ def our_arm(args):
         wall1 = time.time()
         barrier()
     sampler.stop()
-    ms_total = t_start.elapsed_time(t_end)
-    if world > 1:
-        tt = torch.tensor([ms_total], dtype=torch.float64, device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total = float(tt.item())
+    ms_total = reduce_max(t_start.elapsed_time(t_end), device)
     ms_step = ms_total / max(args.steps, 1)
-    value = world * step_bytes * args.steps / (ms_total * 1e-3) / 1e9
+    value = job_throughput_gbs(step_bytes, args.steps, world, ms_total)
     w_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_w[:used])
     x_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_x[:used])
     clocks = sampler.summary(wall0, wall1)
@@ -442,14 +456,10 @@ def our_arm(args):
         b.record(stream)
         torch.cuda.synchronize(device)
         barrier()
-    e2e_ms = a.elapsed_time(b)
-    if world > 1:
-        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = reduce_max(a.elapsed_time(b), device)
     h2d = (hw.numel() + hx.numel()) * 2
     d2h = hwc.numel() + hxc.numel() + (hws.numel() + hxs.numel()) * 4
-    e2e_value = world * step_bytes * e2e_steps / (e2e_ms * 1e-3) / 1e9
+    e2e_value = job_throughput_gbs(step_bytes, e2e_steps, world, e2e_ms)
 
     result = None
     if rank == 0:
