@@ -322,8 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ CU
         }
         if (!mbar_wait(&sc_full[r], sph, p.err)) break;
         const float mult = sc_a[r][row_in_tile] * sc_b[r][half];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sc_empty[r]);
+        const int r_used = r;
         if (++r == kScaleSlots) {
           r = 0;
           sph ^= 1u;
@@ -350,7 +349,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ CU
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[buf]);
+        if (lane == 0) {
+          mbar_arrive(&tempty[buf]);          // TMEM buffer drained
+          mbar_arrive(&sc_empty[r_used]);     // scale slot read (the loads were consumed above)
+        }
         ++acc_use;
         if (++kb == nkb) {
           // tile done: round to bf16 and store this thread's row segment (256 bytes)
