@@ -313,17 +313,59 @@ def supplementary(device, stream, peaks, flush):
         # GEMM (8B up-proj shape) on the quantized config-1 operands
         x = dev_bf16(synth.activations(seed=1), device)
         xc, xs = fq.fp8_quantize(x, fq.E4M3, fq.GROUP_1x128)
+        del x
+
+        def gemm_entry(m, n, k, ms, a, sa, wscale, c):
+            flops = 2.0 * m * n * k
+            nbytes = a.numel() + n * k + c.numel() * 2 + sa.numel() * 4 + wscale.numel() * 4
+            return {"us": round(ms * 1e3, 2), "TFLOP/s": round(flops / ms / 1e9, 1),
+                    "frac_fp8_peak": round(flops / ms / 1e9 / fp8_peak, 3),
+                    "GB/s": round(nbytes / ms / 1e6, 1), "frac_hbm": round(nbytes / ms / 1e6 / hbm, 3)}
+
         try:
-            for m, name in ((8192, "gemm_8b_up_m8192"), (16, "gemm_8b_up_m16")):
-                a, sa = xc[:m].contiguous(), xs[:, :m].contiguous()
-                cbuf = torch.empty((m, W_SHAPE[0]), dtype=torch.bfloat16, device=device)
-                fq.fp8_gemm_blockscaled(a, sa, wc, ws, out=cbuf)
-                ms = timed(lambda: fq.fp8_gemm_blockscaled(a, sa, wc, ws, out=cbuf), 10, stream, flush)
-                flops = 2.0 * m * W_SHAPE[0] * W_SHAPE[1]
-                nbytes = a.numel() + wc.numel() + cbuf.numel() * 2 + sa.numel() * 4 + ws.numel() * 4
-                out[name] = {"us": round(ms * 1e3, 2), "TFLOP/s": round(flops / ms / 1e9, 1),
-                             "frac_fp8_peak": round(flops / ms / 1e9 / fp8_peak, 3),
-                             "GB/s": round(nbytes / ms / 1e6, 1)}
+            # prefill: one call per timing, L2 flushed before each
+            m = 8192
+            a, sa = xc[:m].contiguous(), xs[:, :m].contiguous()
+            cbuf = torch.empty((m, W_SHAPE[0]), dtype=torch.bfloat16, device=device)
+            fq.fp8_gemm_blockscaled(a, sa, wc, ws, out=cbuf)
+            ms = timed(lambda: fq.fp8_gemm_blockscaled(a, sa, wc, ws, out=cbuf), 10, stream, flush)
+            out["gemm_8b_up_m8192"] = gemm_entry(m, W_SHAPE[0], W_SHAPE[1], ms, a, sa, ws, cbuf)
+            del cbuf
+            # decode: back-to-back calls as in a decode step, each on one of four copies of the
+            # weight codes (4 x 58.7 MB > L2), so every call streams its weights from HBM
+            m = 16
+            a, sa = xc[:m].contiguous(), xs[:, :m].contiguous()
+            cbuf = torch.empty((m, W_SHAPE[0]), dtype=torch.bfloat16, device=device)
+            copies = [wc.clone() for _ in range(4)]
+            calls = 32
+            fq.fp8_gemm_blockscaled(a, sa, copies[0], ws, out=cbuf)
+
+            def batch():
+                for i in range(calls):
+                    fq.fp8_gemm_blockscaled(a, sa, copies[i % 4], ws, out=cbuf)
+
+            ms = timed(batch, 5, stream, flush) / calls
+            out["gemm_8b_up_m16"] = gemm_entry(m, W_SHAPE[0], W_SHAPE[1], ms, a, sa, ws, cbuf)
+            out["gemm_8b_up_m16"]["timing"] = f"{calls} back-to-back calls over 4 weight copies, mean per call"
+            del copies, cbuf
+            # decode on the 70B up-projection (one weight, 235 MB > L2)
+            w70 = dev_bf16(synth.weight_70b(seed=4, which="up"), device)
+            b70, s70 = fq.fp8_quantize(w70, fq.E4M3, fq.BLOCK_128x128)
+            del w70
+            x70 = dev_bf16(synth.activations_70b(seed=4, m=64, which="up"), device)
+            a70, sa70 = fq.fp8_quantize(x70, fq.E4M3, fq.GROUP_1x128)
+            c70 = torch.empty((64, b70.shape[0]), dtype=torch.bfloat16, device=device)
+            fq.fp8_gemm_blockscaled(a70, sa70, b70, s70, out=c70)
+            calls = 8
+
+            def batch70():
+                for _ in range(calls):
+                    fq.fp8_gemm_blockscaled(a70, sa70, b70, s70, out=c70)
+
+            ms = timed(batch70, 5, stream, flush) / calls
+            out["gemm_70b_up_m64"] = gemm_entry(64, b70.shape[0], b70.shape[1], ms, a70, sa70, s70, c70)
+            out["gemm_70b_up_m64"]["timing"] = f"{calls} back-to-back calls (weight 235 MB > L2), mean per call"
+            del b70, s70, a70, sa70, c70
         except fq.Fp8qError as err:
             out["gemm"] = f"not measured: {err}"
     return out

@@ -83,8 +83,15 @@ def lib() -> ctypes.CDLL:
 
 
 def device_status() -> int:
-    """Synchronize the device; return and clear the kernels' error bits (0 = none)."""
-    return int(lib().fp8q_device_status())
+    """Synchronize the device; return and clear the kernels' error bits (0 = none).
+
+    Bit 0: a bounded wait inside a kernel gave up.  Bit 1: a GEMM workspace counter was not
+    zero on entry.  After any error the cached GEMM workspaces are dropped (a kernel that ended
+    early may have left counters behind)."""
+    status = int(lib().fp8q_device_status())
+    if status:
+        _gemm_ws.clear()
+    return status
 
 
 def _status_string(status: int) -> str:
@@ -169,6 +176,22 @@ def _workspace(nbytes: int, device, ws: torch.Tensor | None) -> torch.Tensor | N
     if ws is None:
         return torch.empty(nbytes, dtype=torch.uint8, device=device)
     return ws
+
+
+# GEMM workspaces must be zero-filled before their first use and every successful call leaves
+# them zero again, so one zeroed buffer per (device, stream) is kept and grown on demand.
+_gemm_ws: dict = {}
+
+
+def _gemm_workspace(nbytes: int, device) -> torch.Tensor | None:
+    if nbytes == 0:
+        return None
+    key = (device.index, torch.cuda.current_stream(device).cuda_stream)
+    buf = _gemm_ws.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
+        _gemm_ws[key] = buf
+    return buf
 
 
 # ------------------------------------------------------------------ codec
@@ -275,7 +298,11 @@ def fp8_kv_quantize_noalloc(k: torch.Tensor, v: torch.Tensor, fmt: int = E4M3, g
 def fp8_gemm_blockscaled(a: torch.Tensor, sa: torch.Tensor, b: torch.Tensor, sb: torch.Tensor,
                          ga: int = GROUP_1x128, gb: int = BLOCK_128x128, out: torch.Tensor | None = None,
                          ws: torch.Tensor | None = None) -> torch.Tensor:
-    """C[M][N] (bf16) = block-scaled FP8 product of A [M][K] and B [N][K] (E4M3 codes, K-major)."""
+    """C[M][N] (bf16) = block-scaled FP8 product of A [M][K] and B [N][K] (E4M3 codes, K-major).
+
+    Decode shapes (M <= 64) need a workspace.  Without `ws` a zero-filled buffer kept per
+    (device, stream) is used; a caller-provided `ws` must be zero-filled before its first use
+    (every successful call leaves it zero) and not shared by calls that may overlap."""
     _dev(a, "a", torch.uint8)
     _dev(b, "b", torch.uint8)
     _dev(sa, "sa", torch.float32)
@@ -285,8 +312,13 @@ def fp8_gemm_blockscaled(a: torch.Tensor, sa: torch.Tensor, b: torch.Tensor, sb:
     if K != K2:
         raise ValueError("a and b disagree on K")
     out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device) if out is None else _dev(out, "out", torch.bfloat16)
-    ws = _workspace(gemm_workspace_bytes(M, N, K), a.device, ws)
+    need = gemm_workspace_bytes(M, N, K)
+    cached = ws is None
+    if cached:
+        ws = _gemm_workspace(need, a.device)
     st = lib().fp8_gemm_blockscaled(_ptr(a), _ptr(sa), ga, _ptr(b), _ptr(sb), gb, M, N, K, _ptr(out), _ptr(ws),
                                     0 if ws is None else ws.numel() * ws.element_size(), _stream(a.device))
+    if st != 0 and cached:
+        _gemm_ws.clear()
     _check("fp8_gemm_blockscaled", st)
     return out

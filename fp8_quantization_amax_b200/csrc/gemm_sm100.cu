@@ -423,14 +423,421 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ CU
 
 constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + (2 * kStages + 4) * sizeof(uint64_t) + 16;
 
+
+// ============================================================================ decode shapes
+//
+// For M <= 64 (decode) the tile walk above would leave most SMs idle and waste the MMA's
+// 128-row side on padding.  Here the operands swap roles: the weights' 128-row tile is the
+// MMA's M side and the tokens (M rounded up to 16) its N side, so each MMA computes
+// P^T[n][m] for 128 weight rows.  The (weight tile, K block) units are split evenly and
+// contiguously over all CTAs (a CTA's range may cross tile boundaries); each CTA promotes its
+// units per K block (acc[m] += sB[tile][kb] * sA[kb][m] * P^T[n][m], thread = weight row n).
+// A tile that lies wholly in one CTA's range is rounded to bf16 and stored directly.  A tile
+// shared by several CTAs: each writes its fp32 partial to the workspace and counts itself in on
+// the tile's counter; the CTA that completes the count adds the partials in ascending CTA order
+// (deterministic: the same sum whichever CTA finishes last), stores the tile and resets the
+// counter to zero, so the workspace is zero again after every call.
+//   warp 0 TMA producer, warp 1 MMA issuer (four TMEM buffers), warp 2 scale producer,
+//   warps 3-6 promotion.
+namespace dec {
+
+constexpr int BM = 128;                 // weight rows per tile (the MMA's M)
+constexpr int kThreads = 32 * 7;
+constexpr int kTBuf = 4;                // TMEM buffers of kMaxMp columns
+constexpr int kMaxMp = 64;
+constexpr uint32_t kTmemCols = kTBuf * kMaxMp;
+constexpr int kScaleSlots = 8;
+constexpr uint32_t kStageW = BM * BK;   // 16 KB of weight codes
+constexpr int kMaxStages = 10;
+
+struct Params {
+  int M, N, K, nkb;
+  uint32_t W;         // units: N / 128 tiles x nkb K blocks
+  int G;              // CTAs
+  int maxseg;         // most tile segments any CTA touches
+  const float* sA;
+  const float* sB;
+  int gA_group, gB_block;
+  uint32_t* counters; // [N / 128]: segments counted in per tile; zero between calls
+  float* partials;    // [G][maxseg][Mp][128]
+  uint16_t* C;
+  int stages;
+  uint32_t stage_bytes;
+  uint32_t* err;
+};
+
+// first unit of CTA c when W units are split over G CTAs (W * G < 2^32, checked by the planner)
+__host__ __device__ __forceinline__ uint32_t range_lo(uint32_t c, uint32_t W, uint32_t G) { return (c * W) / G; }
+
+// the CTA whose range holds unit u
+__host__ __device__ __forceinline__ uint32_t cta_of(uint32_t u, uint32_t W, uint32_t G) {
+  uint32_t c = (u * G) / W;
+  while (c > 0 && range_lo(c, W, G) > u) --c;
+  while (c + 1 < G && range_lo(c + 1, W, G) <= u) ++c;
+  return c;
+}
+
+template <int MP>
+__global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constant__ CUtensorMap tW,
+                                                             const __grid_constant__ CUtensorMap tX, Params p) {
+  constexpr uint32_t kIdescD = (1u << 4) | ((uint32_t)(MP >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ float sc_a[kScaleSlots][MP];
+  __shared__ float sc_b[kScaleSlots];
+  __shared__ uint64_t bars[2 * kMaxStages + 2 * kTBuf + 2 * kScaleSlots + 2];
+  __shared__ uint32_t tmem_slot;
+  __shared__ uint32_t s_last;
+  uint8_t* smem = smem_raw + (((smem_u32(smem_raw) + 1023u) & ~1023u) - smem_u32(smem_raw));
+  const int S = p.stages;
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kMaxStages;
+  uint64_t* tfull = bars + 2 * kMaxStages;
+  uint64_t* tempty = tfull + kTBuf;
+  uint64_t* sfull = tempty + kTBuf;
+  uint64_t* sempty = sfull + kScaleSlots;
+  uint64_t* seg_written = sempty + kScaleSlots;   // the four promotion warps' partials are out
+  uint64_t* seg_decided = seg_written + 1;        // the tile's counter has been bumped
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t lo = range_lo(blockIdx.x, p.W, p.G), hi = range_lo(blockIdx.x + 1, p.W, p.G);
+  const uint32_t n_units = hi - lo;
+  const int nkb = p.nkb;
+  if (warp == 0 && lane == 0) {
+    // the weights are read once: start their first tiles towards L2 before waiting on the
+    // previous grid (a prefetch only warms L2, which stays coherent with any later write)
+    tma_prefetch_desc(&tW);
+    tma_prefetch_desc(&tX);
+    for (uint32_t i = 0; i < n_units && i < (uint32_t)S; ++i) {
+      const uint32_t u = lo + i, t = u / nkb;
+      tma_prefetch_l2_2d(&tW, (int32_t)((u - t * nkb) * BK), (int32_t)(t * BM));
+    }
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(seg_written, 4);
+    mbar_init(seg_decided, 1);
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int b = 0; b < kTBuf; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    for (int r = 0; r < kScaleSlots; ++r) {
+      mbar_init(&sfull[r], 32);
+      mbar_init(&sempty[r], 4);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_slot;
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  if (warp == 0) {
+    if (lane == 0 && n_units > 0) {
+      int s = 0;
+      uint32_t ph = 0, i = 0;
+      for (; i < n_units; ++i) {
+        const uint32_t u = lo + i, t = u / nkb, kb = u - t * nkb;
+        if (i >= (uint32_t)S && !mbar_wait(&empty[s], ph ^ 1u, p.err)) break;
+        uint8_t* st = smem + s * p.stage_bytes;
+        mbar_arrive_expect_tx(&full[s], p.stage_bytes);
+        tma_load_2d(st, &tW, (int32_t)(kb * BK), (int32_t)(t * BM), &full[s]);
+        tma_load_2d(st + kStageW, &tX, (int32_t)(kb * BK), 0, &full[s]);
+        if (++s == S) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+      for (uint32_t j = 0; j < (uint32_t)S && j < i; ++j) {
+        const uint32_t kk = i - 1 - j;
+        mbar_wait(&full[kk % S], (kk / S) & 1u, p.err);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && n_units > 0) {
+      int s = 0;
+      uint32_t ph = 0, i = 0;
+      for (; i < n_units; ++i) {
+        const uint32_t buf = i % kTBuf;
+        if (i >= (uint32_t)kTBuf) {
+          if (!mbar_wait(&tempty[buf], ((i / kTBuf) - 1) & 1u, p.err)) break;
+          tc_fence_after();
+        }
+        if (!mbar_wait(&full[s], ph, p.err)) break;
+        tc_fence_after();
+        const uint8_t* st = smem + s * p.stage_bytes;
+        const uint64_t adesc = umma_desc_sw128(smem_u32(st));
+        const uint64_t bdesc = umma_desc_sw128(smem_u32(st + kStageW));
+#pragma unroll
+        for (int kk = 0; kk < BK / 32; ++kk)
+          umma_f8(tmem_base + buf * kMaxMp, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), kIdescD,
+                  kk > 0 ? 1u : 0u);
+        umma_commit(&empty[s]);
+        umma_commit(&tfull[buf]);
+        if (++s == S) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+      if (i > 0) mbar_wait(&tfull[(i - 1) % kTBuf], ((i - 1) / kTBuf) & 1u, p.err);
+    }
+  } else if (warp == 2) {
+    // scale producer: the K block's activation scales (one per token, zero beyond M) and the
+    // tile's weight scale, copied with cp.async into a ring slot
+    uint32_t r = 0, ph = 0;
+    for (uint32_t i = 0; i < n_units; ++i) {
+      const uint32_t u = lo + i, t = u / nkb, kb = u - t * nkb;
+      if (i >= (uint32_t)kScaleSlots && !mbar_wait(&sempty[r], ph ^ 1u, p.err)) break;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int m = lane * 2 + h;
+        if (m < MP) {
+          const float* src = p.gA_group ? p.sA + (size_t)kb * p.M + (m < p.M ? m : 0) : p.sA;
+          const uint32_t nbytes = (p.gA_group && m >= p.M) ? 0u : 4u;
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(&sc_a[r][m])), "l"(src),
+                       "r"(nbytes)
+                       : "memory");
+        }
+      }
+      if (lane == 0) {
+        const float* src = p.gB_block ? p.sB + (size_t)t * nkb + kb : p.sB;
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(&sc_b[r])), "l"(src) : "memory");
+      }
+      asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&sfull[r])) : "memory");
+      if (++r == kScaleSlots) {
+        r = 0;
+        ph ^= 1u;
+      }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+  } else {
+    // promotion: thread = weight row (TMEM lane) of the tile, MP accumulators (one per token)
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+    float acc[MP];
+#pragma unroll
+    for (int m = 0; m < MP; ++m) acc[m] = 0.0f;
+    uint32_t r = 0, sph = 0, seg_k = 0;
+    const uint32_t first_tile = lo / nkb;
+    for (uint32_t i = 0; i < n_units; ++i) {
+      const uint32_t u = lo + i, t = u / nkb;
+      const uint32_t buf = i % kTBuf;
+      if (!mbar_wait(&sfull[r], sph, p.err)) break;
+      if (!mbar_wait(&tfull[buf], (i / kTBuf) & 1u, p.err)) break;
+      tc_fence_after();
+      const float sb = sc_b[r];
+      uint32_t v[MP];
+#pragma unroll
+      for (int c = 0; c < MP / 16; ++c) {
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+            "%14, %15}, [%16];"
+            : "=r"(v[c * 16 + 0]), "=r"(v[c * 16 + 1]), "=r"(v[c * 16 + 2]), "=r"(v[c * 16 + 3]),
+              "=r"(v[c * 16 + 4]), "=r"(v[c * 16 + 5]), "=r"(v[c * 16 + 6]), "=r"(v[c * 16 + 7]),
+              "=r"(v[c * 16 + 8]), "=r"(v[c * 16 + 9]), "=r"(v[c * 16 + 10]), "=r"(v[c * 16 + 11]),
+              "=r"(v[c * 16 + 12]), "=r"(v[c * 16 + 13]), "=r"(v[c * 16 + 14]), "=r"(v[c * 16 + 15])
+            : "r"(tmem_base + lane_addr + buf * kMaxMp + c * 16));
+      }
+      tmem_ld_wait();
+#pragma unroll
+      for (int m = 0; m < MP; ++m) acc[m] = __fmaf_rn(sc_a[r][m] * sb, __uint_as_float(v[m]), acc[m]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&tempty[buf]);
+        mbar_arrive(&sempty[r]);
+      }
+      if (++r == kScaleSlots) {
+        r = 0;
+        sph ^= 1u;
+      }
+      if (u + 1 == hi || (u + 1) % nkb == 0) {
+        // this CTA's segment of tile t ends
+        const uint32_t c_first = cta_of(t * nkb, p.W, p.G), c_last = cta_of(t * nkb + nkb - 1, p.W, p.G);
+        bool finish = c_first == c_last;   // the whole tile is this CTA's
+        if (!finish) {
+          // publish this row's partial ([m][row] layout, coalesced over rows), then count the
+          // segment in; the CTA that brings the count to the number of contributors adds them up
+          float* dst = p.partials + ((size_t)(blockIdx.x * p.maxseg + (t - first_tile)) * MP) * BM + row;
+#pragma unroll
+          for (int m = 0; m < MP; ++m) dst[(size_t)m * BM] = acc[m];
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(seg_written);
+          if (warp == 3 && lane == 0) {
+            const bool ok = mbar_wait(seg_written, seg_k & 1u, p.err);
+            uint32_t last = 0;
+            if (ok) {
+              __threadfence();
+              const uint32_t n_contrib = c_last - c_first + 1;
+              const uint32_t old = atomicAdd(p.counters + t, 1u);
+              if (old >= n_contrib) raise_device_error(p.err, kErrWorkspaceDirty);
+              last = old + 1 == n_contrib;
+              if (last) p.counters[t] = 0;   // every contributor has counted in: leave it zero
+            }
+            s_last = last;
+            mbar_arrive(seg_decided);
+          }
+          if (!mbar_wait(seg_decided, seg_k & 1u, p.err)) break;
+          ++seg_k;
+          finish = s_last != 0;
+          if (finish) {
+            // sum the tile's partials in ascending CTA order (this CTA's own included: each
+            // thread re-reads the row it wrote), so the result does not depend on which CTA
+            // finishes last
+            __threadfence();
+#pragma unroll
+            for (int m = 0; m < MP; ++m) acc[m] = 0.0f;
+#pragma unroll 1
+            for (uint32_t c = c_first; c <= c_last; ++c) {
+              const uint32_t clo = range_lo(c, p.W, p.G);
+              const float* src = p.partials + ((size_t)(c * (uint32_t)p.maxseg + (t - clo / nkb)) * MP) * BM + row;
+#pragma unroll
+              for (int m0 = 0; m0 < MP; m0 += 16) {
+                float part[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) part[j] = __ldcg(src + (size_t)(m0 + j) * BM);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) acc[m0 + j] += part[j];
+              }
+            }
+          }
+        }
+        if (finish) {
+          uint16_t* out = p.C + (size_t)t * BM + row;
+          const size_t ldc = (size_t)p.N;
+#pragma unroll
+          for (int m = 0; m < MP; ++m) {
+            if (m < p.M) *out = (uint16_t)(f32x2_to_bf16x2(acc[m], 0.0f) & 0xFFFFu);
+            out += ldc;
+          }
+        }
+#pragma unroll
+        for (int m = 0; m < MP; ++m) acc[m] = 0.0f;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+}  // namespace dec
 }  // namespace gemm
 
-size_t gemm_workspace_bytes(int64_t, int64_t, int64_t) { return 0; }
+namespace {
+
+// decode plan: CTAs, segments per CTA and workspace bytes for M <= 64
+struct DecodePlan {
+  int mp = 0, G = 0, maxseg = 0;
+  uint32_t W = 0;
+  size_t ws_bytes = 0, counter_bytes = 0;
+};
+
+DecodePlan decode_plan(int64_t M, int64_t N, int64_t K) {
+  DecodePlan d;
+  if (M <= 0 || M > gemm::dec::kMaxMp || N % 128 != 0 || K % 128 != 0 || N == 0 || K == 0) return d;
+  d.mp = (int)((M + 15) / 16 * 16);
+  const int64_t nkb = K / 128, tiles = N / 128;
+  if ((uint64_t)tiles * nkb * (uint64_t)std::max(1, device_sm_count()) >= (1ull << 32)) return d;
+  d.W = (uint32_t)(tiles * nkb);
+  d.G = (int)std::min<int64_t>(device_sm_count(), d.W);
+  for (int c = 0; c < d.G; ++c) {
+    const uint32_t lo = gemm::dec::range_lo(c, d.W, d.G), hi = gemm::dec::range_lo(c + 1, d.W, d.G);
+    if (hi > lo) d.maxseg = std::max<int>(d.maxseg, (int)((hi - 1) / nkb - lo / nkb + 1));
+  }
+  d.counter_bytes = ((size_t)tiles * sizeof(uint32_t) + 255) / 256 * 256;
+  d.ws_bytes = d.counter_bytes + (size_t)d.G * d.maxseg * d.mp * gemm::dec::BM * sizeof(float);
+  return d;
+}
+
+template <int MP>
+cudaError_t launch_decode(const CUtensorMap& mW, const CUtensorMap& mX, gemm::dec::Params& p, cudaStream_t st) {
+  using namespace gemm::dec;
+  const size_t smem = 1024 + (size_t)p.stages * p.stage_bytes;
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(k_decode_mma<MP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    attr = true;
+  }
+  // a programmatic dependent of what precedes it on the stream: its set-up (and the L2 prefetch
+  // of the first weight tiles) overlaps that grid's tail; griddepcontrol.wait orders every
+  // load and store of operands, scales, workspace and output after it
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)p.G);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_decode_mma<MP>, mW, mX, p);
+}
+
+cudaError_t launch_decode_gemm(const DecodePlan& plan, const uint8_t* A, const float* sA, int gA, const uint8_t* B,
+                               const float* sB, int gB, int64_t M, int64_t N, int64_t K, uint16_t* C, void* ws,
+                               size_t ws_bytes, cudaStream_t st) {
+  using namespace gemm::dec;
+  using gemm::BK;
+  if (!ws || ws_bytes < plan.ws_bytes) return cudaErrorInvalidValue;
+  CUtensorMap mW, mX;
+  std::memset(&mW, 0, sizeof(mW));
+  std::memset(&mX, 0, sizeof(mX));
+  if (!make_tmap_2d(&mW, 1, B, (uint64_t)K, (uint64_t)N, (uint64_t)K, BK, BM, 1)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&mX, 1, A, (uint64_t)K, (uint64_t)M, (uint64_t)K, BK, (uint32_t)plan.mp, 1))
+    return cudaErrorInvalidValue;
+  gemm::dec::Params d;
+  d.M = (int)M;
+  d.N = (int)N;
+  d.K = (int)K;
+  d.nkb = (int)(K / BK);
+  d.W = plan.W;
+  d.G = plan.G;
+  d.maxseg = plan.maxseg;
+  d.sA = sA;
+  d.sB = sB;
+  d.gA_group = gA == 1;
+  d.gB_block = gB == 2;
+  d.counters = static_cast<uint32_t*>(ws);
+  d.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + plan.counter_bytes);
+  d.C = C;
+  d.stage_bytes = kStageW + (uint32_t)plan.mp * BK;
+  d.stages = (int)std::max<uint32_t>(2, std::min<uint32_t>(kMaxStages, (200u * 1024u) / d.stage_bytes));
+  d.err = device_error_word();
+  switch (plan.mp) {
+    case 16: return launch_decode<16>(mW, mX, d, st);
+    case 32: return launch_decode<32>(mW, mX, d, st);
+    case 48: return launch_decode<48>(mW, mX, d, st);
+    default: return launch_decode<64>(mW, mX, d, st);
+  }
+}
+
+}  // namespace
+
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) { return decode_plan(M, N, K).ws_bytes; }
 
 cudaError_t launch_gemm(const uint8_t* A, const float* sA, int gA, const uint8_t* B, const float* sB, int gB,
-                        int64_t M, int64_t N, int64_t K, uint16_t* C, void*, size_t, cudaStream_t st) {
+                        int64_t M, int64_t N, int64_t K, uint16_t* C, void* ws, size_t ws_bytes, cudaStream_t st) {
   using namespace gemm;
   if (M == 0 || N == 0) return cudaSuccess;
+  const DecodePlan plan = decode_plan(M, N, K);
+  if (plan.mp > 0) return launch_decode_gemm(plan, A, sA, gA, B, sB, gB, M, N, K, C, ws, ws_bytes, st);
   CUtensorMap mA, mB;
   std::memset(&mA, 0, sizeof(mA));
   std::memset(&mB, 0, sizeof(mB));

@@ -18,6 +18,8 @@ namespace fp8q {
 // Device error word (bit flags); kernels receive its address, the host reads and clears it
 // through fp8q_device_status().
 constexpr uint32_t kErrWaitTimeout = 1u;
+// a workspace counter held a value no call leaves behind (workspace not zero-filled)
+constexpr uint32_t kErrWorkspaceDirty = 2u;
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 
@@ -94,6 +96,14 @@ __device__ __forceinline__ void release_stage(uint64_t* empty_bar, int lane) {
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// Hint: pull one box of a 2-D tensor into L2 (no shared memory, no completion to wait for).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y)
+               : "memory");
 }
 
 // 2-D tiled load of one box into shared memory; completion counted on `bar` in bytes.

@@ -105,8 +105,9 @@ FP8Q_API int fp8q_version(void);
 /*
  * Synchronizes the current device, returns the library's device error bits and clears them.
  * 0: no error.  Bit 0: a bounded wait inside a kernel (a pipeline barrier that never completed)
- * gave up after its time limit, so that kernel's outputs are incomplete.  0xFFFFFFFF: the
- * device could not be queried (e.g. an earlier fault).
+ * gave up after its time limit, so that kernel's outputs are incomplete.  Bit 1: a GEMM
+ * workspace was not zero-filled (see fp8_gemm_blockscaled), so some output tiles were not
+ * written.  0xFFFFFFFF: the device could not be queried (e.g. an earlier fault).
  */
 FP8Q_API uint32_t fp8q_device_status(void);
 
@@ -211,8 +212,17 @@ FP8Q_API fp8q_status fp8_kv_quantize_noalloc(const void *k, const void *v, int64
  *   B   E4M3 codes [N][K] (K-major, W in R^{N x K});
  *       sB: gB = FP8Q_BLOCK_128x128 ([N/128][K/128]) or FP8Q_PER_TENSOR ([1])
  *   C   bf16 [M][N] (device, written)
- * When both are per-tensor the product is accumulated over all of K and scaled once
- * at the end: C = bf16(sA * sB * sum_k a*b).
+ * When both are per-tensor and M > 64 the product is accumulated over all of K and
+ * scaled once at the end: C = bf16(sA * sB * sum_k a*b).
+ * Decode shapes (M <= 64) split the (128-row weight tile, K block) pairs evenly over the SMs;
+ * per-tensor scales are then applied per K block.  A tile shared by several SMs has its fp32
+ * partial sums added in a fixed order, so results are deterministic.  ws: caller-owned device
+ * memory of at least fp8q_gemm_workspace_bytes(M, N, K) bytes, 16-byte aligned (else
+ * FP8Q_ERR_WORKSPACE), which must be ZERO-FILLED before its first use; every call that runs
+ * to completion leaves it zero-filled again, so it can be reused as is.  After a device error
+ * (fp8q_device_status() != 0) zero it again.  Calls that may run concurrently (e.g. on
+ * unordered streams) need separate workspaces.  A counter found non-zero raises device error
+ * bit 1 and leaves the affected output tiles unwritten.
  * Requirements: M >= 1; N % 128 == 0; K % 128 == 0 (else FP8Q_ERR_UNSUPPORTED);
  * A, B, C 16-byte aligned.  ws may be NULL when fp8q_gemm_workspace_bytes() is 0.
  */

@@ -58,6 +58,10 @@ def test_sizes(L):
     assert fq.kv_num_scales(131072, 8, fq.KV_PER_TENSOR) == 1
     assert fq.kv_workspace_bytes(131072, 8, 128, fq.KV_PER_HEAD_TOK128) == 0
     assert fq.kv_workspace_bytes(131072, 8, 128, fq.KV_PER_HEAD) >= fq.kv_workspace_bytes(131072, 8, 128, fq.KV_PER_TENSOR)
+    # decode shapes (M <= 64) keep fp32 partial sums in the workspace; larger M needs none
+    assert fq.gemm_workspace_bytes(16, 14336, 4096) >= 16 * 14336 * 4
+    assert fq.gemm_workspace_bytes(64, 128, 128) == 256 + 64 * 128 * 4     # tile counters + one partial
+    assert fq.gemm_workspace_bytes(65, 14336, 4096) == 0
 
 
 P = ctypes.c_void_p
@@ -107,6 +111,7 @@ def test_gemm_rejects(L):
     assert L.fp8_gemm_blockscaled(a, a, 1, a, a, 1, 128, 128, 128, a, None, 0, None) == 1      # gB
     assert L.fp8_gemm_blockscaled(MISALIGNED, a, 1, a, a, 2, 128, 128, 128, a, None, 0, None) == 1
     assert L.fp8_gemm_blockscaled(a, a, 1, a, a, 2, 0, 128, 128, a, None, 0, None) == 0
+    assert L.fp8_gemm_blockscaled(a, a, 1, a, a, 2, 16, 128, 128, a, None, 0, None) == 3        # no workspace
 
 
 def test_binding_refuses_cpu_tensors():

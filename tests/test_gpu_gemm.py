@@ -107,6 +107,56 @@ def test_gemm_block_scale_selection(orc):
     check_tolerance(got, ref, "single block")
 
 
+@pytest.mark.parametrize("ga,gb", [(1, 2), (0, 0)])
+@pytest.mark.parametrize("M", [1, 7, 16, 33, 48, 64, 65])
+@pytest.mark.parametrize("NK", [(128, 128), (384, 640), (1024, 4096), (2048, 1280)])
+def test_gemm_decode_split(orc, ga, gb, M, NK):
+    """Decode shapes (M <= 64) split the (weight tile, K block) units over all SMs; these N, K
+    give ranges that start and end inside tiles, a tile spread over several CTAs and a single
+    unit.  M = 65 is the first shape past the split path."""
+    N, K = NK
+    a, sa, b, sb = operands(orc, M, N, K, ga, gb, seed=7 * M + N + K)
+    got = run_gpu(a, sa, b, sb, ga, gb)
+    ref = orc.gemm_rows(a, sa, ga, b, sb, gb, np.arange(M))
+    check_tolerance(got, ref, f"M={M} N={N} K={K} gA={ga} gB={gb}")
+
+
+def test_gemm_decode_deterministic(orc):
+    """The split path adds a tile's partial sums in a fixed order: two runs agree bit for bit."""
+    M, N, K = 16, 2048, 4096
+    a, sa, b, sb = operands(orc, M, N, K, 1, 2, seed=11)
+    args = (dev(a), dev(sa), dev(b), dev(sb), 1, 2)
+    first = fq.fp8_gemm_blockscaled(*args)
+    second = fq.fp8_gemm_blockscaled(*args)
+    torch.cuda.synchronize()
+    assert torch.equal(first.view(torch.int16), second.view(torch.int16))
+
+
+def test_gemm_decode_workspace_left_zero(orc):
+    """A caller-provided zero-filled workspace: the per-tile counters are zero again afterwards,
+    so the same workspace serves the next call."""
+    M, N, K = 16, 2048, 4096
+    a, sa, b, sb = operands(orc, M, N, K, 1, 2, seed=12)
+    ws = torch.zeros(fq.gemm_workspace_bytes(M, N, K), dtype=torch.uint8, device="cuda")
+    args = (dev(a), dev(sa), dev(b), dev(sb), 1, 2)
+    ref = orc.gemm_rows(a, sa, 1, b, sb, 2, np.arange(M))
+    for _ in range(3):
+        got = fq.fp8_gemm_blockscaled(*args, ws=ws)
+        torch.cuda.synchronize()
+        check_tolerance(host(got), ref, "reused workspace")
+        assert int(ws[: 4 * (N // 128)].count_nonzero()) == 0
+    assert fq.device_status() == 0
+
+
+def test_gemm_decode_dirty_workspace_is_reported(orc):
+    """Counters that are not zero on entry raise device error bit 1 (no wait depends on them)."""
+    M, N, K = 16, 2048, 4096
+    a, sa, b, sb = operands(orc, M, N, K, 1, 2, seed=13)
+    ws = torch.full((fq.gemm_workspace_bytes(M, N, K),), 0xFF, dtype=torch.uint8, device="cuda")
+    fq.fp8_gemm_blockscaled(dev(a), dev(sa), dev(b), dev(sb), 1, 2, ws=ws)
+    assert fq.device_status() & 2
+
+
 def test_gemm_config2_prefill_8b(orc):
     M, N, K = 8192, 14336, 4096
     x = synth.activations(seed=1)
