@@ -671,7 +671,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
           float* dst = p.partials + ((size_t)(blockIdx.x * p.maxseg + (t - first_tile)) * MP) * BM + row;
 #pragma unroll
           for (int m = 0; m < MP; ++m) dst[(size_t)m * BM] = acc[m];
-          __threadfence();
+          // the four warps hand their writes to one thread through the mbarrier (release /
+          // acquire at CTA scope); its gpu-scope fence then orders all of them (cumulatively)
+          // before its atomic, so no per-thread fence is needed
           __syncwarp();
           if (lane == 0) mbar_arrive(seg_written);
           if (warp == 3 && lane == 0) {
@@ -683,7 +685,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
               const uint32_t old = atomicAdd(p.counters + t, 1u);
               if (old >= n_contrib) raise_device_error(p.err, kErrWorkspaceDirty);
               last = old + 1 == n_contrib;
-              if (last) p.counters[t] = 0;   // every contributor has counted in: leave it zero
+              if (last) {
+                __threadfence();           // acquire: the other contributors' partials
+                p.counters[t] = 0;         // every contributor has counted in: leave it zero
+              }
             }
             s_last = last;
             mbar_arrive(seg_decided);
