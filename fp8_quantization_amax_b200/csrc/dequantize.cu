@@ -12,6 +12,7 @@
 
 #include "fp8q_device.cuh"
 #include "internal.h"
+#include "sm100.cuh"
 
 namespace fp8q {
 
@@ -38,6 +39,8 @@ template <int FMT, int GRAN, int UNROLL>
 __global__ void __launch_bounds__(256) k_dequant(const uint8_t* __restrict__ codes, const float* __restrict__ scales,
                                                  uint16_t* __restrict__ y, uint32_t npieces, FastDiv ppr,
                                                  uint32_t rows, uint32_t nbc) {
+  allow_dependent_launch();
+  grid_dependency_wait();
   const uint32_t stride = gridDim.x * blockDim.x;
   for (uint32_t i0 = blockIdx.x * blockDim.x + threadIdx.x; i0 < npieces; i0 += stride * UNROLL) {
     uint2 c[UNROLL];
@@ -79,10 +82,9 @@ static cudaError_t launch_dequant_impl(const uint8_t* codes, const float* scales
   }
   const int64_t need = (npieces + 256 * kUnroll - 1) / (256 * kUnroll);
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(need, (int64_t)device_sm_count() * occ));
-  k_dequant<FMT, GRAN, kUnroll><<<grid, 256, 0, st>>>(codes, scales, y, (uint32_t)npieces,
-                                                      make_fastdiv((uint32_t)(cols / 8)), (uint32_t)rows,
-                                                      (uint32_t)((cols + 127) / 128));
-  return cudaGetLastError();
+  return launch_pdl(k_dequant<FMT, GRAN, kUnroll>, dim3(grid), dim3(256), 0, st, codes, scales, y,
+                    (uint32_t)npieces, make_fastdiv((uint32_t)(cols / 8)), (uint32_t)rows,
+                    (uint32_t)((cols + 127) / 128));
 }
 
 template <int FMT>
@@ -103,6 +105,8 @@ cudaError_t launch_dequant(const uint8_t* codes, const float* scales, int64_t ro
 
 template <int FMT>
 __global__ void __launch_bounds__(256) k_encode(const float* __restrict__ q, int64_t n, uint8_t* __restrict__ codes) {
+  allow_dependent_launch();
+  grid_dependency_wait();
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   const int64_t n4 = n / 4;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride) {
@@ -116,6 +120,8 @@ __global__ void __launch_bounds__(256) k_encode(const float* __restrict__ q, int
 
 template <int FMT>
 __global__ void __launch_bounds__(256) k_decode(const uint8_t* __restrict__ codes, int64_t n, float* __restrict__ out) {
+  allow_dependent_launch();
+  grid_dependency_wait();
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   const int64_t n4 = n / 4;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride) {
@@ -136,20 +142,14 @@ static int codec_grid(int64_t n) {
 
 cudaError_t launch_encode(const float* q, int64_t n, int fmt, uint8_t* codes, cudaStream_t st) {
   if (n == 0) return cudaSuccess;
-  if (fmt == kE4M3)
-    k_encode<kE4M3><<<codec_grid(n), 256, 0, st>>>(q, n, codes);
-  else
-    k_encode<kE5M2><<<codec_grid(n), 256, 0, st>>>(q, n, codes);
-  return cudaGetLastError();
+  return fmt == kE4M3 ? launch_pdl(k_encode<kE4M3>, dim3(codec_grid(n)), dim3(256), 0, st, q, n, codes)
+                      : launch_pdl(k_encode<kE5M2>, dim3(codec_grid(n)), dim3(256), 0, st, q, n, codes);
 }
 
 cudaError_t launch_decode(const uint8_t* codes, int64_t n, int fmt, float* out, cudaStream_t st) {
   if (n == 0) return cudaSuccess;
-  if (fmt == kE4M3)
-    k_decode<kE4M3><<<codec_grid(n), 256, 0, st>>>(codes, n, out);
-  else
-    k_decode<kE5M2><<<codec_grid(n), 256, 0, st>>>(codes, n, out);
-  return cudaGetLastError();
+  return fmt == kE4M3 ? launch_pdl(k_decode<kE4M3>, dim3(codec_grid(n)), dim3(256), 0, st, codes, n, out)
+                      : launch_pdl(k_decode<kE5M2>, dim3(codec_grid(n)), dim3(256), 0, st, codes, n, out);
 }
 
 }  // namespace fp8q

@@ -178,9 +178,18 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 // four bf16 (two words) -> four codes, fast path
 template <int FMT>
 __device__ __forceinline__ uint32_t quant4_fast(uint32_t w0, uint32_t w1, float d, float r) {
-  const uint32_t a = cvt2<FMT>(markstein_div(bf16_lo(w0), d, r), markstein_div(bf16_hi(w0), d, r));
-  const uint32_t b = cvt2<FMT>(markstein_div(bf16_lo(w1), d, r), markstein_div(bf16_hi(w1), d, r));
-  return __byte_perm(a, b, 0x5410);
+  // The same three rounded steps as markstein_div, on fp32 pairs (one FMUL2 / FFMA2 per pair)
+  // and with every value negated, so no operand needs a sign flip: p = RN(x * -r) = -q0,
+  // f = RN(p * d + x) = x - q0 * d (exact), n = RN(f * -r + p) = -RN(q0 + (x - q0 * d) * r)
+  // = -q, because round-to-nearest is odd-symmetric (a zero residual is +0 in both forms, and
+  // x = +-0 gives n = -+0).  The codes of -q are those of q with the sign bit flipped, and the
+  // saturating conversion is sign-symmetric, so one XOR restores them.
+  const float2 d2 = make_float2(d, d), nr2 = make_float2(-r, -r);
+  const float2 x0 = make_float2(bf16_lo(w0), bf16_hi(w0)), x1 = make_float2(bf16_lo(w1), bf16_hi(w1));
+  const float2 p0 = __fmul2_rn(x0, nr2), p1 = __fmul2_rn(x1, nr2);
+  const float2 f0 = __ffma2_rn(p0, d2, x0), f1 = __ffma2_rn(p1, d2, x1);
+  const float2 n0 = __ffma2_rn(f0, nr2, p0), n1 = __ffma2_rn(f1, nr2, p1);
+  return __byte_perm(cvt2<FMT>(n0.x, n0.y), cvt2<FMT>(n1.x, n1.y), 0x5410) ^ 0x80808080u;
 }
 
 // eight bf16 (16 bytes) -> eight codes (8 bytes), fast path

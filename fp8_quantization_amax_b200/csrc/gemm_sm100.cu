@@ -172,6 +172,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ CU
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  allow_dependent_launch();
+  grid_dependency_wait();
   const int my_tiles = p.tiles > (int)blockIdx.x ? (p.tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
 
   if (warp < kFirstEpiWarp) {
@@ -538,8 +540,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = tmem_slot;
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  allow_dependent_launch();
+  grid_dependency_wait();
 
   if (warp == 0) {
     if (lane == 0 && n_units > 0) {
@@ -870,16 +872,15 @@ cudaError_t launch_gemm(const uint8_t* A, const float* sA, int gA, const uint8_t
       cudaFuncSetAttribute(k_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
       attr = true;
     }
-    k_gemm<true><<<grid, kThreads, kSmemBytes, st>>>(mA, mB, p);
+    return launch_pdl(k_gemm<true>, dim3(grid), dim3(kThreads), kSmemBytes, st, mA, mB, p);
   } else {
     static bool attr = false;
     if (!attr) {
       cudaFuncSetAttribute(k_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
       attr = true;
     }
-    k_gemm<false><<<grid, kThreads, kSmemBytes, st>>>(mA, mB, p);
+    return launch_pdl(k_gemm<false>, dim3(grid), dim3(kThreads), kSmemBytes, st, mA, mB, p);
   }
-  return cudaGetLastError();
 }
 
 }  // namespace fp8q

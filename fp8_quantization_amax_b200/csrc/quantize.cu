@@ -145,11 +145,20 @@ __global__ void __launch_bounds__(kThreads, 2) k_group128(const __grid_constant_
     }
     fence_mbar_init();
   }
-  __syncthreads();
   const uint32_t nk = items_of_cta(p.nitems);
+  if (warp == kConsumerWarps && lane == 0) {
+    // warm L2 with this CTA's first boxes while the previous grid on the stream finishes
+    tma_prefetch_desc(&tx);
+    for (uint32_t k = 0; k < nk && k < (uint32_t)S; ++k) {
+      const uint32_t i = blockIdx.x + k * gridDim.x, rb = fdiv(i, p.ngc), g = i - rb * p.ngc.d;
+      tma_prefetch_l2_2d(&tx, (int32_t)(g * 128), (int32_t)(rb * kGroupBoxRows));
+    }
+  }
+  __syncthreads();
+  allow_dependent_launch();
+  grid_dependency_wait();
   if (warp == kConsumerWarps) {
     if (lane == 0 && nk > 0) {
-      tma_prefetch_desc(&tx);
       run_producer(
           full, empty, S, nk, kGroupStage, p.err, [&](uint32_t k) { return blockIdx.x + k * gridDim.x; },
           [&](uint32_t i, int s, uint64_t* bar) {
@@ -224,8 +233,7 @@ static cudaError_t launch_group128_fmt(const uint16_t* x, int64_t rows, int64_t 
     attr = true;
   }
   const int grid = grid_for(k_group128<FMT>, smem, p.nitems);
-  k_group128<FMT><<<grid, kThreads, smem, st>>>(map, p);
-  return cudaGetLastError();
+  return launch_pdl(k_group128<FMT>, dim3(grid), dim3(kThreads), smem, st, map, p);
 }
 
 cudaError_t launch_quant_1x128(const uint16_t* x, int64_t rows, int64_t cols, int fmt, uint8_t* codes,
@@ -311,12 +319,21 @@ __global__ void __launch_bounds__(kThreads, 2) k_tile128(const __grid_constant__
     }
     fence_mbar_init();
   }
-  __syncthreads();
   const uint32_t nk = items_of_cta(p.nitems);
+  if (warp == kConsumerWarps && lane == 0) {
+    // warm L2 with this CTA's first boxes while the previous grid on the stream finishes
+    tma_prefetch_desc(&t0);
+    tma_prefetch_desc(&t1);
+    for (uint32_t k = 0; k < nk && k < (uint32_t)S; ++k) {
+      const TileItem it = tile_item(tile_item_index<MODE>(k, p.nitems), p);
+      tma_prefetch_l2_2d(it.tens ? &t1 : &t0, (int32_t)(it.bj * p.bc), (int32_t)(it.bi * 128));
+    }
+  }
+  __syncthreads();
+  allow_dependent_launch();
+  grid_dependency_wait();
   if (warp == kConsumerWarps) {
     if (lane == 0 && nk > 0) {
-      tma_prefetch_desc(&t0);
-      tma_prefetch_desc(&t1);
       run_producer(
           full, empty, S, nk, p.stage_bytes, p.err, [&](uint32_t k) { return tile_item_index<MODE>(k, p.nitems); },
           [&](uint32_t i, int s, uint64_t* bar) {
@@ -471,8 +488,7 @@ static cudaError_t launch_tile_impl(const CUtensorMap& m0, const CUtensorMap& m1
   int grid = grid_for(k_tile128<FMT, MODE, CPR, MAXC>, smem, std::max<uint32_t>(p.nitems, 1));
   if (max_grid > 0) grid = std::min(grid, max_grid);
   if (grid_used) *grid_used = grid;
-  k_tile128<FMT, MODE, CPR, MAXC><<<grid, kThreads, smem, st>>>(m0, m1, p);
-  return cudaGetLastError();
+  return launch_pdl(k_tile128<FMT, MODE, CPR, MAXC>, dim3(grid), dim3(kThreads), smem, st, m0, m1, p);
 }
 
 template <int FMT, int MODE>

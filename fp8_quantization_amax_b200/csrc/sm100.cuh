@@ -92,6 +92,18 @@ __device__ __forceinline__ void release_stage(uint64_t* empty_bar, int lane) {
   if (lane == 0) mbar_arrive(empty_bar);
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+//
+// Kernels are launched with the programmatic stream-serialization attribute (launch_pdl), so a
+// grid may start while the previous grid on its stream is still finishing.  Everything before
+// grid_dependency_wait() must leave global memory alone (L2 prefetches excepted: they only warm
+// a coherent cache); the wait returns once the previous grid has completed and its writes are
+// visible.  allow_dependent_launch() lets the next grid start its own set-up early.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_dependent_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
