@@ -68,6 +68,8 @@ def _load():
             lib.orc_gemm_rows.restype = i32
             lib.orc_int8_level.argtypes = [f64, f64]
             lib.orc_int8_level.restype = i32
+            lib.orc_quantize_delayed.argtypes = [vp, i64, i64, i64, i32, vp, i64, i64, vp, vp, vp]
+            lib.orc_quantize_delayed.restype = i32
             _lib = lib
     return _lib
 
@@ -215,6 +217,35 @@ def kv_quantize(k_bf16: np.ndarray, v_bf16: np.ndarray, fmt: int, gran: int):
     rc = _load().orc_kv_quantize(_p(k), _p(v), T, H, D, fmt, gran, _p(kc), _p(vc), _p(ks), _p(vs))
     assert rc == 0
     return kc, vc, ks, vs
+
+
+# ---------------------------------------------------------------- delayed scaling
+
+def quantize_delayed(x_bf16: np.ndarray, fmt: int, history: np.ndarray, step: int, counts: np.ndarray | None = None):
+    """Delayed-scaling quantization of bf16 bits x [rows][ngroups * gw] with one scale group per
+    column block of gw columns, ngroups = history.shape[1].
+
+    history float32 [H][ngroups] is read (step >= 1) and then updated in place: slot step % H
+    receives this call's amax.  counts (uint64 [2], optional) accumulates saturated and
+    underflowed elements.  Returns (codes uint8 like x, scales float32 [ngroups]).
+    """
+    x = np.ascontiguousarray(x_bf16, np.uint16)
+    rows = x.shape[0]
+    cols = int(np.prod(x.shape[1:])) if x.ndim > 1 else x.shape[0]
+    if x.ndim == 1:
+        rows = 1
+    assert history.dtype == np.float32 and history.flags["C_CONTIGUOUS"] and history.ndim == 2
+    H, ngroups = history.shape
+    assert cols % ngroups == 0
+    codes = np.empty(x.shape, np.uint8)
+    scales = np.empty((ngroups,), np.float32)
+    cnt = counts if counts is not None else None
+    if cnt is not None:
+        assert cnt.dtype == np.uint64 and cnt.shape == (2,)
+    rc = _load().orc_quantize_delayed(_p(x), rows, ngroups, cols // ngroups, fmt, _p(history), H, step,
+                                      _p(codes), _p(scales), _p(cnt) if cnt is not None else None)
+    assert rc == 0
+    return codes, scales
 
 
 # ---------------------------------------------------------------- GEMM

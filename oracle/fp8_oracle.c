@@ -401,3 +401,82 @@ int orc_int8_level(double x, double amax) {
     if (l < -127) l = -127;
     return (int)l;
 }
+
+/* ------------------------------------------------------------------------ */
+/* delayed scaling and per-call counts                                       */
+/*
+ * Delayed scaling ([C] "scale 是控制面": the scale follows a history of amax
+ * values recorded by earlier steps instead of the tensor being cast; [M]
+ * section 二: the forward pass takes its scale factor from the previous
+ * micro-batch's max).  Counts of saturated and underflowed elements are the
+ * overflow / underflow signals [C] "scale 是控制面" asks to be observable.
+ *
+ * Readings (also in the design notes):
+ *   - One scale group is a column block over all rows: columns
+ *     [g*gw, (g+1)*gw) of x [rows][ngroups*gw] (per-tensor: ngroups = 1,
+ *     gw = cols; a KV cache per head: rows = tokens, ngroups = heads,
+ *     gw = head_dim).
+ *   - history [H][ngroups] holds amax values of earlier calls, zero where no
+ *     call has written; entries are >= 0 or NaN.
+ *   - step 0 has no history yet: its scale comes from its own amax (the
+ *     dynamic rule).  Step t >= 1: s = RN(max over the H entries / FMAX), NaN
+ *     sticky.  Either way the cast is the usual FP8(RN(x / s)), saturating; an
+ *     all-zero history gives s = 0 and sign-only codes (as for an all-zero
+ *     group).
+ *   - Afterwards history[t mod H][g] = this call's own amax of group g.
+ *   - counts[0] += elements that saturate: round-to-nearest-even of |x / s| on
+ *     the format's grid continued past FMAX lands above FMAX.
+ *     counts[1] += elements with x != 0 (NaN excluded) whose code is +-0.
+ */
+
+/* does |q| round (ties to even) above FMAX on the grid continued past FMAX? */
+static int saturates(int fmt, float q) {
+    orc_fmt f = fmt_of(fmt);
+    double a = fabs((double)q);
+    if (isnan(q)) return 0;
+    /* FMAX = (2 - 2^(1-M)) * 2^E: the next point of the continued grid is FMAX + 2^(E-M) */
+    int e;
+    frexp((double)f.fmax, &e);                 /* FMAX = m * 2^e with m in [0.5, 1): E = e - 1 */
+    double next = (double)f.fmax + ldexp(1.0, (e - 1) - f.mbits);
+    double mid = 0.5 * ((double)f.fmax + next);
+    if (a > mid) return 1;
+    if (a < mid) return 0;
+    return (f.max_code & 1) != 0;              /* a tie goes to the even mantissa: next if FMAX's is odd */
+}
+
+int orc_quantize_delayed(const uint16_t *x, int64_t rows, int64_t ngroups, int64_t gw, int fmt,
+                         float *history, int64_t H, int64_t step, uint8_t *codes, float *scales,
+                         uint64_t *counts) {
+    if (H < 1 || step < 0 || ngroups < 1 || gw < 1) return -1;
+    FPENV_ENTER;
+    int64_t ld = ngroups * gw;
+    float *cur = (float *)malloc(sizeof(float) * (size_t)ngroups);
+    for (int64_t g = 0; g < ngroups; ++g) {
+        cur[g] = region_amax(x + g * gw, rows, gw, ld);
+        float a = cur[g];
+        if (step > 0) {
+            a = 0.0f;
+            for (int64_t t = 0; t < H; ++t) {
+                float h = history[t * ngroups + g];
+                if (isnan(h) || isnan(a)) a = NAN;
+                else if (h > a) a = h;
+            }
+        }
+        float s = orc_scale(fmt, a);
+        scales[g] = s;
+        for (int64_t r = 0; r < rows; ++r)
+            for (int64_t c = 0; c < gw; ++c) {
+                float xv = bf16_value(x[r * ld + g * gw + c]);
+                uint8_t code = cast_one(fmt, xv, s);
+                codes[r * ld + g * gw + c] = code;
+                if (counts) {
+                    if (s != 0.0f && saturates(fmt, xv / s)) counts[0] += 1;
+                    if (!isnan(xv) && xv != 0.0f && (code & 0x7F) == 0) counts[1] += 1;
+                }
+            }
+    }
+    for (int64_t g = 0; g < ngroups; ++g) history[(step % H) * ngroups + g] = cur[g];
+    free(cur);
+    FPENV_LEAVE;
+    return 0;
+}

@@ -13,6 +13,7 @@ import numpy as np
 import pytest
 
 import test_oracle_codec as tc
+import test_oracle_delayed as td
 import test_oracle_gemm as tg
 import test_oracle_quantize as tq
 
@@ -42,6 +43,11 @@ MUTANTS = {
     "gemm_drop_sa": ("* (double)scale_at(sA, M, K, gA, rows[i], k);", ";"),
     "gemm_b_index": ("scale_at(sB, N, K, gB, n, k)", "scale_at(sB, N, K, gB, k % N, n % K)"),
     "gemm_b_transposed": ("b[k] = (double)orc_decode(fmtB, B[n * K + k])", "b[k] = (double)orc_decode(fmtB, B[(k % N) * K + (n % K)])"),
+    "delayed_ignores_history": ("        if (step > 0) {\n            a = 0.0f;", "        if (0) {\n            a = 0.0f;"),
+    "delayed_history_slot": ("history[(step % H) * ngroups + g] = cur[g];", "history[((step + 1) % H) * ngroups + g] = cur[g];"),
+    "saturation_tie_flipped": ("return (f.max_code & 1) != 0;", "return (f.max_code & 1) == 0;"),
+    "saturation_at_fmax": ("if (a > mid) return 1;", "if (a > (double)f.fmax) return 1;"),
+    "underflow_counts_zeros": ("if (!isnan(xv) && xv != 0.0f && (code & 0x7F) == 0)", "if (!isnan(xv) && (code & 0x7F) == 0)"),
 }
 
 
@@ -64,6 +70,11 @@ def _pins(m):
     for gran in (0, 1, 2):
         checks.append(lambda gran=gran: tq.test_kv_bruteforce_tiny(m, 0, gran, (257, 8, 64)))
     checks += [
+        lambda: td.test_hand_worked_e4m3_unit_scale(m),
+        lambda: td.test_hand_worked_e5m2_unit_scale(m),
+        lambda: td.test_ring_update_and_window_max(m),
+        lambda: td.test_zero_history_gives_sign_only_codes(m),
+        lambda: td.test_history_holding_the_current_amax_reduces_to_dynamic(m),
         lambda: tg.test_closed_form_constant_operands(m),
         lambda: tg.test_matches_numpy_matmul(m, 1, 2, (130, 384, 256)),
         lambda: tg.test_blockwise_identity(m),
