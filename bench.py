@@ -309,6 +309,18 @@ def supplementary(device, stream, peaks, flush):
             ms = timed(lambda: fq.fp8_kv_quantize(kd, vd, fmt, gran, *r, ws=None), 10, stream, flush)
             nbytes = e2 * (3 if passes == 1 else 5) + 2 * r[2].numel() * 4
             out[name] = gbs(nbytes, ms)
+        # delayed scaling (per head, E4M3): after the first call every call reads the cache once
+        hk = torch.zeros((4, 8), dtype=torch.float32, device=device)
+        hv = torch.zeros_like(hk)
+        r = fq.fp8_kv_quantize_delayed(kd, vd, hk, hv, 0, fq.E4M3, fq.KV_PER_HEAD)
+        step_no = [0]
+
+        def delayed_call():
+            step_no[0] += 1
+            fq.fp8_kv_quantize_delayed(kd, vd, hk, hv, step_no[0], fq.E4M3, fq.KV_PER_HEAD, *r)
+
+        ms = timed(delayed_call, 10, stream, flush)
+        out["kv_head_e4m3_delayed"] = gbs(e2 * 3 + 2 * r[2].numel() * 4, ms)
         del kd, vd, r
         # GEMM (8B up-proj shape) on the quantized config-1 operands
         x = dev_bf16(synth.activations(seed=1), device)

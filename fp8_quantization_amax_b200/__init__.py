@@ -21,7 +21,7 @@ __all__ = [
     "Fp8qError", "lib", "library_path", "device_status", "num_scales", "workspace_bytes", "kv_num_scales",
     "kv_workspace_bytes", "gemm_workspace_bytes", "scale_shape", "kv_scale_shape",
     "fp8_encode", "fp8_decode", "fp8_quantize", "fp8_dequantize", "fp8_kv_quantize",
-    "fp8_kv_quantize_noalloc", "fp8_gemm_blockscaled",
+    "fp8_kv_quantize_noalloc", "fp8_gemm_blockscaled", "fp8_quantize_delayed", "fp8_kv_quantize_delayed",
 ]
 
 E4M3, E5M2 = 0, 1
@@ -75,8 +75,12 @@ def lib() -> ctypes.CDLL:
             L.fp8_kv_quantize.argtypes = [vp, vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, sz, vp]
             L.fp8_gemm_blockscaled.argtypes = [vp, vp, i32, vp, vp, i32, i64, i64, i64, vp, vp, sz, vp]
             L.fp8_kv_quantize_noalloc.argtypes = [vp, vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp]
+            L.fp8_quantize_delayed.argtypes = [vp, i64, i64, i32, vp, i64, i64, vp, vp, vp, vp, sz, vp]
+            L.fp8_kv_quantize_delayed.argtypes = [vp, vp, i64, i64, i64, i32, i32, vp, vp, i64, i64, vp, vp, vp, vp,
+                                                  vp, vp, sz, vp]
             for fn in ("fp8_encode", "fp8_decode", "fp8_quantize", "fp8_dequantize", "fp8_kv_quantize",
-                       "fp8_gemm_blockscaled", "fp8_kv_quantize_noalloc"):
+                       "fp8_gemm_blockscaled", "fp8_kv_quantize_noalloc", "fp8_quantize_delayed",
+                       "fp8_kv_quantize_delayed"):
                 getattr(L, fn).restype = i32
             _lib = L
     return _lib
@@ -232,6 +236,69 @@ def fp8_quantize(x: torch.Tensor, fmt: int = E4M3, gran: int = GROUP_1x128, code
                             0 if ws is None else ws.numel() * ws.element_size(), _stream(x.device))
     _check("fp8_quantize", st)
     return codes, scales
+
+
+def _counts(counts):
+    if counts is None:
+        return None
+    if counts.dtype != torch.int64 or counts.numel() != 2 or not counts.is_cuda or not counts.is_contiguous():
+        raise ValueError("counts must be a contiguous int64 CUDA tensor of 2 entries")
+    return counts
+
+
+def fp8_quantize_delayed(x: torch.Tensor, history: torch.Tensor, step: int, fmt: int = E4M3,
+                         codes: torch.Tensor | None = None, scale: torch.Tensor | None = None,
+                         counts: torch.Tensor | None = None, ws: torch.Tensor | None = None):
+    """Per-tensor delayed scaling: bf16 [rows][cols] -> (codes, scale [1]).  history fp32 [H]
+    (zero-filled before step 0) is read and updated in place; counts (int64 [2], optional)
+    accumulates saturated and underflowed elements."""
+    _dev(x, "x", torch.bfloat16)
+    _dev(history, "history", torch.float32)
+    if x.dim() != 2:
+        raise ValueError("x must be 2-D [rows][cols]")
+    rows, cols = x.shape
+    codes = torch.empty((rows, cols), dtype=torch.uint8, device=x.device) if codes is None else \
+        _dev(codes, "codes", torch.uint8)
+    scale = torch.empty((1,), dtype=torch.float32, device=x.device) if scale is None else _dev(scale, "scale", torch.float32)
+    counts = _counts(counts)
+    ws = _workspace(workspace_bytes(rows, cols, PER_TENSOR), x.device, ws)
+    st = lib().fp8_quantize_delayed(_ptr(x), rows, cols, fmt, _ptr(history), history.numel(), step, _ptr(codes),
+                                    _ptr(scale), _ptr(counts), _ptr(ws), ws.numel() * ws.element_size(),
+                                    _stream(x.device))
+    _check("fp8_quantize_delayed", st)
+    return codes, scale
+
+
+def fp8_kv_quantize_delayed(k: torch.Tensor, v: torch.Tensor, k_history: torch.Tensor, v_history: torch.Tensor,
+                            step: int, fmt: int = E4M3, gran: int = KV_PER_HEAD, k_codes=None, v_codes=None,
+                            k_scales=None, v_scales=None, counts: torch.Tensor | None = None, ws=None):
+    """KV delayed scaling (per tensor or per head): histories fp32 [H][heads] (per head) or [H]
+    (per tensor), read and updated in place -> (k_codes, v_codes, k_scales, v_scales)."""
+    _dev(k, "k", torch.bfloat16)
+    _dev(v, "v", torch.bfloat16)
+    _dev(k_history, "k_history", torch.float32)
+    _dev(v_history, "v_history", torch.float32)
+    if k.dim() != 3 or k.shape != v.shape:
+        raise ValueError("k and v must both be [tokens][heads][head_dim]")
+    T, H, D = k.shape
+    per = H if gran == KV_PER_HEAD else 1
+    if k_history.numel() % max(per, 1) or k_history.shape != v_history.shape:
+        raise ValueError("histories must be [history_len][heads] (per head) or [history_len] (per tensor)")
+    hlen = k_history.numel() // max(per, 1)
+    dev = k.device
+    k_codes = torch.empty(k.shape, dtype=torch.uint8, device=dev) if k_codes is None else _dev(k_codes, "k_codes", torch.uint8)
+    v_codes = torch.empty(v.shape, dtype=torch.uint8, device=dev) if v_codes is None else _dev(v_codes, "v_codes", torch.uint8)
+    shp = kv_scale_shape(T, H, gran)
+    k_scales = torch.empty(shp, dtype=torch.float32, device=dev) if k_scales is None else _dev(k_scales, "k_scales", torch.float32)
+    v_scales = torch.empty(shp, dtype=torch.float32, device=dev) if v_scales is None else _dev(v_scales, "v_scales", torch.float32)
+    counts = _counts(counts)
+    ws = _workspace(kv_workspace_bytes(T, H, D, gran), dev, ws)
+    st = lib().fp8_kv_quantize_delayed(_ptr(k), _ptr(v), T, H, D, fmt, gran, _ptr(k_history), _ptr(v_history), hlen,
+                                       step, _ptr(k_codes), _ptr(v_codes), _ptr(k_scales), _ptr(v_scales),
+                                       _ptr(counts), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+                                       _stream(dev))
+    _check("fp8_kv_quantize_delayed", st)
+    return k_codes, v_codes, k_scales, v_scales
 
 
 def fp8_dequantize(codes: torch.Tensor, scales: torch.Tensor, fmt: int = E4M3, gran: int = GROUP_1x128,

@@ -10,6 +10,7 @@
 namespace {
 
 constexpr int64_t kMaxElems = int64_t(1) << 33;   // 32-bit indexing of 16-byte pieces of two tensors
+constexpr int64_t kMaxHistory = int64_t(1) << 20;   // amax history entries per group (the kernels index with int)
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 bool valid_fmt(int f) { return f == FP8Q_E4M3 || f == FP8Q_E5M2; }
@@ -114,6 +115,23 @@ fp8q_status fp8_quantize(const void* x, int64_t rows, int64_t cols, fp8q_format 
       fp8q::launch_quant_tiles(xs, nullptr, codes, nullptr, scales, nullptr, 1, rows, cols, cols, 128, f, st));
 }
 
+fp8q_status fp8_quantize_delayed(const void* x, int64_t rows, int64_t cols, fp8q_format f, float* amax_history,
+                                 int64_t history_len, int64_t step, uint8_t* codes, float* scale,
+                                 unsigned long long* counts, void* ws, size_t ws_bytes, fp8q_stream_t stream) {
+  const int64_t n = checked_elems(rows, cols);
+  if (rows < 0 || cols < 0 || !valid_fmt(f) || cols % 8 != 0 || history_len < 1 || step < 0)
+    return FP8Q_ERR_INVALID_ARGUMENT;
+  if (n < 0 || history_len > kMaxHistory) return FP8Q_ERR_UNSUPPORTED;
+  if (n > 0 && (!x || !codes || !aligned(x, 16) || !aligned(codes, 16))) return FP8Q_ERR_INVALID_ARGUMENT;
+  if (!scale || !aligned(scale, 4) || !amax_history || !aligned(amax_history, 4)) return FP8Q_ERR_INVALID_ARGUMENT;
+  if (counts && !aligned(counts, 8)) return FP8Q_ERR_INVALID_ARGUMENT;
+  const size_t need = fp8q_workspace_bytes(rows, cols, FP8Q_PER_TENSOR);
+  if (!ws || ws_bytes < need || !aligned(ws, 4)) return FP8Q_ERR_WORKSPACE;
+  return from_cuda(fp8q::launch_quant_delayed(static_cast<const uint16_t*>(x), nullptr, codes, nullptr, scale, nullptr,
+                                              1, rows, 1, cols, f, amax_history, nullptr, history_len, step, counts,
+                                              static_cast<float*>(ws), (cudaStream_t)stream));
+}
+
 fp8q_status fp8_dequantize(const uint8_t* codes, const float* scales, int64_t rows, int64_t cols, fp8q_format f,
                            fp8q_granularity g, void* y, fp8q_stream_t stream) {
   const int64_t n = checked_elems(rows, cols);
@@ -157,6 +175,38 @@ fp8q_status fp8_kv_quantize(const void* k, const void* v, int64_t tokens, int64_
   const int64_t d = g == FP8Q_KV_PER_TENSOR ? row : head_dim;
   return from_cuda(fp8q::launch_quant_two_pass(ks, vs, k_codes, v_codes, k_scales, v_scales, 2, tokens, h, d, f,
                                                static_cast<float*>(ws), st));
+}
+
+fp8q_status fp8_kv_quantize_delayed(const void* k, const void* v, int64_t tokens, int64_t heads, int64_t head_dim,
+                                    fp8q_format f, fp8q_kv_granularity g, float* k_history, float* v_history,
+                                    int64_t history_len, int64_t step, uint8_t* k_codes, uint8_t* v_codes,
+                                    float* k_scales, float* v_scales, unsigned long long* counts, void* ws,
+                                    size_t ws_bytes, fp8q_stream_t stream) {
+  if (tokens < 0 || heads < 0 || head_dim < 0 || !valid_fmt(f) || !valid_kv_gran(g) || head_dim % 8 != 0 ||
+      history_len < 1 || step < 0)
+    return FP8Q_ERR_INVALID_ARGUMENT;
+  if (g == FP8Q_KV_PER_HEAD_TOK128) return FP8Q_ERR_UNSUPPORTED;   // already one pass: no history to keep
+  const int64_t row = checked_elems(heads, head_dim);
+  const int64_t n = row < 0 ? -1 : checked_elems(tokens, row);
+  if (n < 0 || history_len > kMaxHistory) return FP8Q_ERR_UNSUPPORTED;
+  if (g == FP8Q_KV_PER_HEAD && (heads > 128 || head_dim > 256)) return FP8Q_ERR_UNSUPPORTED;
+  const size_t nsc = fp8q_kv_num_scales(tokens, heads, g);
+  if (n > 0 && (!k || !v || !k_codes || !v_codes || !aligned(k, 16) || !aligned(v, 16) || !aligned(k_codes, 16) ||
+                !aligned(v_codes, 16)))
+    return FP8Q_ERR_INVALID_ARGUMENT;
+  if (nsc > 0 && (!k_scales || !v_scales || !aligned(k_scales, 4) || !aligned(v_scales, 4) || !k_history ||
+                  !v_history || !aligned(k_history, 4) || !aligned(v_history, 4)))
+    return FP8Q_ERR_INVALID_ARGUMENT;
+  if (counts && !aligned(counts, 8)) return FP8Q_ERR_INVALID_ARGUMENT;
+  if (nsc == 0) return FP8Q_OK;   // no heads: nothing to write
+  const size_t need = fp8q_kv_workspace_bytes(tokens, heads, head_dim, g);
+  if (!ws || ws_bytes < need || !aligned(ws, 4)) return FP8Q_ERR_WORKSPACE;
+  const int64_t h = g == FP8Q_KV_PER_TENSOR ? 1 : heads;
+  const int64_t d = g == FP8Q_KV_PER_TENSOR ? row : head_dim;
+  return from_cuda(fp8q::launch_quant_delayed(static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v),
+                                              k_codes, v_codes, k_scales, v_scales, 2, tokens, h, d, f, k_history,
+                                              v_history, history_len, step, counts, static_cast<float*>(ws),
+                                              (cudaStream_t)stream));
 }
 
 fp8q_status fp8_gemm_blockscaled(const uint8_t* A, const float* sA, fp8q_granularity gA, const uint8_t* B,

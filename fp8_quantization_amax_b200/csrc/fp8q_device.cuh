@@ -205,10 +205,17 @@ __device__ __forceinline__ uint4 quant16_fast(uint4 a, uint4 b, float d, float r
                     quant4_fast<FMT>(b.x, b.y, d, r), quant4_fast<FMT>(b.z, b.w, d, r));
 }
 
-// eight bf16 -> eight codes with IEEE divisions (groups with tiny, infinite or NaN amax)
+// eight bf16 -> eight codes with IEEE divisions (groups with tiny, infinite or NaN amax).
+// d == 0 is a zero scale met by delayed scaling (an all-zero amax history while the tensor is
+// not zero): every code is the zero with the element's sign, as for an all-zero group.
 template <int FMT>
 __device__ __noinline__ uint2 quant8_slow(uint4 v, float d) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  if (d == 0.0f) {
+    const uint32_t lo = ((w[0] >> 8) & 0x80u) | ((w[0] >> 16) & 0x8000u) | ((w[1] << 8) & 0x800000u) | (w[1] & 0x80000000u);
+    const uint32_t hi = ((w[2] >> 8) & 0x80u) | ((w[2] >> 16) & 0x8000u) | ((w[3] << 8) & 0x800000u) | (w[3] & 0x80000000u);
+    return make_uint2(lo, hi);
+  }
   uint32_t c[2];
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
@@ -222,6 +229,42 @@ __device__ __noinline__ uint2 quant8_slow(uint4 v, float d) {
 template <int FMT>
 __device__ __forceinline__ uint2 quant8(uint4 v, const GroupScale& g) {
   return g.fast ? quant8_fast<FMT>(v, g.d, g.r) : quant8_slow<FMT>(v, g.d);
+}
+
+// ---------------------------------------------------------------- delayed scaling, counts
+
+// Scale of a delayed-scaling group from the largest amax in its history (>= 0 or NaN).  A zero
+// history gives s = 0 with d = 0, which quant8_slow turns into sign-only codes.
+template <int FMT>
+__device__ __forceinline__ GroupScale make_delayed_scale(float hmax) {
+  if (hmax == 0.0f) {
+    GroupScale g;
+    g.s = 0.0f;
+    g.d = 0.0f;
+    g.r = 0.0f;
+    g.fast = false;
+    return g;
+  }
+  return make_group_scale<FMT>(hmax);
+}
+
+// Counts of one chunk of eight bf16 and their codes: `sat` += elements whose quotient rounds
+// above FMAX on the grid continued past it (ties to even: E4M3 |q| > 464, the tie going to 448;
+// E5M2 |q| >= 61440, the tie going to 65536); `und` += elements with x != 0 (NaN excluded)
+// whose code is +-0.
+template <int FMT>
+__device__ __forceinline__ void count8(uint4 v, uint2 codes, const GroupScale& g, uint32_t& sat, uint32_t& und) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float x = (i & 1) ? bf16_hi(w[i >> 1]) : bf16_lo(w[i >> 1]);
+    const uint32_t code = ((i < 4 ? codes.x : codes.y) >> (8 * (i & 3))) & 0xFFu;
+    if (g.d != 0.0f) {
+      const float a = fabsf(g.fast ? markstein_div(x, g.d, g.r) : __fdiv_rn(x, g.d));
+      sat += (FMT == kE4M3) ? (a > 464.0f) : (a >= 61440.0f);
+    }
+    und += (x == x && x != 0.0f && (code & 0x7Fu) == 0u);
+  }
 }
 
 }  // namespace fp8q

@@ -70,6 +70,15 @@ cudaError_t launch_quant_two_pass(const uint16_t* x0, const uint16_t* x1, uint8_
                                   float* s1, int ntens, int64_t rows, int64_t heads, int64_t head_dim, int fmt,
                                   float* ws, cudaStream_t st);
 
+// delayed scaling over the same groups as launch_quant_two_pass: step 0 scales from the groups'
+// own amax (two passes), step >= 1 from max(history) / FMAX in one pass; afterwards history
+// slot step % hlen ([hlen][heads] per tensor) holds this call's amax.  counters (optional, [2])
+// accumulate saturated and underflowed elements.
+cudaError_t launch_quant_delayed(const uint16_t* x0, const uint16_t* x1, uint8_t* c0, uint8_t* c1, float* s0,
+                                 float* s1, int ntens, int64_t rows, int64_t heads, int64_t head_dim, int fmt,
+                                 float* h0, float* h1, int64_t hlen, int64_t step, unsigned long long* counters,
+                                 float* ws, cudaStream_t st);
+
 // y = bf16(decode(code) * s) under a granularity (0 tensor, 1 1x128, 2 128x128)
 cudaError_t launch_dequant(const uint8_t* codes, const float* scales, int64_t rows, int64_t cols, int fmt,
                            int gran, uint16_t* y, cudaStream_t st);

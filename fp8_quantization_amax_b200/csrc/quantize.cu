@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_group128(const __grid_constant_
     fence_mbar_init();
   }
   const uint32_t nk = items_of_cta(p.nitems);
-  if (warp == kConsumerWarps && lane == 0) {
+  if (warp == kConsumerWarps && lane == 0 && nk > 0) {
     // warm L2 with this CTA's first boxes while the previous grid on the stream finishes
     tma_prefetch_desc(&tx);
     for (uint32_t k = 0; k < nk && k < (uint32_t)S; ++k) {
@@ -258,6 +258,8 @@ cudaError_t launch_quant_1x128(const uint16_t* x, int64_t rows, int64_t cols, in
 constexpr int kOnePass = 0;
 constexpr int kAmax = 1;
 constexpr int kCast = 2;
+constexpr int kDelayed = 3;   // delayed scaling: cast with scales from an amax history, and
+                              // record this call's per-CTA maxima like kAmax
 constexpr int kMaxGroups = 256;
 
 struct TileParams {
@@ -277,6 +279,10 @@ struct TileParams {
   int ngroups;
   int stages;
   uint32_t stage_bytes;
+  const float* h0;                 // kDelayed: amax histories [hlen][heads] of tensors 0 and 1
+  const float* h1;
+  int hlen;
+  unsigned long long* counters;    // kCast / kDelayed, optional: [2] saturated, underflowed (added to)
   uint32_t* err;
 };
 
@@ -305,9 +311,12 @@ __global__ void __launch_bounds__(kThreads, 2) k_tile128(const __grid_constant__
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = ring_base(smem_raw);
   __shared__ uint32_t red[2][kConsumerWarps];
-  __shared__ uint32_t wmax[MODE == kAmax ? kConsumerWarps : 1][MODE == kAmax ? kMaxGroups : 1];
+  constexpr bool kRecordsAmax = MODE == kAmax || MODE == kDelayed;
+  constexpr bool kUsesTable = MODE == kCast || MODE == kDelayed;
+  constexpr bool kCanCount = MODE == kCast || MODE == kDelayed;
+  __shared__ uint32_t wmax[kRecordsAmax ? kConsumerWarps : 1][kRecordsAmax ? kMaxGroups : 1];
   __shared__ uint32_t fold[MODE == kCast ? kMaxGroups : 1];
-  __shared__ GroupScale table[MODE == kCast ? kMaxGroups : 1];
+  __shared__ GroupScale table[kUsesTable ? kMaxGroups : 1];
   const int S = p.stages;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * p.stage_bytes);
   uint64_t* empty = full + kMaxStages;
@@ -320,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_tile128(const __grid_constant__
     fence_mbar_init();
   }
   const uint32_t nk = items_of_cta(p.nitems);
-  if (warp == kConsumerWarps && lane == 0) {
+  if (warp == kConsumerWarps && lane == 0 && nk > 0) {
     // warm L2 with this CTA's first boxes while the previous grid on the stream finishes
     tma_prefetch_desc(&t0);
     tma_prefetch_desc(&t1);
@@ -348,8 +357,22 @@ __global__ void __launch_bounds__(kThreads, 2) k_tile128(const __grid_constant__
   const int cpr = CPR > 0 ? CPR : p.cpr;
   const int nchunks = 128 * cpr;
 
-  if (MODE == kAmax) {
+  if (kRecordsAmax) {
     for (int g = lane; g < kMaxGroups; g += 32) wmax[warp][g] = 0u;
+    __syncwarp();
+  }
+  if (MODE == kDelayed) {
+    // the scale of each group comes from the largest amax of its history (entries >= 0 or NaN,
+    // which order like their bit patterns; NaN stays)
+    for (int g = t; g < p.ngroups; g += kConsumers) {
+      const int tens = g / p.heads, gl = g - tens * p.heads;
+      const float* h = tens ? p.h1 : p.h0;
+      uint32_t hm = 0u;
+      for (int j = 0; j < p.hlen; ++j) hm = max(hm, __float_as_uint(h[(size_t)j * p.heads + gl]));
+      table[g] = make_delayed_scale<FMT>(__uint_as_float(hm));
+      if (blockIdx.x == 0) (tens ? p.s1 : p.s0)[gl] = table[g].s;
+    }
+    named_barrier(1, kConsumers);
   }
   if (MODE == kCast) {
     // fold the partial maxima: non-negative floats (or NaN) order like their bit patterns
@@ -377,6 +400,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_tile128(const __grid_constant__
   constexpr int ROWSTEP = CPR > 0 ? kConsumers / PPR : 1;
   const int r0 = CPR > 0 ? t / PPR : 0, cp = CPR > 0 ? t % PPR : 0;
   const bool wide = (p.ld % 16) == 0;
+  const bool count = kCanCount && p.counters != nullptr;
+  uint32_t n_sat = 0, n_und = 0;
   int s = 0;
   uint32_t ph = 0;
   for (uint32_t k = 0; k < nk; ++k) {
@@ -413,13 +438,13 @@ __global__ void __launch_bounds__(kThreads, 2) k_tile128(const __grid_constant__
 #pragma unroll
       for (int d = 16; d >= 1; d >>= 1) m = absmax2(m, __shfl_xor_sync(0xFFFFFFFFu, m, d));
     }
-    if (MODE == kAmax) {
+    if (kRecordsAmax) {
       if (lane == 0) {
         const int g = (int)it.tens * p.heads + (p.head_groups ? (int)it.bj : 0);
         const uint32_t a = __float_as_uint(packed_amax_to_f32(m));
         wmax[warp][g] = max(wmax[warp][g], a);
       }
-      continue;
+      if (MODE == kAmax) continue;
     }
     GroupScale gs;
     if (MODE == kOnePass) {
@@ -441,15 +466,30 @@ __global__ void __launch_bounds__(kThreads, 2) k_tile128(const __grid_constant__
         uint8_t* dst = codes + (row_base + r0) * p.ld + col_base + cp * 16;
         const int64_t step = (int64_t)ROWSTEP * p.ld;
 #pragma unroll
-        for (int jp = 0; jp < MAXP; ++jp) st_stream_v4(dst + jp * step, quant16_fast<FMT>(va[jp], vb[jp], gs.d, gs.r));
+        for (int jp = 0; jp < MAXP; ++jp) {
+          const uint4 q = quant16_fast<FMT>(va[jp], vb[jp], gs.d, gs.r);
+          st_stream_v4(dst + jp * step, q);
+          if (count) {
+            count8<FMT>(va[jp], make_uint2(q.x, q.y), gs, n_sat, n_und);
+            count8<FMT>(vb[jp], make_uint2(q.z, q.w), gs, n_sat, n_und);
+          }
+        }
       } else {
 #pragma unroll
         for (int jp = 0; jp < MAXP; ++jp) {
           const int64_t row = row_base + r0 + jp * ROWSTEP;
           const int64_t col = col_base + cp * 16;
           uint8_t* dst = codes + row * p.ld + col;
-          if (row < p.rows && col < p.cols) st_stream_v2(dst, quant8<FMT>(va[jp], gs));
-          if (row < p.rows && col + 8 < p.cols) st_stream_v2(dst + 8, quant8<FMT>(vb[jp], gs));
+          if (row < p.rows && col < p.cols) {
+            const uint2 q = quant8<FMT>(va[jp], gs);
+            st_stream_v2(dst, q);
+            if (count) count8<FMT>(va[jp], q, gs, n_sat, n_und);
+          }
+          if (row < p.rows && col + 8 < p.cols) {
+            const uint2 q = quant8<FMT>(vb[jp], gs);
+            st_stream_v2(dst + 8, q);
+            if (count) count8<FMT>(vb[jp], q, gs, n_sat, n_und);
+          }
         }
       }
     } else {
@@ -460,12 +500,26 @@ __global__ void __launch_bounds__(kThreads, 2) k_tile128(const __grid_constant__
         const int64_t row = row_base + r;
         const int64_t col = col_base + cc * 8;
         const uint2 q = quant8<FMT>(va[j], gs);
-        if (c < nchunks && row < p.rows && col < p.cols) st_stream_v2(codes + row * p.ld + col, q);
+        if (c < nchunks && row < p.rows && col < p.cols) {
+          st_stream_v2(codes + row * p.ld + col, q);
+          if (count) count8<FMT>(va[j], q, gs, n_sat, n_und);
+        }
       }
     }
     if (MODE == kCast) release_stage(release, lane);
   }
-  if (MODE == kAmax) {
+  if (count) {
+#pragma unroll
+    for (int d = 16; d >= 1; d >>= 1) {
+      n_sat += __shfl_xor_sync(0xFFFFFFFFu, n_sat, d);
+      n_und += __shfl_xor_sync(0xFFFFFFFFu, n_und, d);
+    }
+    if (lane == 0) {
+      if (n_sat) atomicAdd(p.counters, (unsigned long long)n_sat);
+      if (n_und) atomicAdd(p.counters + 1, (unsigned long long)n_und);
+    }
+  }
+  if (kRecordsAmax) {
     named_barrier(1, kConsumers);
     for (int g = t; g < p.ngroups; g += kConsumers) {
       uint32_t mx = wmax[0][g];
@@ -528,6 +582,9 @@ static bool tile_setup(TileParams& p, CUtensorMap& m0, CUtensorMap& m1, const ui
   p.err = device_error_word();
   p.partials = nullptr;
   p.nparts = 0;
+  p.h0 = p.h1 = nullptr;
+  p.hlen = 0;
+  p.counters = nullptr;
   p.head_groups = 0;
   p.heads = 1;
   p.ngroups = ntens;
@@ -563,18 +620,16 @@ size_t two_pass_workspace_bytes(int ntens, int64_t heads) {
   return (size_t)kMaxPartials * (size_t)ntens * (size_t)std::max<int64_t>(heads, 1) * sizeof(float);
 }
 
-cudaError_t launch_quant_two_pass(const uint16_t* x0, const uint16_t* x1, uint8_t* c0, uint8_t* c1, float* s0,
-                                  float* s1, int ntens, int64_t rows, int64_t heads, int64_t head_dim, int fmt,
-                                  float* ws, cudaStream_t st) {
-  // per-tensor: boxes of 128 x 128 over [rows][heads * head_dim]; per-head: boxes of
-  // 128 tokens x head_dim, one group per (tensor, head)
+// shared set-up of the two-pass and delayed launches: boxes of 128 x 128 over
+// [rows][heads * head_dim] for per-tensor groups, 128 tokens x head_dim per (tensor, head)
+static bool group_setup(TileParams& p, CUtensorMap& m0, CUtensorMap& m1, const uint16_t* x0, const uint16_t* x1,
+                        uint8_t* c0, uint8_t* c1, float* s0, float* s1, int ntens, int64_t rows, int64_t heads,
+                        int64_t head_dim, float* ws) {
   const int64_t cols = heads * head_dim;
   const bool per_head = heads > 1;
   const int bc = per_head ? (int)head_dim : 128;
-  if (ntens * (per_head ? heads : 1) > kMaxGroups) return cudaErrorInvalidValue;
-  TileParams p;
-  CUtensorMap m0, m1;
-  if (!tile_setup(p, m0, m1, x0, x1, ntens, rows, cols, cols, bc)) return cudaErrorInvalidValue;
+  if (ntens * (per_head ? heads : 1) > kMaxGroups) return false;
+  if (!tile_setup(p, m0, m1, x0, x1, ntens, rows, cols, cols, bc)) return false;
   p.c0 = c0;
   p.c1 = ntens > 1 ? c1 : c0;
   p.s0 = s0;
@@ -583,9 +638,16 @@ cudaError_t launch_quant_two_pass(const uint16_t* x0, const uint16_t* x1, uint8_
   p.heads = per_head ? (int)heads : 1;
   p.ngroups = ntens * p.heads;
   p.partials = ws;
+  return true;
+}
+
+// the two passes; *nparts receives the number of partial rows pass 1 wrote (0 for empty input)
+static cudaError_t two_pass(TileParams& p, const CUtensorMap& m0, const CUtensorMap& m1, int fmt, cudaStream_t st,
+                            int* nparts) {
   if (p.nitems == 0) {
     // empty tensors: amax = 0 for every group, so pass 2 alone writes s = 0
     p.nparts = 0;
+    *nparts = 0;
     return launch_tile<kCast>(fmt, m0, m1, p, 1, st);
   }
   const int grid1 = (int)std::min<int64_t>((int64_t)p.nitems, std::min<int64_t>(kMaxPartials, 2 * device_sm_count()));
@@ -594,7 +656,61 @@ cudaError_t launch_quant_two_pass(const uint16_t* x0, const uint16_t* x1, uint8_
   cudaError_t e = launch_tile<kAmax>(fmt, m0, m1, p, grid1, st, &written);
   if (e != cudaSuccess) return e;
   p.nparts = written;   // partial rows pass 1 wrote (its grid size)
+  *nparts = written;
   return launch_tile<kCast>(fmt, m0, m1, p, written, st);
+}
+
+cudaError_t launch_quant_two_pass(const uint16_t* x0, const uint16_t* x1, uint8_t* c0, uint8_t* c1, float* s0,
+                                  float* s1, int ntens, int64_t rows, int64_t heads, int64_t head_dim, int fmt,
+                                  float* ws, cudaStream_t st) {
+  TileParams p;
+  CUtensorMap m0, m1;
+  if (!group_setup(p, m0, m1, x0, x1, c0, c1, s0, s1, ntens, rows, heads, head_dim, ws)) return cudaErrorInvalidValue;
+  int nparts = 0;
+  return two_pass(p, m0, m1, fmt, st, &nparts);
+}
+
+// ============================================================================ delayed scaling
+//
+// Step 0 has no history: the two passes above (the group's own amax).  Step t >= 1: one pass
+// (kDelayed) casting with s = RN(max(history) / FMAX) while it records per-CTA maxima.  Either
+// way k_history_update then folds the recorded maxima into history slot t mod hlen.
+
+__global__ void __launch_bounds__(256) k_history_update(const float* partials, int nparts, int ngroups, int heads,
+                                                        float* h0, float* h1, int64_t slot) {
+  allow_dependent_launch();
+  grid_dependency_wait();
+  for (int g = threadIdx.x; g < ngroups; g += blockDim.x) {
+    uint32_t m = 0u;   // amax values are >= 0 or NaN and order like their bit patterns
+    for (int c = 0; c < nparts; ++c) m = max(m, __float_as_uint(partials[(size_t)c * ngroups + g]));
+    const int tens = g / heads, gl = g - tens * heads;
+    (tens ? h1 : h0)[slot * heads + gl] = __uint_as_float(m);
+  }
+}
+
+cudaError_t launch_quant_delayed(const uint16_t* x0, const uint16_t* x1, uint8_t* c0, uint8_t* c1, float* s0,
+                                 float* s1, int ntens, int64_t rows, int64_t heads, int64_t head_dim, int fmt,
+                                 float* h0, float* h1, int64_t hlen, int64_t step, unsigned long long* counters,
+                                 float* ws, cudaStream_t st) {
+  TileParams p;
+  CUtensorMap m0, m1;
+  if (!group_setup(p, m0, m1, x0, x1, c0, c1, s0, s1, ntens, rows, heads, head_dim, ws)) return cudaErrorInvalidValue;
+  p.counters = counters;
+  p.h0 = h0;
+  p.h1 = ntens > 1 ? h1 : h0;
+  p.hlen = (int)hlen;
+  int nparts = 0;
+  cudaError_t e;
+  if (step == 0) {
+    e = two_pass(p, m0, m1, fmt, st, &nparts);
+  } else {
+    const int grid = (int)std::max<int64_t>(
+        1, std::min<int64_t>((int64_t)p.nitems, std::min<int64_t>(kMaxPartials, 2 * device_sm_count())));
+    e = launch_tile<kDelayed>(fmt, m0, m1, p, grid, st, &nparts);
+  }
+  if (e != cudaSuccess) return e;
+  return launch_pdl(k_history_update, dim3(1), dim3(256), 0, st, (const float*)ws, nparts, p.ngroups, p.heads, h0,
+                    ntens > 1 ? h1 : h0, step % hlen);
 }
 
 }  // namespace fp8q

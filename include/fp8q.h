@@ -201,6 +201,49 @@ FP8Q_API fp8q_status fp8_kv_quantize_noalloc(const void *k, const void *v, int64
                                              uint8_t *k_codes, uint8_t *v_codes, float *k_scales,
                                              float *v_scales, fp8q_stream_t stream);
 
+/* ---------------------------------------------------------------- delayed scaling */
+
+/*
+ * Per-tensor quantization with delayed scaling ([C] "scale 是控制面": the scale follows a
+ * history of amax values instead of the tensor being cast; [M] 二: the forward pass takes its
+ * scale factor from the previous micro-batch's max), with the overflow / underflow counts
+ * that section asks to be observable.
+ *   x             bf16 [rows][cols] (device); cols % 8 == 0
+ *   amax_history  fp32 [history_len] (device, read and written): amax values of earlier calls,
+ *                 zero-filled by the caller before step 0; entries must be >= 0 or NaN
+ *   step          this call's index, 0, 1, 2, ...: step 0 scales from x's own amax (two
+ *                 kernels, as fp8_quantize per-tensor); step t >= 1 uses
+ *                 s = RN(max(amax_history) / FMAX) and reads x once.  An all-zero history gives
+ *                 s = 0 and sign-only codes.  Afterwards amax_history[step % history_len] holds
+ *                 x's own amax.
+ *   codes         uint8 [rows][cols] (device, written);  scale: fp32 [1] (device, written)
+ *   counts        NULL, or uint64 [2] (device, 8-byte aligned) to which the call adds the
+ *                 number of elements that saturated (|x / s| rounds above FMAX: E4M3 > 464,
+ *                 E5M2 >= 61440) and of nonzero elements whose code is +-0
+ *   ws            at least fp8q_workspace_bytes(rows, cols, FP8Q_PER_TENSOR) bytes (device)
+ * history_len in 1 .. 2^20.  Calls that share a history must be ordered (one stream).
+ */
+FP8Q_API fp8q_status fp8_quantize_delayed(const void *x, int64_t rows, int64_t cols, fp8q_format f,
+                                          float *amax_history, int64_t history_len, int64_t step,
+                                          uint8_t *codes, float *scale, unsigned long long *counts,
+                                          void *ws, size_t ws_bytes, fp8q_stream_t stream);
+
+/*
+ * KV-cache quantization with delayed scaling, per tensor or per head (the two-pass
+ * granularities; per-head x 128-token is one pass already and returns FP8Q_ERR_UNSUPPORTED).
+ * Arguments as fp8_kv_quantize, plus histories as for fp8_quantize_delayed, one per tensor:
+ *   k_history, v_history   fp32 [history_len][heads] (per head) or [history_len] (per tensor)
+ *   counts                 NULL or uint64 [2], K and V together
+ *   ws                     at least fp8q_kv_workspace_bytes(tokens, heads, head_dim, g) bytes
+ * With step >= 1 the cache is read once (3 B per element instead of 5).
+ */
+FP8Q_API fp8q_status fp8_kv_quantize_delayed(const void *k, const void *v, int64_t tokens, int64_t heads,
+                                             int64_t head_dim, fp8q_format f, fp8q_kv_granularity g,
+                                             float *k_history, float *v_history, int64_t history_len,
+                                             int64_t step, uint8_t *k_codes, uint8_t *v_codes,
+                                             float *k_scales, float *v_scales, unsigned long long *counts,
+                                             void *ws, size_t ws_bytes, fp8q_stream_t stream);
+
 /* ---------------------------------------------------------------- GEMM */
 
 /*

@@ -87,6 +87,22 @@ def test_quantize_rejects(L, args, status):
     assert L.fp8_quantize(*args) == status
 
 
+def test_delayed_rejects(L):
+    a, m = ALIGNED, MISALIGNED
+    # (x, rows, cols, fmt, history, history_len, step, codes, scale, counts, ws, ws_bytes, stream)
+    assert L.fp8_quantize_delayed(a, 4, 8, 0, a, 0, 1, a, a, None, a, 1 << 20, None) == 1      # empty history
+    assert L.fp8_quantize_delayed(a, 4, 8, 0, a, 4, -1, a, a, None, a, 1 << 20, None) == 1     # negative step
+    assert L.fp8_quantize_delayed(a, 4, 8, 0, None, 4, 1, a, a, None, a, 1 << 20, None) == 1   # null history
+    assert L.fp8_quantize_delayed(a, 4, 8, 0, a, 4, 1, a, a, m, a, 1 << 20, None) == 1         # misaligned counts
+    assert L.fp8_quantize_delayed(a, 4, 8, 0, a, 4, 1, a, a, None, None, 0, None) == 3         # no workspace
+    assert L.fp8_quantize_delayed(a, 4, 8, 0, a, 1 << 21, 1, a, a, None, a, 1 << 20, None) == 2  # history too long
+    # (k, v, T, H, D, fmt, g, kh, vh, hlen, step, kc, vc, ks, vs, counts, ws, ws_bytes, stream)
+    assert L.fp8_kv_quantize_delayed(a, a, 16, 8, 128, 0, 2, a, a, 4, 1, a, a, a, a, None, a, 1 << 20, None) == 2
+    assert L.fp8_kv_quantize_delayed(a, a, 16, 8, 128, 0, 1, None, a, 4, 1, a, a, a, a, None, a, 1 << 20, None) == 1
+    assert L.fp8_kv_quantize_delayed(a, a, 16, 8, 128, 0, 1, a, a, 4, 1, a, a, a, a, None, None, 0, None) == 3
+    assert L.fp8_kv_quantize_delayed(a, a, 16, 0, 128, 0, 1, a, a, 4, 1, a, a, a, a, None, None, 0, None) == 0
+
+
 def test_dequantize_rejects(L):
     assert L.fp8_dequantize(ALIGNED, ALIGNED, 4, 12, 0, 1, ALIGNED, None) == 1
     assert L.fp8_dequantize(ALIGNED, None, 4, 8, 0, 1, ALIGNED, None) == 1
