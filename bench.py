@@ -359,6 +359,26 @@ def supplementary(device, stream, peaks, flush):
             ms = timed(batch, 5, stream, flush) / calls
             out["gemm_8b_up_m16"] = gemm_entry(m, W_SHAPE[0], W_SHAPE[1], ms, a, sa, ws, cbuf)
             out["gemm_8b_up_m16"]["timing"] = f"{calls} back-to-back calls over 4 weight copies, mean per call"
+            # the same decode GEMM from bf16 activations: the caller's two calls, and the linear
+            # entry point (the same two kernels as one call)
+            xb = dev_bf16(synth.activations(seed=1)[:m], device)
+
+            def two_step():
+                for i in range(calls):
+                    a2, s2 = fq.fp8_quantize(xb, fq.E4M3, fq.GROUP_1x128, codes=a, scales=sa)
+                    fq.fp8_gemm_blockscaled(a2, s2, copies[i % 4], ws, out=cbuf)
+
+            act_ws = torch.empty(fq.linear_act_workspace_bytes(m, W_SHAPE[1]), dtype=torch.uint8, device=device)
+
+            def fused():
+                for i in range(calls):
+                    fq.fp8_linear_dynamic(xb, copies[i % 4], ws, out=cbuf, act_ws=act_ws)
+
+            ms2 = timed(two_step, 5, stream, flush) / calls
+            ms3 = timed(fused, 5, stream, flush) / calls
+            out["linear_8b_m16_quantize_then_gemm"] = gemm_entry(m, W_SHAPE[0], W_SHAPE[1], ms2, a, sa, ws, cbuf)
+            out["linear_8b_m16_dynamic"] = gemm_entry(m, W_SHAPE[0], W_SHAPE[1], ms3, a, sa, ws, cbuf)
+            out["linear_8b_m16_dynamic"]["timing"] = "bf16 activations in; same batching as gemm_8b_up_m16"
             del copies, cbuf
             # decode on the 70B up-projection (one weight, 235 MB > L2)
             w70 = dev_bf16(synth.weight_70b(seed=4, which="up"), device)

@@ -22,6 +22,7 @@ __all__ = [
     "kv_workspace_bytes", "gemm_workspace_bytes", "scale_shape", "kv_scale_shape",
     "fp8_encode", "fp8_decode", "fp8_quantize", "fp8_dequantize", "fp8_kv_quantize",
     "fp8_kv_quantize_noalloc", "fp8_gemm_blockscaled", "fp8_quantize_delayed", "fp8_kv_quantize_delayed",
+    "linear_act_workspace_bytes", "fp8_linear_dynamic",
 ]
 
 E4M3, E5M2 = 0, 1
@@ -68,6 +69,9 @@ def lib() -> ctypes.CDLL:
             L.fp8q_kv_workspace_bytes.restype = sz
             L.fp8q_gemm_workspace_bytes.argtypes = [i64, i64, i64]
             L.fp8q_gemm_workspace_bytes.restype = sz
+            L.fp8q_linear_act_workspace_bytes.argtypes = [i64, i64]
+            L.fp8q_linear_act_workspace_bytes.restype = sz
+            L.fp8_linear_dynamic.argtypes = [vp, i64, i64, i64, vp, vp, i32, vp, vp, sz, vp, sz, vp]
             L.fp8_encode.argtypes = [vp, i64, i32, vp, vp]
             L.fp8_decode.argtypes = [vp, i64, i32, vp, vp]
             L.fp8_quantize.argtypes = [vp, i64, i64, i32, i32, vp, vp, vp, sz, vp]
@@ -80,7 +84,7 @@ def lib() -> ctypes.CDLL:
                                                   vp, vp, sz, vp]
             for fn in ("fp8_encode", "fp8_decode", "fp8_quantize", "fp8_dequantize", "fp8_kv_quantize",
                        "fp8_gemm_blockscaled", "fp8_kv_quantize_noalloc", "fp8_quantize_delayed",
-                       "fp8_kv_quantize_delayed"):
+                       "fp8_kv_quantize_delayed", "fp8_linear_dynamic"):
                 getattr(L, fn).restype = i32
             _lib = L
     return _lib
@@ -388,4 +392,36 @@ def fp8_gemm_blockscaled(a: torch.Tensor, sa: torch.Tensor, b: torch.Tensor, sb:
     if st != 0 and cached:
         _gemm_ws.clear()
     _check("fp8_gemm_blockscaled", st)
+    return out
+
+
+def linear_act_workspace_bytes(M: int, K: int) -> int:
+    return int(lib().fp8q_linear_act_workspace_bytes(M, K))
+
+
+def fp8_linear_dynamic(x: torch.Tensor, b: torch.Tensor, sb: torch.Tensor, gb: int = BLOCK_128x128,
+                       out: torch.Tensor | None = None, act_ws: torch.Tensor | None = None,
+                       ws: torch.Tensor | None = None) -> torch.Tensor:
+    """C[M][N] (bf16) = block-scaled FP8 GEMM of the dynamically 1x128-quantized bf16 x [M][K] and
+    B [N][K] (E4M3 codes): bit-identical to fp8_quantize(x, E4M3, GROUP_1x128) followed by
+    fp8_gemm_blockscaled.  act_ws receives the codes and scales (allocated when not given); ws is
+    the GEMM workspace (the zero-filled buffer kept per device and stream when not given)."""
+    _dev(x, "x", torch.bfloat16)
+    _dev(b, "b", torch.uint8)
+    _dev(sb, "sb", torch.float32)
+    M, K = x.shape
+    N, K2 = b.shape
+    if K != K2:
+        raise ValueError("x and b disagree on K")
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if out is None else _dev(out, "out", torch.bfloat16)
+    act_ws = _workspace(linear_act_workspace_bytes(M, K), x.device, act_ws)
+    cached = ws is None
+    if cached:
+        ws = _gemm_workspace(gemm_workspace_bytes(M, N, K), x.device)
+    st = lib().fp8_linear_dynamic(_ptr(x), M, N, K, _ptr(b), _ptr(sb), gb, _ptr(out), _ptr(act_ws),
+                                  0 if act_ws is None else act_ws.numel() * act_ws.element_size(), _ptr(ws),
+                                  0 if ws is None else ws.numel() * ws.element_size(), _stream(x.device))
+    if st != 0 and cached:
+        _gemm_ws.clear()
+    _check("fp8_linear_dynamic", st)
     return out

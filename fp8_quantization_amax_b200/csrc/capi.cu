@@ -75,6 +75,11 @@ size_t fp8q_kv_workspace_bytes(int64_t tokens, int64_t heads, int64_t head_dim, 
   return 0;
 }
 
+size_t fp8q_linear_act_workspace_bytes(int64_t M, int64_t K) {
+  if (M <= 0 || K <= 0 || K % 128 != 0 || checked_elems(M, K) < 0) return 0;
+  return fp8q::linear_act_workspace_bytes(M, K);
+}
+
 size_t fp8q_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   if (M < 0 || N < 0 || K < 0) return 0;
   return fp8q::gemm_workspace_bytes(M, N, K);
@@ -226,6 +231,28 @@ fp8q_status fp8_gemm_blockscaled(const uint8_t* A, const float* sA, fp8q_granula
   if (need > 0 && (!ws || ws_bytes < need || !aligned(ws, 16))) return FP8Q_ERR_WORKSPACE;
   const cudaError_t e = fp8q::launch_gemm(A, sA, gA, B, sB, gB, M, N, K, static_cast<uint16_t*>(C), ws, ws_bytes,
                                           (cudaStream_t)stream);
+  if (e == cudaErrorNotSupported) return FP8Q_ERR_UNSUPPORTED;
+  return from_cuda(e);
+}
+
+fp8q_status fp8_linear_dynamic(const void* X, int64_t M, int64_t N, int64_t K, const uint8_t* B, const float* sB,
+                               fp8q_granularity gB, void* C, void* act_ws, size_t act_ws_bytes, void* gemm_ws,
+                               size_t gemm_ws_bytes, fp8q_stream_t stream) {
+  if (M < 0 || N < 0 || K < 0) return FP8Q_ERR_INVALID_ARGUMENT;
+  if (!(gB == FP8Q_BLOCK_128x128 || gB == FP8Q_PER_TENSOR)) return FP8Q_ERR_INVALID_ARGUMENT;
+  if (M == 0 || N == 0) return FP8Q_OK;
+  if (N % 128 != 0 || K % 128 != 0 || K == 0) return FP8Q_ERR_UNSUPPORTED;
+  if (checked_elems(M, K) < 0 || checked_elems(N, K) < 0 || checked_elems(M, N) < 0) return FP8Q_ERR_UNSUPPORTED;
+  if (M > (int64_t(1) << 31) - 1 || N > (int64_t(1) << 31) - 1) return FP8Q_ERR_UNSUPPORTED;
+  if (!X || !B || !C || !sB || !aligned(X, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(sB, 4))
+    return FP8Q_ERR_INVALID_ARGUMENT;
+  if (!act_ws || act_ws_bytes < fp8q::linear_act_workspace_bytes(M, K) || !aligned(act_ws, 16))
+    return FP8Q_ERR_WORKSPACE;
+  const size_t need = fp8q::gemm_workspace_bytes(M, N, K);
+  if (need > 0 && (!gemm_ws || gemm_ws_bytes < need || !aligned(gemm_ws, 16))) return FP8Q_ERR_WORKSPACE;
+  const cudaError_t e = fp8q::launch_linear(static_cast<const uint16_t*>(X), B, sB, gB, M, N, K,
+                                            static_cast<uint16_t*>(C), act_ws, gemm_ws, gemm_ws_bytes,
+                                            (cudaStream_t)stream);
   if (e == cudaErrorNotSupported) return FP8Q_ERR_UNSUPPORTED;
   return from_cuda(e);
 }

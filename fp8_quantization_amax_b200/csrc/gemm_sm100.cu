@@ -437,8 +437,8 @@ constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + (2 * kStages + 4) *
 // A tile that lies wholly in one CTA's range is rounded to bf16 and stored directly.  A tile
 // shared by several CTAs: each writes its fp32 partial to the workspace and counts itself in on
 // the tile's counter; the CTA that completes the count adds the partials in ascending CTA order
-// (deterministic: the same sum whichever CTA finishes last), stores the tile and resets the
-// counter to zero, so the workspace is zero again after every call.
+// (deterministic: the same sum whichever CTA finishes last), stores the tile, and clears the
+// partials and the counter, so every completed call leaves the whole workspace zero.
 //   warp 0 TMA producer, warp 1 MMA issuer (four TMEM buffers), warp 2 scale producer,
 //   warps 3-6 promotion.
 namespace dec {
@@ -701,21 +701,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
           if (finish) {
             // sum the tile's partials in ascending CTA order (this CTA's own included: each
             // thread re-reads the row it wrote), so the result does not depend on which CTA
-            // finishes last
+            // finishes last; then clear them, so that a completed call leaves the whole
+            // workspace zero whatever the shape of the next call that reuses it
             __threadfence();
 #pragma unroll
             for (int m = 0; m < MP; ++m) acc[m] = 0.0f;
 #pragma unroll 1
             for (uint32_t c = c_first; c <= c_last; ++c) {
               const uint32_t clo = range_lo(c, p.W, p.G);
-              const float* src = p.partials + ((size_t)(c * (uint32_t)p.maxseg + (t - clo / nkb)) * MP) * BM + row;
+              float* src = p.partials + ((size_t)(c * (uint32_t)p.maxseg + (t - clo / nkb)) * MP) * BM + row;
 #pragma unroll
               for (int m0 = 0; m0 < MP; m0 += 16) {
                 float part[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) part[j] = __ldcg(src + (size_t)(m0 + j) * BM);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) acc[m0 + j] += part[j];
+                for (int j = 0; j < 16; ++j) {
+                  acc[m0 + j] += part[j];
+                  src[(size_t)(m0 + j) * BM] = 0.0f;
+                }
               }
             }
           }
@@ -881,6 +885,26 @@ cudaError_t launch_gemm(const uint8_t* A, const float* sA, int gA, const uint8_t
     }
     return launch_pdl(k_gemm<false>, dim3(grid), dim3(kThreads), kSmemBytes, st, mA, mB, p);
   }
+}
+
+// Linear layer with dynamic activation quantization: C = GEMM(quantize_1x128_E4M3(X), B), as the
+// 1x128 quantizer into act_ws followed by the block-scaled GEMM (two programmatic-dependent
+// launches; for decode shapes the codes stay in L2 between them).  gemm_ws is the GEMM's own
+// workspace (decode shapes), with its zero-fill rule.
+size_t linear_act_workspace_bytes(int64_t M, int64_t K) {
+  const size_t codes = ((size_t)M * (size_t)K + 255) / 256 * 256;
+  return codes + (size_t)((K + 127) / 128) * (size_t)M * sizeof(float);
+}
+
+cudaError_t launch_linear(const uint16_t* X, const uint8_t* B, const float* sB, int gB, int64_t M, int64_t N,
+                          int64_t K, uint16_t* C, void* act_ws, void* gemm_ws, size_t gemm_ws_bytes,
+                          cudaStream_t st) {
+  if (M == 0 || N == 0) return cudaSuccess;
+  uint8_t* codes = static_cast<uint8_t*>(act_ws);
+  float* scales = reinterpret_cast<float*>(codes + ((size_t)M * (size_t)K + 255) / 256 * 256);
+  const cudaError_t e = launch_quant_1x128(X, M, K, 0, codes, scales, st);
+  if (e != cudaSuccess) return e;
+  return launch_gemm(codes, scales, 1, B, sB, gB, M, N, K, C, gemm_ws, gemm_ws_bytes, st);
 }
 
 }  // namespace fp8q

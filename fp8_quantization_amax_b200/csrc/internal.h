@@ -89,4 +89,11 @@ cudaError_t launch_gemm(const uint8_t* A, const float* sA, int gA, const uint8_t
                         cudaStream_t st);
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
+// C = GEMM(quantize_1x128_E4M3(X), B) for bf16 X [M][K]: the 1x128 quantizer into act_ws
+// (linear_act_workspace_bytes) and the block-scaled GEMM with gemm_ws
+size_t linear_act_workspace_bytes(int64_t M, int64_t K);
+cudaError_t launch_linear(const uint16_t* X, const uint8_t* B, const float* sB, int gB, int64_t M, int64_t N,
+                          int64_t K, uint16_t* C, void* act_ws, void* gemm_ws, size_t gemm_ws_bytes,
+                          cudaStream_t st);
+
 }  // namespace fp8q

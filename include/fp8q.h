@@ -262,7 +262,8 @@ FP8Q_API fp8q_status fp8_kv_quantize_delayed(const void *k, const void *v, int64
  * partial sums added in a fixed order, so results are deterministic.  ws: caller-owned device
  * memory of at least fp8q_gemm_workspace_bytes(M, N, K) bytes, 16-byte aligned (else
  * FP8Q_ERR_WORKSPACE), which must be ZERO-FILLED before its first use; every call that runs
- * to completion leaves it zero-filled again, so it can be reused as is.  After a device error
+ * to completion leaves all of it zero-filled again (counters and partial sums), so it can be
+ * reused as is, by calls of any shape.  After a device error
  * (fp8q_device_status() != 0) zero it again.  Calls that may run concurrently (e.g. on
  * unordered streams) need separate workspaces.  A counter found non-zero raises device error
  * bit 1 and leaves the affected output tiles unwritten.
@@ -273,6 +274,26 @@ FP8Q_API fp8q_status fp8_gemm_blockscaled(const uint8_t *A, const float *sA, fp8
                                  const uint8_t *B, const float *sB, fp8q_granularity gB,
                                  int64_t M, int64_t N, int64_t K, void *C,
                                  void *ws, size_t ws_bytes, fp8q_stream_t stream);
+
+/*
+ * Linear layer with dynamic activation quantization ([W] "激活动态量化": per-token 1x128
+ * groups computed at run time, then "FP8 矩阵乘"):
+ *   C = fp8_gemm_blockscaled(codes, scales, FP8Q_GROUP_1x128, B, sB, gB)  with
+ *   (codes, scales) = fp8_quantize(X, E4M3, FP8Q_GROUP_1x128),
+ * bit-identical to those two calls, issued as two programmatic-dependent launches on `stream`
+ * (for decode shapes the codes stay in L2 between them).
+ *   X        bf16 [M][K] (device, K-major);  B, sB, gB, C as for fp8_gemm_blockscaled
+ *   act_ws   device, 16-byte aligned, at least fp8q_linear_act_workspace_bytes(M, K) bytes:
+ *            receives the activation codes and scales; needs no initialisation
+ *   gemm_ws  the GEMM's workspace, fp8q_gemm_workspace_bytes(M, N, K) bytes (may be NULL
+ *            when that is 0), under the zero-fill rule stated for fp8_gemm_blockscaled
+ * Requirements as for fp8_gemm_blockscaled: N % 128 == 0, K % 128 == 0.
+ */
+FP8Q_API size_t fp8q_linear_act_workspace_bytes(int64_t M, int64_t K);
+FP8Q_API fp8q_status fp8_linear_dynamic(const void *X, int64_t M, int64_t N, int64_t K, const uint8_t *B,
+                                        const float *sB, fp8q_granularity gB, void *C, void *act_ws,
+                                        size_t act_ws_bytes, void *gemm_ws, size_t gemm_ws_bytes,
+                                        fp8q_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -148,6 +148,19 @@ def test_gemm_decode_workspace_left_zero(orc):
     assert fq.device_status() == 0
 
 
+def test_gemm_decode_workspace_reused_across_shapes(orc):
+    """One zero-filled workspace serves decode calls of different shapes in turn: after each call
+    the whole workspace (counters and partial sums) is zero again."""
+    ws = torch.zeros(fq.gemm_workspace_bytes(64, 14336, 4096), dtype=torch.uint8, device="cuda")
+    for (M, N, K) in [(16, 1024, 4096), (64, 2048, 1280), (16, 14336, 4096), (33, 384, 640)]:
+        a, sa, b, sb = operands(orc, M, N, K, 1, 2, seed=M * 7 + N)
+        got = fq.fp8_gemm_blockscaled(dev(a), dev(sa), dev(b), dev(sb), 1, 2, ws=ws)
+        torch.cuda.synchronize()
+        assert int(ws.count_nonzero()) == 0, (M, N, K)
+        check_tolerance(host(got), orc.gemm_rows(a, sa, 1, b, sb, 2, np.arange(M)), f"{M}x{N}x{K}")
+    assert fq.device_status() == 0
+
+
 def test_gemm_decode_dirty_workspace_is_reported(orc):
     """Counters that are not zero on entry raise device error bit 1 (no wait depends on them)."""
     M, N, K = 16, 2048, 4096
