@@ -274,7 +274,8 @@ def supplementary(device, stream, peaks, flush):
     import synth
     out = {}
     hbm = peaks["hbm_gbs"]
-    fp8_peak = 2.0 * peaks["bf16_tflops"]
+    fp8_peak = 2.0 * peaks["bf16_tflops"]                                   # burst
+    fp8_peak_sustained = 2.0 * peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])   # under the power cap
 
     def gbs(nbytes, ms):
         return {"us": round(ms * 1e3, 2), "GB/s": round(nbytes / ms / 1e6, 1), "frac_hbm": round(nbytes / ms / 1e6 / hbm, 3)}
@@ -332,6 +333,7 @@ def supplementary(device, stream, peaks, flush):
             nbytes = a.numel() + n * k + c.numel() * 2 + sa.numel() * 4 + wscale.numel() * 4
             return {"us": round(ms * 1e3, 2), "TFLOP/s": round(flops / ms / 1e9, 1),
                     "frac_fp8_peak": round(flops / ms / 1e9 / fp8_peak, 3),
+                    "frac_fp8_peak_sustained": round(flops / ms / 1e9 / fp8_peak_sustained, 3),
                     "GB/s": round(nbytes / ms / 1e6, 1), "frac_hbm": round(nbytes / ms / 1e6 / hbm, 3)}
 
         try:
@@ -397,7 +399,30 @@ def supplementary(device, stream, peaks, flush):
             ms = timed(batch70, 5, stream, flush) / calls
             out["gemm_70b_up_m64"] = gemm_entry(64, b70.shape[0], b70.shape[1], ms, a70, sa70, s70, c70)
             out["gemm_70b_up_m64"]["timing"] = f"{calls} back-to-back calls (weight 235 MB > L2), mean per call"
-            del b70, s70, a70, sa70, c70
+            del a70, sa70, c70
+            # prefill on the 70B up and down projections (M = 16384), block-scaled and per-tensor
+            for which in ("up", "down"):
+                if which == "down":
+                    del b70, s70
+                    w70 = dev_bf16(synth.weight_70b(seed=4, which="down"), device)
+                    b70, s70 = fq.fp8_quantize(w70, fq.E4M3, fq.BLOCK_128x128)
+                    del w70
+                x70 = dev_bf16(synth.activations_70b(seed=4, m=16384, which=which), device)
+                a70, sa70 = fq.fp8_quantize(x70, fq.E4M3, fq.GROUP_1x128)
+                del x70
+                c70 = torch.empty((16384, b70.shape[0]), dtype=torch.bfloat16, device=device)
+                fq.fp8_gemm_blockscaled(a70, sa70, b70, s70, out=c70)
+                ms = timed(lambda: fq.fp8_gemm_blockscaled(a70, sa70, b70, s70, out=c70), 3, stream, flush)
+                out[f"gemm_70b_{which}_m16384"] = gemm_entry(16384, b70.shape[0], b70.shape[1], ms, a70, sa70, s70, c70)
+                if which == "up":
+                    one = torch.ones(1, dtype=torch.float32, device=device)
+                    fq.fp8_gemm_blockscaled(a70, one, b70, one, fq.PER_TENSOR, fq.PER_TENSOR, out=c70)
+                    ms = timed(lambda: fq.fp8_gemm_blockscaled(a70, one, b70, one, fq.PER_TENSOR, fq.PER_TENSOR,
+                                                               out=c70), 3, stream, flush)
+                    out["gemm_70b_up_m16384_per_tensor"] = gemm_entry(16384, b70.shape[0], b70.shape[1], ms, a70, one,
+                                                                      one, c70)
+                del a70, sa70, c70
+            del b70, s70
         except fq.Fp8qError as err:
             out["gemm"] = f"not measured: {err}"
     return out
