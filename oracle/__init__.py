@@ -70,6 +70,12 @@ def _load():
             lib.orc_int8_level.restype = i32
             lib.orc_quantize_delayed.argtypes = [vp, i64, i64, i64, i32, vp, i64, i64, vp, vp, vp]
             lib.orc_quantize_delayed.restype = i32
+            lib.orc_mx_exponent.argtypes = [i32, f32]
+            lib.orc_mx_exponent.restype = i32
+            lib.orc_quantize_mx.argtypes = [vp, i64, i64, i32, vp, vp]
+            lib.orc_quantize_mx.restype = i32
+            lib.orc_dequantize_mx.argtypes = [vp, vp, i64, i64, i32, vp]
+            lib.orc_dequantize_mx.restype = i32
             _lib = lib
     return _lib
 
@@ -246,6 +252,36 @@ def quantize_delayed(x_bf16: np.ndarray, fmt: int, history: np.ndarray, step: in
                                       _p(codes), _p(scales), _p(cnt) if cnt is not None else None)
     assert rc == 0
     return codes, scales
+
+
+# ---------------------------------------------------------------- MXFP8 (1x32, power-of-two scales)
+
+def mx_exponent(amax: float, fmt: int) -> int:
+    """Smallest k with amax <= FMAX * 2^k (clamped at -127; 128 for NaN / Inf amax)."""
+    return int(_load().orc_mx_exponent(fmt, float(amax)))
+
+
+def quantize_mx(x_bf16: np.ndarray, fmt: int, threads: int | None = None):
+    """bf16 bits [rows][cols] (cols % 32 == 0) -> (codes uint8 [rows][cols], scales uint8 [rows][cols/32])."""
+    x = np.ascontiguousarray(x_bf16, np.uint16)
+    rows, cols = x.shape
+    codes = np.empty((rows, cols), np.uint8)
+    scales = np.empty((rows, cols // 32), np.uint8)
+    lib = _load()
+
+    def run(r0, n):
+        assert lib.orc_quantize_mx(_p(x[r0:r0 + n]), n, cols, fmt, _p(codes[r0:r0 + n]), _p(scales[r0:r0 + n])) == 0
+    _parallel(rows, run, threads, 64)
+    return codes, scales
+
+
+def dequantize_mx(codes: np.ndarray, scales: np.ndarray, fmt: int) -> np.ndarray:
+    c = np.ascontiguousarray(codes, np.uint8)
+    s = np.ascontiguousarray(scales, np.uint8)
+    rows, cols = c.shape
+    y = np.empty((rows, cols), np.uint16)
+    assert _load().orc_dequantize_mx(_p(c), _p(s), rows, cols, fmt, _p(y)) == 0
+    return y
 
 
 # ---------------------------------------------------------------- GEMM

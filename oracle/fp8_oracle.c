@@ -480,3 +480,61 @@ int orc_quantize_delayed(const uint16_t *x, int64_t rows, int64_t ngroups, int64
     FPENV_LEAVE;
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* MXFP8: 1x32 groups with power-of-two scales                               */
+/*
+ * [M] section on Microscaling (block size 32, native on Blackwell): per-block
+ * scaling with blocks of 32 elements.  The pages give no scale rule for it;
+ * the reading taken (design notes) is the pages' own rule restricted to powers
+ * of two: the scale of a group is the smallest 2^k with amax <= FMAX * 2^k (so
+ * the amax element never saturates), stored as the 8-bit exponent k + 127, k
+ * clamped at -127 (byte 0); an all-zero group takes byte 0; NaN or infinite
+ * amax takes byte 255 (a NaN scale).  Codes are FP8(RN(x / 2^k)).
+ */
+
+/* smallest k with amax <= fmax * 2^k, by exact comparison (both sides binary) */
+int orc_mx_exponent(int fmt, float amax) {
+    double fm = (double)fmt_of(fmt).fmax;
+    if (isnan(amax) || isinf(amax)) return 128;              /* NaN scale */
+    if (amax == 0.0f) return -127;
+    int k = 0;
+    while ((double)amax > ldexp(fm, k)) ++k;
+    while (k > -127 && (double)amax <= ldexp(fm, k - 1)) --k;
+    return k;
+}
+
+/* x bf16 [rows][cols], cols % 32 == 0; codes [rows][cols]; scales uint8 [rows][cols / 32] */
+int orc_quantize_mx(const uint16_t *x, int64_t rows, int64_t cols, int fmt, uint8_t *codes, uint8_t *scales) {
+    if (cols % 32 != 0) return -1;
+    FPENV_ENTER;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t g = 0; g < cols / 32; ++g) {
+            const uint16_t *xg = x + r * cols + g * 32;
+            float amax = region_amax(xg, 1, 32, 32);
+            int k = orc_mx_exponent(fmt, amax);
+            scales[r * (cols / 32) + g] = (uint8_t)(k + 127);
+            for (int c = 0; c < 32; ++c) {
+                float xv = bf16_value(xg[c]);
+                float q = (k == 128) ? xv / NAN : xv / (float)ldexp(1.0, k);
+                codes[r * cols + g * 32 + c] = orc_encode(fmt, q);
+            }
+        }
+    FPENV_LEAVE;
+    return 0;
+}
+
+/* y = RN_bf16(RN_fp32(decode(code) * 2^(byte - 127))); byte 255 is a NaN scale */
+int orc_dequantize_mx(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t cols, int fmt,
+                      uint16_t *y) {
+    if (cols % 32 != 0) return -1;
+    FPENV_ENTER;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c) {
+            int b = scales[r * (cols / 32) + c / 32];
+            float s = b == 255 ? NAN : (float)ldexp(1.0, b - 127);
+            y[r * cols + c] = bf16_round(orc_decode(fmt, codes[r * cols + c]) * s);
+        }
+    FPENV_LEAVE;
+    return 0;
+}

@@ -14,6 +14,7 @@ import pytest
 
 import test_oracle_codec as tc
 import test_oracle_delayed as td
+import test_oracle_mx as tmx
 import test_oracle_gemm as tg
 import test_oracle_quantize as tq
 
@@ -48,6 +49,11 @@ MUTANTS = {
     "saturation_tie_flipped": ("return (f.max_code & 1) != 0;", "return (f.max_code & 1) == 0;"),
     "saturation_at_fmax": ("if (a > mid) return 1;", "if (a > (double)f.fmax) return 1;"),
     "underflow_counts_zeros": ("if (!isnan(xv) && xv != 0.0f && (code & 0x7F) == 0)", "if (!isnan(xv) && (code & 0x7F) == 0)"),
+    "mx_exponent_not_minimal": ("(double)amax <= ldexp(fm, k - 1)) --k;", "(double)amax < ldexp(fm, k - 1)) --k;"),
+    "mx_scale_bias": ("scales[r * (cols / 32) + g] = (uint8_t)(k + 127);", "scales[r * (cols / 32) + g] = (uint8_t)(k + 128);"),
+    "mx_group_16": ("float amax = region_amax(xg, 1, 32, 32);", "float amax = region_amax(xg, 1, 16, 32);"),
+    "mx_dequant_drops_scale": ("y[r * cols + c] = bf16_round(orc_decode(fmt, codes[r * cols + c]) * s);",
+                               "y[r * cols + c] = bf16_round(orc_decode(fmt, codes[r * cols + c]));"),
 }
 
 
@@ -75,6 +81,9 @@ def _pins(m):
         lambda: td.test_ring_update_and_window_max(m),
         lambda: td.test_zero_history_gives_sign_only_codes(m),
         lambda: td.test_history_holding_the_current_amax_reduces_to_dynamic(m),
+        lambda: tmx.test_exponent_at_powers_of_two_of_fmax(m, 0),
+        lambda: tmx.test_bruteforce_tiny(m, 0, (3, 96)),
+        lambda: tmx.test_dequantize_matches_torch(m, 0),
         lambda: tg.test_closed_form_constant_operands(m),
         lambda: tg.test_matches_numpy_matmul(m, 1, 2, (130, 384, 256)),
         lambda: tg.test_blockwise_identity(m),
