@@ -323,6 +323,15 @@ def supplementary(device, stream, peaks, flush):
         ms = timed(delayed_call, 10, stream, flush)
         out["kv_head_e4m3_delayed"] = gbs(e2 * 3 + 2 * r[2].numel() * 4, ms)
         del kd, vd, r
+        # MXFP8 (1x32 groups, power-of-two scales) on the config-1 activations, and its dequantizer
+        xa = dev_bf16(synth.activations(seed=1), device)
+        mc, ms_ = fq.fp8_quantize_mx(xa)
+        ms = timed(lambda: fq.fp8_quantize_mx(xa, fq.E4M3, codes=mc, scales=ms_), 20, stream, flush)
+        out["mx_1x32_activations_8b"] = gbs(xa.numel() * 3 + ms_.numel(), ms)
+        ymx = torch.empty_like(xa)
+        ms = timed(lambda: fq.fp8_dequantize_mx(mc, ms_, fq.E4M3, out=ymx), 20, stream, flush)
+        out["mx_dequant_8b"] = gbs(xa.numel() * 3 + ms_.numel(), ms)
+        del xa, mc, ms_, ymx
         # GEMM (8B up-proj shape) on the quantized config-1 operands
         x = dev_bf16(synth.activations(seed=1), device)
         xc, xs = fq.fp8_quantize(x, fq.E4M3, fq.GROUP_1x128)

@@ -22,7 +22,7 @@ __all__ = [
     "kv_workspace_bytes", "gemm_workspace_bytes", "scale_shape", "kv_scale_shape",
     "fp8_encode", "fp8_decode", "fp8_quantize", "fp8_dequantize", "fp8_kv_quantize",
     "fp8_kv_quantize_noalloc", "fp8_gemm_blockscaled", "fp8_quantize_delayed", "fp8_kv_quantize_delayed",
-    "linear_act_workspace_bytes", "fp8_linear_dynamic",
+    "linear_act_workspace_bytes", "fp8_linear_dynamic", "fp8_quantize_mx", "fp8_dequantize_mx",
 ]
 
 E4M3, E5M2 = 0, 1
@@ -69,6 +69,8 @@ def lib() -> ctypes.CDLL:
             L.fp8q_kv_workspace_bytes.restype = sz
             L.fp8q_gemm_workspace_bytes.argtypes = [i64, i64, i64]
             L.fp8q_gemm_workspace_bytes.restype = sz
+            L.fp8_quantize_mx.argtypes = [vp, i64, i64, i32, vp, vp, vp]
+            L.fp8_dequantize_mx.argtypes = [vp, vp, i64, i64, i32, vp, vp]
             L.fp8q_linear_act_workspace_bytes.argtypes = [i64, i64]
             L.fp8q_linear_act_workspace_bytes.restype = sz
             L.fp8_linear_dynamic.argtypes = [vp, i64, i64, i64, vp, vp, i32, vp, vp, sz, vp, sz, vp]
@@ -84,7 +86,7 @@ def lib() -> ctypes.CDLL:
                                                   vp, vp, sz, vp]
             for fn in ("fp8_encode", "fp8_decode", "fp8_quantize", "fp8_dequantize", "fp8_kv_quantize",
                        "fp8_gemm_blockscaled", "fp8_kv_quantize_noalloc", "fp8_quantize_delayed",
-                       "fp8_kv_quantize_delayed", "fp8_linear_dynamic"):
+                       "fp8_kv_quantize_delayed", "fp8_linear_dynamic", "fp8_quantize_mx", "fp8_dequantize_mx"):
                 getattr(L, fn).restype = i32
             _lib = L
     return _lib
@@ -424,4 +426,32 @@ def fp8_linear_dynamic(x: torch.Tensor, b: torch.Tensor, sb: torch.Tensor, gb: i
     if st != 0 and cached:
         _gemm_ws.clear()
     _check("fp8_linear_dynamic", st)
+    return out
+
+
+def fp8_quantize_mx(x: torch.Tensor, fmt: int = E4M3, codes: torch.Tensor | None = None,
+                    scales: torch.Tensor | None = None):
+    """MXFP8: bf16 [rows][cols] (cols % 32 == 0) -> (codes uint8 [rows][cols], scales uint8
+    [rows][cols/32] holding k + 127 for the power-of-two scale 2^k)."""
+    _dev(x, "x", torch.bfloat16)
+    if x.dim() != 2:
+        raise ValueError("x must be 2-D [rows][cols]")
+    rows, cols = x.shape
+    codes = torch.empty((rows, cols), dtype=torch.uint8, device=x.device) if codes is None else _dev(codes, "codes", torch.uint8)
+    scales = torch.empty((rows, cols // 32), dtype=torch.uint8, device=x.device) if scales is None else \
+        _dev(scales, "scales", torch.uint8)
+    _check("fp8_quantize_mx", lib().fp8_quantize_mx(_ptr(x), rows, cols, fmt, _ptr(codes), _ptr(scales), _stream(x.device)))
+    return codes, scales
+
+
+def fp8_dequantize_mx(codes: torch.Tensor, scales: torch.Tensor, fmt: int = E4M3,
+                      out: torch.Tensor | None = None) -> torch.Tensor:
+    """MXFP8 codes + byte exponents -> bf16 [rows][cols]."""
+    _dev(codes, "codes", torch.uint8)
+    _dev(scales, "scales", torch.uint8)
+    rows, cols = codes.shape
+    out = torch.empty((rows, cols), dtype=torch.bfloat16, device=codes.device) if out is None else \
+        _dev(out, "out", torch.bfloat16)
+    _check("fp8_dequantize_mx", lib().fp8_dequantize_mx(_ptr(codes), _ptr(scales), rows, cols, fmt, _ptr(out),
+                                                       _stream(codes.device)))
     return out

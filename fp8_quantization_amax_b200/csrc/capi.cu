@@ -120,6 +120,28 @@ fp8q_status fp8_quantize(const void* x, int64_t rows, int64_t cols, fp8q_format 
       fp8q::launch_quant_tiles(xs, nullptr, codes, nullptr, scales, nullptr, 1, rows, cols, cols, 128, f, st));
 }
 
+fp8q_status fp8_quantize_mx(const void* x, int64_t rows, int64_t cols, fp8q_format f, uint8_t* codes,
+                            uint8_t* scales, fp8q_stream_t stream) {
+  const int64_t n = checked_elems(rows, cols);
+  if (rows < 0 || cols < 0 || !valid_fmt(f) || cols % 32 != 0) return FP8Q_ERR_INVALID_ARGUMENT;
+  if (n < 0) return FP8Q_ERR_UNSUPPORTED;
+  if (n == 0) return FP8Q_OK;
+  if (!x || !codes || !scales || !aligned(x, 16) || !aligned(codes, 16)) return FP8Q_ERR_INVALID_ARGUMENT;
+  return from_cuda(fp8q::launch_quant_mx(static_cast<const uint16_t*>(x), rows, cols, f, codes, scales,
+                                         (cudaStream_t)stream));
+}
+
+fp8q_status fp8_dequantize_mx(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols, fp8q_format f,
+                              void* y, fp8q_stream_t stream) {
+  const int64_t n = checked_elems(rows, cols);
+  if (rows < 0 || cols < 0 || !valid_fmt(f) || cols % 32 != 0) return FP8Q_ERR_INVALID_ARGUMENT;
+  if (n < 0) return FP8Q_ERR_UNSUPPORTED;
+  if (n == 0) return FP8Q_OK;
+  if (!codes || !scales || !y || !aligned(codes, 16) || !aligned(y, 16)) return FP8Q_ERR_INVALID_ARGUMENT;
+  return from_cuda(fp8q::launch_dequant(codes, reinterpret_cast<const float*>(scales), rows, cols, f, 3,
+                                        static_cast<uint16_t*>(y), (cudaStream_t)stream));
+}
+
 fp8q_status fp8_quantize_delayed(const void* x, int64_t rows, int64_t cols, fp8q_format f, float* amax_history,
                                  int64_t history_len, int64_t step, uint8_t* codes, float* scale,
                                  unsigned long long* counts, void* ws, size_t ws_bytes, fp8q_stream_t stream) {

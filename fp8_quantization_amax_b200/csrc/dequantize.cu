@@ -52,12 +52,17 @@ __global__ void __launch_bounds__(256) k_dequant(const uint8_t* __restrict__ cod
         c[k] = ld_stream_v2(codes + (size_t)i * 8);
         const uint32_t r = fdiv_u32(i, ppr);
         const uint32_t col = (i - r * ppr.d) * 8;
-        if (GRAN == 0)
+        if (GRAN == 0) {
           s[k] = __ldg(scales);
-        else if (GRAN == 1)
+        } else if (GRAN == 1) {
           s[k] = __ldg(scales + (size_t)(col >> 7) * rows + r);
-        else
+        } else if (GRAN == 2) {
           s[k] = __ldg(scales + (size_t)(r >> 7) * nbc + (col >> 7));
+        } else {
+          // MX: byte exponents [rows][cols / 32] (nbc = cols / 32), scale 2^(b - 127); 255 is NaN
+          const uint32_t b = __ldg(reinterpret_cast<const uint8_t*>(scales) + (size_t)r * nbc + (col >> 5));
+          s[k] = __uint_as_float(b == 255u ? 0x7FC00000u : (b == 0u ? 0x00400000u : b << 23));
+        }
       }
     }
 #pragma unroll
@@ -84,7 +89,7 @@ static cudaError_t launch_dequant_impl(const uint8_t* codes, const float* scales
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(need, (int64_t)device_sm_count() * occ));
   return launch_pdl(k_dequant<FMT, GRAN, kUnroll>, dim3(grid), dim3(256), 0, st, codes, scales, y,
                     (uint32_t)npieces, make_fastdiv((uint32_t)(cols / 8)), (uint32_t)rows,
-                    (uint32_t)((cols + 127) / 128));
+                    (uint32_t)(GRAN == 3 ? cols / 32 : (cols + 127) / 128));
 }
 
 template <int FMT>
@@ -92,7 +97,8 @@ static cudaError_t launch_dequant_fmt(const uint8_t* codes, const float* scales,
                                       int gran, uint16_t* y, cudaStream_t st) {
   if (gran == 0) return launch_dequant_impl<FMT, 0>(codes, scales, rows, cols, y, st);
   if (gran == 1) return launch_dequant_impl<FMT, 1>(codes, scales, rows, cols, y, st);
-  return launch_dequant_impl<FMT, 2>(codes, scales, rows, cols, y, st);
+  if (gran == 2) return launch_dequant_impl<FMT, 2>(codes, scales, rows, cols, y, st);
+  return launch_dequant_impl<FMT, 3>(codes, scales, rows, cols, y, st);   // MX: byte exponents
 }
 
 cudaError_t launch_dequant(const uint8_t* codes, const float* scales, int64_t rows, int64_t cols, int fmt,

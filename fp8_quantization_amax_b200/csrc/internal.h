@@ -79,7 +79,12 @@ cudaError_t launch_quant_delayed(const uint16_t* x0, const uint16_t* x1, uint8_t
                                  float* h0, float* h1, int64_t hlen, int64_t step, unsigned long long* counters,
                                  float* ws, cudaStream_t st);
 
-// y = bf16(decode(code) * s) under a granularity (0 tensor, 1 1x128, 2 128x128)
+// MXFP8: 1x32 groups along rows (cols % 32 == 0), scales as byte exponents [rows][cols / 32]
+cudaError_t launch_quant_mx(const uint16_t* x, int64_t rows, int64_t cols, int fmt, uint8_t* codes, uint8_t* scales,
+                            cudaStream_t st);
+
+// y = bf16(decode(code) * s) under a granularity (0 tensor, 1 1x128, 2 128x128, 3 MX 1x32 with
+// byte exponents passed through `scales`)
 cudaError_t launch_dequant(const uint8_t* codes, const float* scales, int64_t rows, int64_t cols, int fmt,
                            int gran, uint16_t* y, cudaStream_t st);
 

@@ -122,6 +122,7 @@ constexpr uint32_t kGroupStage = kGroupBoxRows * 128 * 2;
 struct GroupParams {
   uint8_t* codes;
   float* scales;
+  uint8_t* mx_scales;  // MX: [rows][cols / 32] power-of-two exponents (k + 127)
   int64_t rows, cols;
   uint32_t nitems;
   FastDiv ngc;        // 128-column groups per row
@@ -130,7 +131,34 @@ struct GroupParams {
   uint32_t* err;
 };
 
+// The exponent k of an MX group's scale 2^k: the smallest k with amax <= FMAX * 2^k, clamped at
+// -127; 128 for a NaN or infinite amax.  FMAX = 1.75 * 2^E (E = 8 for E4M3, 15 for E5M2), so for a
+// normal amax = M * 2^e: k = e - E, plus one when M > 1.75 (mantissa field above 0x600000).
 template <int FMT>
+__device__ __forceinline__ int mx_exponent(float amax) {
+  constexpr int kEmaxF = FMT == kE4M3 ? 8 : 15;
+  const uint32_t b = __float_as_uint(amax);
+  const int e = (int)(b >> 23);
+  if (e == 255) return 128;
+  if (e == 0) return -127;                    // zero or subnormal: below FMAX * 2^-127
+  return max(-127, e - 127 - kEmaxF + ((b & 0x7FFFFFu) > 0x600000u ? 1 : 0));
+}
+
+// eight bf16 times the power of two `mul` (exact) -> eight codes
+template <int FMT>
+__device__ __forceinline__ uint2 mx_quant8(uint4 v, float mul) {
+  const float2 m2 = make_float2(mul, mul);
+  const float2 a = __fmul2_rn(make_float2(bf16_lo(v.x), bf16_hi(v.x)), m2);
+  const float2 b = __fmul2_rn(make_float2(bf16_lo(v.y), bf16_hi(v.y)), m2);
+  const float2 c = __fmul2_rn(make_float2(bf16_lo(v.z), bf16_hi(v.z)), m2);
+  const float2 d = __fmul2_rn(make_float2(bf16_lo(v.w), bf16_hi(v.w)), m2);
+  return make_uint2(__byte_perm(cvt2<FMT>(a.x, a.y), cvt2<FMT>(b.x, b.y), 0x5410),
+                    __byte_perm(cvt2<FMT>(c.x, c.y), cvt2<FMT>(d.x, d.y), 0x5410));
+}
+
+// MX = false: 1x128 groups with fp32 scales.  MX = true: MXFP8, 1x32 groups with power-of-two
+// scales (one group per thread: thread q of a row's four takes columns [32q, 32q + 32) of the box).
+template <int FMT, bool MX>
 __global__ void __launch_bounds__(kThreads, 2) k_group128(const __grid_constant__ CUtensorMap tx, GroupParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = ring_base(smem_raw);
@@ -165,6 +193,39 @@ __global__ void __launch_bounds__(kThreads, 2) k_group128(const __grid_constant_
             const uint32_t rb = fdiv(i, p.ngc), g = i - rb * p.ngc.d;
             tma_load_2d(smem + s * kGroupStage, &tx, (int32_t)(g * 128), (int32_t)(rb * kGroupBoxRows), bar);
           });
+    }
+    return;
+  }
+  if constexpr (MX) {
+    const int t = threadIdx.x, grp = t >> 2, q = t & 3;
+    const uint32_t soff = grp * 256 + q * 64;
+    const int64_t ngroups = p.cols / 32;
+    int s = 0;
+    uint32_t ph = 0;
+    for (uint32_t k = 0; k < nk; ++k) {
+      const uint32_t i = blockIdx.x + k * gridDim.x;
+      if (!mbar_wait(&full[s], ph, p.err)) break;
+      const uint8_t* src = smem + s * kGroupStage + soff;
+      const uint4 v0 = ld_shared_v4(src), v1 = ld_shared_v4(src + 16), v2 = ld_shared_v4(src + 32),
+                  v3 = ld_shared_v4(src + 48);
+      const uint32_t m = absmax_v4(absmax_v4(absmax_v4(absmax_v4(0u, v0), v1), v2), v3);   // consumes every load
+      release_stage(&empty[s], lane);
+      if (++s == S) {
+        s = 0;
+        ph ^= 1u;
+      }
+      const int e = mx_exponent<FMT>(packed_amax_to_f32(m));
+      const float mul = e == 128 ? __uint_as_float(0x7FC00000u) : __uint_as_float((uint32_t)(127 - e) << 23);
+      const uint32_t rb = fdiv(i, p.ngc), g = i - rb * p.ngc.d;
+      const int64_t row = (int64_t)rb * kGroupBoxRows + grp;
+      const int64_t col0 = (int64_t)g * 128 + q * 32;
+      if (row >= p.rows || col0 >= p.cols) continue;
+      uint8_t* dst = p.codes + row * p.cols + col0;
+      const uint2 c0 = mx_quant8<FMT>(v0, mul), c1 = mx_quant8<FMT>(v1, mul), c2 = mx_quant8<FMT>(v2, mul),
+                  c3 = mx_quant8<FMT>(v3, mul);
+      st_stream_v4(dst, make_uint4(c0.x, c0.y, c1.x, c1.y));
+      st_stream_v4(dst + 16, make_uint4(c2.x, c2.y, c3.x, c3.y));
+      p.mx_scales[row * ngroups + g * 4 + q] = (uint8_t)(e + 127);
     }
     return;
   }
@@ -206,9 +267,9 @@ __global__ void __launch_bounds__(kThreads, 2) k_group128(const __grid_constant_
   }
 }
 
-template <int FMT>
+template <int FMT, bool MX>
 static cudaError_t launch_group128_fmt(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* codes,
-                                       float* scales, cudaStream_t st) {
+                                       float* scales, uint8_t* mx_scales, cudaStream_t st) {
   const int64_t ngc = (cols + 127) / 128, nrb = (rows + kGroupBoxRows - 1) / kGroupBoxRows;
   const int64_t nitems = ngc * nrb;
   if (nitems == 0) return cudaSuccess;
@@ -219,6 +280,7 @@ static cudaError_t launch_group128_fmt(const uint16_t* x, int64_t rows, int64_t 
   GroupParams p;
   p.codes = codes;
   p.scales = scales;
+  p.mx_scales = mx_scales;
   p.rows = rows;
   p.cols = cols;
   p.nitems = (uint32_t)nitems;
@@ -229,17 +291,23 @@ static cudaError_t launch_group128_fmt(const uint16_t* x, int64_t rows, int64_t 
   const size_t smem = ring_smem(p.stages, kGroupStage);
   static bool attr = false;
   if (!attr) {
-    cudaFuncSetAttribute(k_group128<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(k_group128<FMT, MX>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     attr = true;
   }
-  const int grid = grid_for(k_group128<FMT>, smem, p.nitems);
-  return launch_pdl(k_group128<FMT>, dim3(grid), dim3(kThreads), smem, st, map, p);
+  const int grid = grid_for(k_group128<FMT, MX>, smem, p.nitems);
+  return launch_pdl(k_group128<FMT, MX>, dim3(grid), dim3(kThreads), smem, st, map, p);
 }
 
 cudaError_t launch_quant_1x128(const uint16_t* x, int64_t rows, int64_t cols, int fmt, uint8_t* codes,
                                float* scales, cudaStream_t st) {
-  return fmt == kE4M3 ? launch_group128_fmt<kE4M3>(x, rows, cols, codes, scales, st)
-                      : launch_group128_fmt<kE5M2>(x, rows, cols, codes, scales, st);
+  return fmt == kE4M3 ? launch_group128_fmt<kE4M3, false>(x, rows, cols, codes, scales, nullptr, st)
+                      : launch_group128_fmt<kE5M2, false>(x, rows, cols, codes, scales, nullptr, st);
+}
+
+cudaError_t launch_quant_mx(const uint16_t* x, int64_t rows, int64_t cols, int fmt, uint8_t* codes, uint8_t* scales,
+                            cudaStream_t st) {
+  return fmt == kE4M3 ? launch_group128_fmt<kE4M3, true>(x, rows, cols, codes, nullptr, scales, st)
+                      : launch_group128_fmt<kE5M2, true>(x, rows, cols, codes, nullptr, scales, st);
 }
 
 // ============================================================================ 128-row tiles

@@ -201,6 +201,27 @@ FP8Q_API fp8q_status fp8_kv_quantize_noalloc(const void *k, const void *v, int64
                                              uint8_t *k_codes, uint8_t *v_codes, float *k_scales,
                                              float *v_scales, fp8q_stream_t stream);
 
+/* ---------------------------------------------------------------- MXFP8 */
+
+/*
+ * MXFP8 quantization: block scaling with blocks of 32 ([M] section on Microscaling, block
+ * size 32).  The scale of each 1x32 group of a row is a power of two 2^k, the smallest with
+ * amax <= FMAX * 2^k (the pages' rule s = amax / FMAX restricted to powers of two: no element
+ * saturates), stored as the byte k + 127 (k clamped at -127; 255 marks a NaN or infinite amax);
+ * codes = FP8(RN(x / 2^k)).
+ *   x       bf16 [rows][cols] (device, 16-byte aligned), cols % 32 == 0
+ *   codes   uint8 [rows][cols] (device, written)
+ *   scales  uint8 [rows][cols / 32] (device, written)
+ * Only the format: no GEMM consumes these scales here (a native block-scaled tensor-core
+ * product is not part of this library).
+ */
+FP8Q_API fp8q_status fp8_quantize_mx(const void *x, int64_t rows, int64_t cols, fp8q_format f, uint8_t *codes,
+                                     uint8_t *scales, fp8q_stream_t stream);
+
+/* y = bf16_rne(fp32(decode(code) * 2^(scale - 127))), layouts as fp8_quantize_mx. */
+FP8Q_API fp8q_status fp8_dequantize_mx(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t cols,
+                                       fp8q_format f, void *y, fp8q_stream_t stream);
+
 /* ---------------------------------------------------------------- delayed scaling */
 
 /*
