@@ -595,6 +595,21 @@ def our_arm(args):
             "gpu_launches": 2 * args.steps,
             "clocks": clocks,
         }
+    if rank == 0 and world == 1 and not args.no_supplementary:
+        # the step's two kernels each on its own, as 40 back-to-back launches over the input sets
+        # (dependent launches overlap each launch's start with the previous one's tail; no event
+        # between launches): context for the per-launch event times above
+        b2b = {}
+        with torch.cuda.stream(stream):
+            for name, fn, nbytes in (
+                    ("quant_128x128_weight", lambda j: fq.fp8_quantize(W[j], fq.E4M3, fq.BLOCK_128x128, codes=WC[j],
+                                                                      scales=WS[j]), bytes_w(n, k)),
+                    ("quant_1x128_activations", lambda j: fq.fp8_quantize(X[j], fq.E4M3, fq.GROUP_1x128, codes=XC[j],
+                                                                         scales=XS[j]), bytes_x(m, k))):
+                ms = timed(lambda: [fn(i % N_SETS) for i in range(40)], 5, stream, None) / 40
+                b2b[name] = {"us": round(ms * 1e3, 2), "GB/s": round(nbytes / ms / 1e6, 1),
+                             "frac_hbm": round(nbytes / ms / 1e6 / peaks["hbm_gbs"], 3)}
+        result["kernels_back_to_back"] = b2b
     del W, X, WC, XC
     if rank == 0 and world == 1:
         if not args.no_supplementary:

@@ -116,7 +116,8 @@ static int grid_for(K kernel, size_t smem, uint32_t nitems) {
 // (32 elements each, four 16-byte pieces), reduce it with two xor-shuffles, and store 32 codes.
 // The 64 scales of a box are 64 consecutive rows of one group column: one 256-byte run.
 
-constexpr uint32_t kGroupBoxRows = 64;
+constexpr uint32_t kGroupBoxRows = 128;      // box: 128 rows x 128 columns (32 KB)
+constexpr int kGroupRowsPerThread = kGroupBoxRows / 64;   // rows each of a row's four threads takes
 constexpr uint32_t kGroupStage = kGroupBoxRows * 128 * 2;
 
 struct GroupParams {
@@ -205,27 +206,37 @@ __global__ void __launch_bounds__(kThreads, 2) k_group128(const __grid_constant_
     for (uint32_t k = 0; k < nk; ++k) {
       const uint32_t i = blockIdx.x + k * gridDim.x;
       if (!mbar_wait(&full[s], ph, p.err)) break;
-      const uint8_t* src = smem + s * kGroupStage + soff;
-      const uint4 v0 = ld_shared_v4(src), v1 = ld_shared_v4(src + 16), v2 = ld_shared_v4(src + 32),
-                  v3 = ld_shared_v4(src + 48);
-      const uint32_t m = absmax_v4(absmax_v4(absmax_v4(absmax_v4(0u, v0), v1), v2), v3);   // consumes every load
-      release_stage(&empty[s], lane);
+      uint4 v[kGroupRowsPerThread][4];
+      uint32_t m[kGroupRowsPerThread];
+#pragma unroll
+      for (int h = 0; h < kGroupRowsPerThread; ++h) {
+        const uint8_t* src = smem + s * kGroupStage + soff + h * 64 * 256;
+        v[h][0] = ld_shared_v4(src);
+        v[h][1] = ld_shared_v4(src + 16);
+        v[h][2] = ld_shared_v4(src + 32);
+        v[h][3] = ld_shared_v4(src + 48);
+        m[h] = absmax_v4(absmax_v4(absmax_v4(absmax_v4(0u, v[h][0]), v[h][1]), v[h][2]), v[h][3]);
+      }
+      release_stage(&empty[s], lane);   // the amax consumed every load
       if (++s == S) {
         s = 0;
         ph ^= 1u;
       }
-      const int e = mx_exponent<FMT>(packed_amax_to_f32(m));
-      const float mul = e == 128 ? __uint_as_float(0x7FC00000u) : __uint_as_float((uint32_t)(127 - e) << 23);
       const uint32_t rb = fdiv(i, p.ngc), g = i - rb * p.ngc.d;
-      const int64_t row = (int64_t)rb * kGroupBoxRows + grp;
-      const int64_t col0 = (int64_t)g * 128 + q * 32;
-      if (row >= p.rows || col0 >= p.cols) continue;
-      uint8_t* dst = p.codes + row * p.cols + col0;
-      const uint2 c0 = mx_quant8<FMT>(v0, mul), c1 = mx_quant8<FMT>(v1, mul), c2 = mx_quant8<FMT>(v2, mul),
-                  c3 = mx_quant8<FMT>(v3, mul);
-      st_stream_v4(dst, make_uint4(c0.x, c0.y, c1.x, c1.y));
-      st_stream_v4(dst + 16, make_uint4(c2.x, c2.y, c3.x, c3.y));
-      p.mx_scales[row * ngroups + g * 4 + q] = (uint8_t)(e + 127);
+#pragma unroll
+      for (int h = 0; h < kGroupRowsPerThread; ++h) {
+        const int e = mx_exponent<FMT>(packed_amax_to_f32(m[h]));
+        const float mul = e == 128 ? __uint_as_float(0x7FC00000u) : __uint_as_float((uint32_t)(127 - e) << 23);
+        const int64_t row = (int64_t)rb * kGroupBoxRows + grp + h * 64;
+        const int64_t col0 = (int64_t)g * 128 + q * 32;
+        if (row >= p.rows || col0 >= p.cols) continue;
+        uint8_t* dst = p.codes + row * p.cols + col0;
+        const uint2 c0 = mx_quant8<FMT>(v[h][0], mul), c1 = mx_quant8<FMT>(v[h][1], mul),
+                    c2 = mx_quant8<FMT>(v[h][2], mul), c3 = mx_quant8<FMT>(v[h][3], mul);
+        st_stream_v4(dst, make_uint4(c0.x, c0.y, c1.x, c1.y));
+        st_stream_v4(dst + 16, make_uint4(c2.x, c2.y, c3.x, c3.y));
+        p.mx_scales[row * ngroups + g * 4 + q] = (uint8_t)(e + 127);
+      }
     }
     return;
   }
@@ -237,33 +248,43 @@ __global__ void __launch_bounds__(kThreads, 2) k_group128(const __grid_constant_
   for (uint32_t k = 0; k < nk; ++k) {
     const uint32_t i = blockIdx.x + k * gridDim.x;
     if (!mbar_wait(&full[s], ph, p.err)) break;
-    const uint8_t* src = smem + s * kGroupStage + soff;
-    const uint4 v0 = ld_shared_v4(src), v1 = ld_shared_v4(src + 16), v2 = ld_shared_v4(src + 128),
-                v3 = ld_shared_v4(src + 144);
-    uint32_t m = absmax_v4(absmax_v4(absmax_v4(absmax_v4(0u, v0), v1), v2), v3);   // consumes every load
-    release_stage(&empty[s], lane);
+    uint4 v[kGroupRowsPerThread][4];
+    uint32_t m[kGroupRowsPerThread];
+#pragma unroll
+    for (int h = 0; h < kGroupRowsPerThread; ++h) {
+      const uint8_t* src = smem + s * kGroupStage + soff + h * 64 * 256;
+      v[h][0] = ld_shared_v4(src);
+      v[h][1] = ld_shared_v4(src + 16);
+      v[h][2] = ld_shared_v4(src + 128);
+      v[h][3] = ld_shared_v4(src + 144);
+      m[h] = absmax_v4(absmax_v4(absmax_v4(absmax_v4(0u, v[h][0]), v[h][1]), v[h][2]), v[h][3]);
+    }
+    release_stage(&empty[s], lane);   // the amax consumed every load
     if (++s == S) {
       s = 0;
       ph ^= 1u;
     }
-    m = absmax2(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-    m = absmax2(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-    const GroupScale gs = make_group_scale<FMT>(packed_amax_to_f32(m));
     const uint32_t rb = fdiv(i, p.ngc), g = i - rb * p.ngc.d;
-    const int64_t row = (int64_t)rb * kGroupBoxRows + grp;
-    if (row >= p.rows) continue;
-    const int64_t col0 = (int64_t)g * 128 + q * 16, col1 = col0 + 64;
-    uint8_t* dst = p.codes + row * p.cols;
-    if (gs.fast && p.wide_stores && (int64_t)g * 128 + 128 <= p.cols) {
-      st_stream_v4(dst + col0, quant16_fast<FMT>(v0, v1, gs.d, gs.r));
-      st_stream_v4(dst + col1, quant16_fast<FMT>(v2, v3, gs.d, gs.r));
-    } else {
-      if (col0 < p.cols) st_stream_v2(dst + col0, quant8<FMT>(v0, gs));
-      if (col0 + 8 < p.cols) st_stream_v2(dst + col0 + 8, quant8<FMT>(v1, gs));
-      if (col1 < p.cols) st_stream_v2(dst + col1, quant8<FMT>(v2, gs));
-      if (col1 + 8 < p.cols) st_stream_v2(dst + col1 + 8, quant8<FMT>(v3, gs));
+#pragma unroll
+    for (int h = 0; h < kGroupRowsPerThread; ++h) {
+      uint32_t mh = absmax2(m[h], __shfl_xor_sync(0xFFFFFFFFu, m[h], 1));
+      mh = absmax2(mh, __shfl_xor_sync(0xFFFFFFFFu, mh, 2));
+      const GroupScale gs = make_group_scale<FMT>(packed_amax_to_f32(mh));
+      const int64_t row = (int64_t)rb * kGroupBoxRows + grp + h * 64;
+      if (row >= p.rows) continue;
+      const int64_t col0 = (int64_t)g * 128 + q * 16, col1 = col0 + 64;
+      uint8_t* dst = p.codes + row * p.cols;
+      if (gs.fast && p.wide_stores && (int64_t)g * 128 + 128 <= p.cols) {
+        st_stream_v4(dst + col0, quant16_fast<FMT>(v[h][0], v[h][1], gs.d, gs.r));
+        st_stream_v4(dst + col1, quant16_fast<FMT>(v[h][2], v[h][3], gs.d, gs.r));
+      } else {
+        if (col0 < p.cols) st_stream_v2(dst + col0, quant8<FMT>(v[h][0], gs));
+        if (col0 + 8 < p.cols) st_stream_v2(dst + col0 + 8, quant8<FMT>(v[h][1], gs));
+        if (col1 < p.cols) st_stream_v2(dst + col1, quant8<FMT>(v[h][2], gs));
+        if (col1 + 8 < p.cols) st_stream_v2(dst + col1 + 8, quant8<FMT>(v[h][3], gs));
+      }
+      if (q == 0) p.scales[(int64_t)g * p.rows + row] = gs.s;
     }
-    if (q == 0) p.scales[(int64_t)g * p.rows + row] = gs.s;
   }
 }
 
