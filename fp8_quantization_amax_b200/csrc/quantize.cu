@@ -769,11 +769,18 @@ __global__ void __launch_bounds__(256) k_history_update(const float* partials, i
                                                         float* h0, float* h1, int64_t slot) {
   allow_dependent_launch();
   grid_dependency_wait();
-  for (int g = threadIdx.x; g < ngroups; g += blockDim.x) {
-    uint32_t m = 0u;   // amax values are >= 0 or NaN and order like their bit patterns
-    for (int c = 0; c < nparts; ++c) m = max(m, __float_as_uint(partials[(size_t)c * ngroups + g]));
-    const int tens = g / heads, gl = g - tens * heads;
-    (tens ? h1 : h0)[slot * heads + gl] = __uint_as_float(m);
+  // one warp per group: lanes stride over the CTAs' partial maxima (independent loads), then a
+  // shuffle reduction; amax values are >= 0 or NaN and order like their bit patterns
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  for (int g = warp; g < ngroups; g += nwarps) {
+    uint32_t m = 0u;
+    for (int c = lane; c < nparts; c += 32) m = max(m, __float_as_uint(partials[(size_t)c * ngroups + g]));
+#pragma unroll
+    for (int d = 16; d >= 1; d >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, d));
+    if (lane == 0) {
+      const int tens = g / heads, gl = g - tens * heads;
+      (tens ? h1 : h0)[slot * heads + gl] = __uint_as_float(m);
+    }
   }
 }
 
