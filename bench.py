@@ -645,12 +645,27 @@ def profile_target(name, reps):
             b, sb = fq.fp8_quantize(w, fq.E4M3, fq.BLOCK_128x128)
             c = torch.empty((a.shape[0], b.shape[0]), dtype=torch.bfloat16, device=device)
             fn = lambda: fq.fp8_gemm_blockscaled(a, sa, b, sb, out=c)  # noqa: E731
+        elif name == "kv_delayed":
+            k, v = synth.kv_70b(seed=3)
+            kd, vd = dev_bf16(k, device), dev_bf16(v, device)
+            hk = torch.zeros((4, 8), dtype=torch.float32, device=device)
+            hv = torch.zeros_like(hk)
+            r = fq.fp8_kv_quantize_delayed(kd, vd, hk, hv, 0, fq.E4M3, fq.KV_PER_HEAD)
+            step_no = [0]
+
+            def fn():
+                step_no[0] += 1
+                fq.fp8_kv_quantize_delayed(kd, vd, hk, hv, step_no[0], fq.E4M3, fq.KV_PER_HEAD, *r)
         elif name.startswith("kv"):
             k, v = synth.kv_70b(seed=3)
             kd, vd = dev_bf16(k, device), dev_bf16(v, device)
             gran = fq.KV_PER_HEAD_TOK128 if name == "kv_tok128" else fq.KV_PER_HEAD
             r = fq.fp8_kv_quantize(kd, vd, fq.E4M3, gran)
             fn = lambda: fq.fp8_kv_quantize(kd, vd, fq.E4M3, gran, *r)  # noqa: E731
+        elif name == "mx_8b":
+            xa = dev_bf16(synth.activations(seed=1), device)
+            mc, msc = fq.fp8_quantize_mx(xa)
+            fn = lambda: fq.fp8_quantize_mx(xa, fq.E4M3, codes=mc, scales=msc)  # noqa: E731
         else:
             w = dev_bf16(synth.weight_8b(seed=1), device)
             wc, ws = fq.fp8_quantize(w, fq.E4M3, fq.BLOCK_128x128)
@@ -674,7 +689,7 @@ def main():
                     help="time the steps only: no e2e, CPU baseline or supplementary kernels (for profiling)")
     ap.add_argument("--profile-target", default=None,
                     choices=["gemm_8b_m8192", "gemm_8b_m16", "gemm_70b_up_m16384", "kv_tok128", "kv_head",
-                             "dequant_8b"],
+                             "kv_delayed", "mx_8b", "dequant_8b"],
                     help="run one workload a few times and exit (a small target for ncu)")
     args = ap.parse_args()
     if args.warmup < 3:
