@@ -280,6 +280,13 @@ def supplementary(device, stream, peaks, flush):
     def gbs(nbytes, ms):
         return {"us": round(ms * 1e3, 2), "GB/s": round(nbytes / ms / 1e6, 1), "frac_hbm": round(nbytes / ms / 1e6 / hbm, 3)}
 
+    def back_to_back(entry, fn, nbytes, calls=40):
+        """Add the mean of `calls` dependent launches (fn(i) over rotating inputs, no event in
+        between) to an entry timed per launch."""
+        ms = timed(lambda: [fn(i) for i in range(calls)], 5, stream, None) / calls
+        b = gbs(nbytes, ms)
+        entry["back_to_back"] = {"us": b["us"], "GB/s": b["GB/s"], "frac_hbm": b["frac_hbm"]}
+
     with torch.cuda.stream(stream):
         # per-tensor 1024x1024, E4M3 and E5M2, quantize + dequantize (launch-latency bound)
         t = dev_bf16(synth.per_tensor_1024(seed=0), device)
@@ -298,7 +305,12 @@ def supplementary(device, stream, peaks, flush):
         y = torch.empty_like(w)
         ms = timed(lambda: fq.fp8_dequantize(wc, ws, fq.E4M3, fq.BLOCK_128x128, out=y), 20, stream, flush)
         out["dequant_14336x4096_128x128"] = gbs(w.numel() * 3 + ws.numel() * 4, ms)
-        del y
+        wcs = [wc.clone() for _ in range(4)]          # 4 x 58.7 MB of codes and 2 x 117 MB of output > L2
+        ys = [y, torch.empty_like(w)]
+        back_to_back(out["dequant_14336x4096_128x128"],
+                     lambda i: fq.fp8_dequantize(wcs[i % 4], ws, fq.E4M3, fq.BLOCK_128x128, out=ys[i % 2]),
+                     w.numel() * 3 + ws.numel() * 4)
+        del y, ys, wcs
         # KV cache, 70B layer: [131072][8][128] for K and V
         k, v = synth.kv_70b(seed=3)
         kd, vd = dev_bf16(k, device), dev_bf16(v, device)
@@ -322,16 +334,25 @@ def supplementary(device, stream, peaks, flush):
 
         ms = timed(delayed_call, 10, stream, flush)
         out["kv_head_e4m3_delayed"] = gbs(e2 * 3 + 2 * r[2].numel() * 4, ms)
+        back_to_back(out["kv_head_e4m3_delayed"], lambda i: delayed_call(), e2 * 3 + 2 * r[2].numel() * 4, calls=8)
         del kd, vd, r
         # MXFP8 (1x32 groups, power-of-two scales) on the config-1 activations, and its dequantizer
         xa = dev_bf16(synth.activations(seed=1), device)
         mc, ms_ = fq.fp8_quantize_mx(xa)
         ms = timed(lambda: fq.fp8_quantize_mx(xa, fq.E4M3, codes=mc, scales=ms_), 20, stream, flush)
         out["mx_1x32_activations_8b"] = gbs(xa.numel() * 3 + ms_.numel(), ms)
+        xas = [xa] + [xa.clone() for _ in range(3)]    # 4 x 67 MB of activations > L2
+        back_to_back(out["mx_1x32_activations_8b"],
+                     lambda i: fq.fp8_quantize_mx(xas[i % 4], fq.E4M3, codes=mc, scales=ms_), xa.numel() * 3 + ms_.numel())
+        del xas
         ymx = torch.empty_like(xa)
         ms = timed(lambda: fq.fp8_dequantize_mx(mc, ms_, fq.E4M3, out=ymx), 20, stream, flush)
         out["mx_dequant_8b"] = gbs(xa.numel() * 3 + ms_.numel(), ms)
-        del xa, mc, ms_, ymx
+        mcs = [mc.clone() for _ in range(8)]          # 8 x 33.5 MB of codes and 4 x 67 MB of output > L2
+        ymxs = [ymx] + [torch.empty_like(xa) for _ in range(3)]
+        back_to_back(out["mx_dequant_8b"], lambda i: fq.fp8_dequantize_mx(mcs[i % 8], ms_, fq.E4M3, out=ymxs[i % 4]),
+                     xa.numel() * 3 + ms_.numel())
+        del xa, mc, ms_, ymx, mcs, ymxs
         # GEMM (8B up-proj shape) on the quantized config-1 operands
         x = dev_bf16(synth.activations(seed=1), device)
         xc, xs = fq.fp8_quantize(x, fq.E4M3, fq.GROUP_1x128)
