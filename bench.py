@@ -12,6 +12,9 @@ value  = algorithmic bytes of all ranks' steps / max-over-ranks device time (GB/
          step moves 2 B read + 1 B written per element plus 4 B per scale.
 e2e    = the same metric through the Python binding of the C ABI with pinned host buffers:
          each step copies the bf16 inputs host->device and codes + scales device->host.
+         Steps are pipelined over upload / compute / download streams and two device buffer
+         sets, as a streaming user would run them: one step's upload overlaps the previous
+         step's download (PCIe is full duplex), so a step costs about its upload time.
 roofline: the 128x128 weight kernel (the larger of the two), per-launch CUDA events.
 cpu_baseline: the CPU oracle on a bounded row sample of the same workload (rank 0, N = 1).
 supplementary: the other measured kernels (per-tensor, KV cache, dequantize, GEMM).
@@ -564,27 +567,50 @@ def our_arm(args):
     hws = torch.empty(WS[0].shape, dtype=torch.float32).pin_memory()
     hxs = torch.empty(XS[0].shape, dtype=torch.float32).pin_memory()
     e2e_steps = max(3, min(args.steps, 20))
-    with torch.cuda.stream(stream):
-        def e2e_step():
-            W[0].copy_(hw, non_blocking=True)
-            X[0].copy_(hx, non_blocking=True)
-            fq.fp8_quantize(W[0], fq.E4M3, fq.BLOCK_128x128, codes=WC[0], scales=WS[0])
-            fq.fp8_quantize(X[0], fq.E4M3, fq.GROUP_1x128, codes=XC[0], scales=XS[0])
-            hwc.copy_(WC[0], non_blocking=True)
-            hws.copy_(WS[0], non_blocking=True)
-            hxc.copy_(XC[0], non_blocking=True)
-            hxs.copy_(XS[0], non_blocking=True)
-        for _ in range(2):
-            e2e_step()
-        torch.cuda.synchronize(device)
-        barrier()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(e2e_steps):
-            e2e_step()
-        b.record(stream)
-        torch.cuda.synchronize(device)
-        barrier()
+    # a streaming pipeline: step i's upload (pinned host -> device), quantization and download
+    # (codes and scales -> pinned host) run on three streams over two device buffer sets, so the
+    # upload of step i + 1 and the download of step i - 1 overlap (PCIe is full duplex); events
+    # keep a set's inputs until its kernels have read them and its codes until they are copied
+    s_up, s_down = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev_up = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_down = [torch.cuda.Event() for _ in range(2)]
+
+    def e2e_step(i):
+        j = i % 2
+        with torch.cuda.stream(s_up):
+            if i >= 2:
+                s_up.wait_event(ev_done[j])
+            W[j].copy_(hw, non_blocking=True)
+            X[j].copy_(hx, non_blocking=True)
+            ev_up[j].record(s_up)
+        with torch.cuda.stream(stream):
+            stream.wait_event(ev_up[j])
+            if i >= 2:
+                stream.wait_event(ev_down[j])
+            fq.fp8_quantize(W[j], fq.E4M3, fq.BLOCK_128x128, codes=WC[j], scales=WS[j])
+            fq.fp8_quantize(X[j], fq.E4M3, fq.GROUP_1x128, codes=XC[j], scales=XS[j])
+            ev_done[j].record(stream)
+        with torch.cuda.stream(s_down):
+            s_down.wait_event(ev_done[j])
+            hwc.copy_(WC[j], non_blocking=True)
+            hws.copy_(WS[j], non_blocking=True)
+            hxc.copy_(XC[j], non_blocking=True)
+            hxs.copy_(XS[j], non_blocking=True)
+            ev_down[j].record(s_down)
+
+    for i in range(2):
+        e2e_step(i)
+    torch.cuda.synchronize(device)
+    barrier()
+    torch.cuda.synchronize(device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(s_up)
+    for i in range(2, 2 + e2e_steps):
+        e2e_step(i)
+    b.record(s_down)
+    torch.cuda.synchronize(device)
+    barrier()
     e2e_ms = reduce_max(a.elapsed_time(b), device)
     h2d = (hw.numel() + hx.numel()) * 2
     d2h = hwc.numel() + hxc.numel() + (hws.numel() + hxs.numel()) * 4
