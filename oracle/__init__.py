@@ -76,6 +76,8 @@ def _load():
             lib.orc_quantize_mx.restype = i32
             lib.orc_dequantize_mx.argtypes = [vp, vp, i64, i64, i32, vp]
             lib.orc_dequantize_mx.restype = i32
+            lib.orc_gemm_mx_rows.argtypes = [vp, vp, vp, vp, i32, i32, i64, i64, i64, vp, i64, vp]
+            lib.orc_gemm_mx_rows.restype = i32
             _lib = lib
     return _lib
 
@@ -282,6 +284,48 @@ def dequantize_mx(codes: np.ndarray, scales: np.ndarray, fmt: int) -> np.ndarray
     y = np.empty((rows, cols), np.uint16)
     assert _load().orc_dequantize_mx(_p(c), _p(s), rows, cols, fmt, _p(y)) == 0
     return y
+
+
+def mx_blocked_bytes(rows: int, cols: int) -> int:
+    """Size of the blocked MX scale layout: one 512-byte chunk per 128 rows x 128 columns."""
+    return cdiv(rows, 128) * cdiv(cols, 128) * 512
+
+
+def mx_blocked_scales(scales: np.ndarray) -> np.ndarray:
+    """Row-major MX scale bytes [rows][cols/32] -> the blocked layout the tensor cores' block-scaled
+    MMA reads (one 512-byte chunk per 128 rows x 4 scale columns, chunks ordered row block by row
+    block with the K blocks inside; in a chunk, byte 16*(r % 32) + 4*((r % 128) // 32) + (j % 4)
+    holds scale (r, j)).  Padding rows and columns hold byte 0."""
+    s = np.ascontiguousarray(scales, np.uint8)
+    rows, ng = s.shape
+    nrb, nkb = cdiv(rows, 128), cdiv(ng, 4)
+    out = np.zeros(nrb * nkb * 512, np.uint8)
+    r, j = np.indices((rows, ng))
+    off = ((r // 128) * nkb + j // 4) * 512 + 16 * (r % 32) + 4 * ((r % 128) // 32) + (j % 4)
+    out[off] = s
+    return out
+
+
+def gemm_mx_rows(a_codes, sa, b_codes, sb, rows, fmt_a: int = E4M3, fmt_b: int = E4M3,
+                 threads: int | None = None) -> np.ndarray:
+    """fp64 rows of the MXFP8 product C = (A * 2^(sA-127)) @ (B * 2^(sB-127))^T, scales row-major
+    [rows][K/32] bytes, for the listed row indices -> [len(rows)][N]."""
+    A = np.ascontiguousarray(a_codes, np.uint8)
+    B = np.ascontiguousarray(b_codes, np.uint8)
+    sA = np.ascontiguousarray(sa, np.uint8)
+    sB = np.ascontiguousarray(sb, np.uint8)
+    M, K = A.shape
+    N, K2 = B.shape
+    assert K == K2 and K % 32 == 0 and sA.shape == (M, K // 32) and sB.shape == (N, K // 32)
+    rows = np.ascontiguousarray(rows, np.int64)
+    out = np.empty((rows.size, N), np.float64)
+    lib = _load()
+
+    def run(i0, n):
+        assert lib.orc_gemm_mx_rows(_p(A), _p(sA), _p(B), _p(sB), fmt_a, fmt_b, M, N, K,
+                                    _p(rows[i0:i0 + n]), n, _p(out[i0:i0 + n])) == 0
+    _parallel(rows.size, run, threads, 4)
+    return out
 
 
 # ---------------------------------------------------------------- GEMM

@@ -538,3 +538,41 @@ int orc_dequantize_mx(const uint8_t *codes, const uint8_t *scales, int64_t rows,
     FPENV_LEAVE;
     return 0;
 }
+
+/*
+ * MXFP8 GEMM ([M] section on Microscaling: every 32 consecutive elements along K
+ * carry one power-of-two scale; [W] "FP8 矩阵乘": FP8 products, accumulation in
+ * high precision, the scales multiplied back):
+ *   C[m][n] = sum_k (decode(A[m][k]) * 2^(sA[m][k/32] - 127))
+ *                 * (decode(B[n][k]) * 2^(sB[n][k/32] - 127))            in fp64
+ * A [M][K] and B [N][K] codes (K % 32 == 0), scale bytes row-major [rows][K/32];
+ * byte 255 is a NaN scale.  Only the listed rows of C are computed:
+ * out[i][n] = C[rows[i]][n].
+ */
+static double mx_scale_value(uint8_t b) { return b == 255 ? NAN : ldexp(1.0, (int)b - 127); }
+
+int orc_gemm_mx_rows(const uint8_t *A, const uint8_t *sA, const uint8_t *B, const uint8_t *sB, int fmtA, int fmtB,
+                     int64_t M, int64_t N, int64_t K, const int64_t *rows, int64_t nrows, double *out) {
+    if (K % 32 != 0) return -1;
+    FPENV_ENTER;
+    const int64_t G = K / 32;
+    double *a = (double *)malloc(sizeof(double) * (size_t)(K * nrows));
+    double *b = (double *)malloc(sizeof(double) * (size_t)K);
+    for (int64_t i = 0; i < nrows; ++i)
+        for (int64_t k = 0; k < K; ++k)
+            a[i * K + k] = (double)orc_decode(fmtA, A[rows[i] * K + k]) * mx_scale_value(sA[rows[i] * G + k / 32]);
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k)
+            b[k] = (double)orc_decode(fmtB, B[n * K + k]) * mx_scale_value(sB[n * G + k / 32]);
+        for (int64_t i = 0; i < nrows; ++i) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) acc += a[i * K + k] * b[k];
+            out[i * N + n] = acc;
+        }
+    }
+    free(a);
+    free(b);
+    (void)M;
+    FPENV_LEAVE;
+    return 0;
+}

@@ -15,6 +15,7 @@ import pytest
 import test_oracle_codec as tc
 import test_oracle_delayed as td
 import test_oracle_mx as tmx
+import test_oracle_mx_gemm as tmg
 import test_oracle_gemm as tg
 import test_oracle_quantize as tq
 
@@ -52,6 +53,12 @@ MUTANTS = {
     "mx_exponent_not_minimal": ("(double)amax <= ldexp(fm, k - 1)) --k;", "(double)amax < ldexp(fm, k - 1)) --k;"),
     "mx_scale_bias": ("scales[r * (cols / 32) + g] = (uint8_t)(k + 127);", "scales[r * (cols / 32) + g] = (uint8_t)(k + 128);"),
     "mx_group_16": ("float amax = region_amax(xg, 1, 32, 32);", "float amax = region_amax(xg, 1, 16, 32);"),
+    "mx_gemm_group_128": ("mx_scale_value(sA[rows[i] * G + k / 32])", "mx_scale_value(sA[rows[i] * G + k / 128])"),
+    "mx_gemm_bias": ("ldexp(1.0, (int)b - 127)", "ldexp(1.0, (int)b - 126)"),
+    "mx_gemm_b_scale_transposed": ("mx_scale_value(sB[n * G + k / 32])", "mx_scale_value(sB[(k / 32) * N + n])"),
+    "mx_gemm_b_format_of_a": ("b[k] = (double)orc_decode(fmtB, B[n * K + k]) * mx_scale_value",
+                              "b[k] = (double)orc_decode(fmtA, B[n * K + k]) * mx_scale_value"),
+    "mx_gemm_nan_scale_ignored": ("return b == 255 ? NAN : ldexp", "return b == 255 ? 1.0 : ldexp"),
     "mx_dequant_drops_scale": ("y[r * cols + c] = bf16_round(orc_decode(fmt, codes[r * cols + c]) * s);",
                                "y[r * cols + c] = bf16_round(orc_decode(fmt, codes[r * cols + c]));"),
 }
@@ -84,6 +91,10 @@ def _pins(m):
         lambda: tmx.test_exponent_at_powers_of_two_of_fmax(m, 0),
         lambda: tmx.test_bruteforce_tiny(m, 0, (3, 96)),
         lambda: tmx.test_dequantize_matches_torch(m, 0),
+        lambda: tmg.test_uniform_scales_reduce_to_matmul(m, 0, 1),
+        lambda: tmg.test_one_group_special_case(m),
+        lambda: tmg.test_row_and_column_doubling(m),
+        lambda: tmg.test_nan_scale_poisons_its_row(m),
         lambda: tg.test_closed_form_constant_operands(m),
         lambda: tg.test_matches_numpy_matmul(m, 1, 2, (130, 384, 256)),
         lambda: tg.test_blockwise_identity(m),
