@@ -23,6 +23,7 @@ __all__ = [
     "fp8_encode", "fp8_decode", "fp8_quantize", "fp8_dequantize", "fp8_kv_quantize",
     "fp8_kv_quantize_noalloc", "fp8_gemm_blockscaled", "fp8_quantize_delayed", "fp8_kv_quantize_delayed",
     "linear_act_workspace_bytes", "fp8_linear_dynamic", "fp8_quantize_mx", "fp8_dequantize_mx",
+    "mx_blocked_scale_bytes", "fp8_quantize_mx_blocked", "fp8_gemm_mx",
 ]
 
 E4M3, E5M2 = 0, 1
@@ -71,6 +72,10 @@ def lib() -> ctypes.CDLL:
             L.fp8q_gemm_workspace_bytes.restype = sz
             L.fp8_quantize_mx.argtypes = [vp, i64, i64, i32, vp, vp, vp]
             L.fp8_dequantize_mx.argtypes = [vp, vp, i64, i64, i32, vp, vp]
+            L.fp8q_mx_blocked_scale_bytes.argtypes = [i64, i64]
+            L.fp8q_mx_blocked_scale_bytes.restype = sz
+            L.fp8_quantize_mx_blocked.argtypes = [vp, i64, i64, i32, vp, vp, vp]
+            L.fp8_gemm_mx.argtypes = [vp, vp, i32, vp, vp, i32, i64, i64, i64, vp, vp]
             L.fp8q_linear_act_workspace_bytes.argtypes = [i64, i64]
             L.fp8q_linear_act_workspace_bytes.restype = sz
             L.fp8_linear_dynamic.argtypes = [vp, i64, i64, i64, vp, vp, i32, vp, vp, sz, vp, sz, vp]
@@ -86,7 +91,8 @@ def lib() -> ctypes.CDLL:
                                                   vp, vp, sz, vp]
             for fn in ("fp8_encode", "fp8_decode", "fp8_quantize", "fp8_dequantize", "fp8_kv_quantize",
                        "fp8_gemm_blockscaled", "fp8_kv_quantize_noalloc", "fp8_quantize_delayed",
-                       "fp8_kv_quantize_delayed", "fp8_linear_dynamic", "fp8_quantize_mx", "fp8_dequantize_mx"):
+                       "fp8_kv_quantize_delayed", "fp8_linear_dynamic", "fp8_quantize_mx", "fp8_dequantize_mx",
+                       "fp8_quantize_mx_blocked", "fp8_gemm_mx"):
                 getattr(L, fn).restype = i32
             _lib = L
     return _lib
@@ -442,6 +448,50 @@ def fp8_quantize_mx(x: torch.Tensor, fmt: int = E4M3, codes: torch.Tensor | None
         _dev(scales, "scales", torch.uint8)
     _check("fp8_quantize_mx", lib().fp8_quantize_mx(_ptr(x), rows, cols, fmt, _ptr(codes), _ptr(scales), _stream(x.device)))
     return codes, scales
+
+
+def mx_blocked_scale_bytes(rows: int, cols: int) -> int:
+    """Bytes of the blocked MX scale layout (one 512-byte chunk per 128 rows x 128 columns)."""
+    return int(lib().fp8q_mx_blocked_scale_bytes(rows, cols))
+
+
+def fp8_quantize_mx_blocked(x: torch.Tensor, fmt: int = E4M3, codes: torch.Tensor | None = None,
+                            scales: torch.Tensor | None = None):
+    """MXFP8 as fp8_quantize_mx, with the scales in the blocked layout fp8_gemm_mx reads:
+    -> (codes uint8 [rows][cols], scales uint8 [mx_blocked_scale_bytes(rows, cols)])."""
+    _dev(x, "x", torch.bfloat16)
+    if x.dim() != 2:
+        raise ValueError("x must be 2-D [rows][cols]")
+    rows, cols = x.shape
+    codes = torch.empty((rows, cols), dtype=torch.uint8, device=x.device) if codes is None else _dev(codes, "codes", torch.uint8)
+    nbytes = mx_blocked_scale_bytes(rows, cols)
+    scales = torch.empty(nbytes, dtype=torch.uint8, device=x.device) if scales is None else \
+        _dev(scales, "scales", torch.uint8)
+    if scales.numel() < nbytes:
+        raise ValueError(f"scales needs {nbytes} bytes")
+    _check("fp8_quantize_mx_blocked", lib().fp8_quantize_mx_blocked(_ptr(x), rows, cols, fmt, _ptr(codes), _ptr(scales),
+                                                                   _stream(x.device)))
+    return codes, scales
+
+
+def fp8_gemm_mx(a: torch.Tensor, sa: torch.Tensor, b: torch.Tensor, sb: torch.Tensor, fa: int = E4M3,
+                fb: int = E4M3, out: torch.Tensor | None = None) -> torch.Tensor:
+    """C[M][N] (bf16) = MXFP8 product of A [M][K] (format fa) and B [N][K] (format fb), both with
+    blocked scales (fp8_quantize_mx_blocked), on the tensor cores' block-scaled MMA."""
+    _dev(a, "a", torch.uint8)
+    _dev(b, "b", torch.uint8)
+    _dev(sa, "sa", torch.uint8)
+    _dev(sb, "sb", torch.uint8)
+    M, K = a.shape
+    N, K2 = b.shape
+    if K != K2:
+        raise ValueError("a and b disagree on K")
+    if sa.numel() < mx_blocked_scale_bytes(M, K) or sb.numel() < mx_blocked_scale_bytes(N, K):
+        raise ValueError("blocked scales too small")
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device) if out is None else _dev(out, "out", torch.bfloat16)
+    _check("fp8_gemm_mx", lib().fp8_gemm_mx(_ptr(a), _ptr(sa), fa, _ptr(b), _ptr(sb), fb, M, N, K, _ptr(out),
+                                           _stream(a.device)))
+    return out
 
 
 def fp8_dequantize_mx(codes: torch.Tensor, scales: torch.Tensor, fmt: int = E4M3,

@@ -127,7 +127,23 @@ fp8q_status fp8_quantize_mx(const void* x, int64_t rows, int64_t cols, fp8q_form
   if (n < 0) return FP8Q_ERR_UNSUPPORTED;
   if (n == 0) return FP8Q_OK;
   if (!x || !codes || !scales || !aligned(x, 16) || !aligned(codes, 16)) return FP8Q_ERR_INVALID_ARGUMENT;
-  return from_cuda(fp8q::launch_quant_mx(static_cast<const uint16_t*>(x), rows, cols, f, codes, scales,
+  return from_cuda(fp8q::launch_quant_mx(static_cast<const uint16_t*>(x), rows, cols, f, codes, scales, 0,
+                                         (cudaStream_t)stream));
+}
+
+size_t fp8q_mx_blocked_scale_bytes(int64_t rows, int64_t cols) {
+  if (rows < 0 || cols < 0) return 0;
+  return (size_t)(cdiv(rows, 128) * cdiv(cols, 128) * 512);
+}
+
+fp8q_status fp8_quantize_mx_blocked(const void* x, int64_t rows, int64_t cols, fp8q_format f, uint8_t* codes,
+                                    uint8_t* scales, fp8q_stream_t stream) {
+  const int64_t n = checked_elems(rows, cols);
+  if (rows < 0 || cols < 0 || !valid_fmt(f) || cols % 32 != 0) return FP8Q_ERR_INVALID_ARGUMENT;
+  if (n < 0) return FP8Q_ERR_UNSUPPORTED;
+  if (n == 0) return FP8Q_OK;
+  if (!x || !codes || !scales || !aligned(x, 16) || !aligned(codes, 16)) return FP8Q_ERR_INVALID_ARGUMENT;
+  return from_cuda(fp8q::launch_quant_mx(static_cast<const uint16_t*>(x), rows, cols, f, codes, scales, 1,
                                          (cudaStream_t)stream));
 }
 
@@ -277,6 +293,20 @@ fp8q_status fp8_linear_dynamic(const void* X, int64_t M, int64_t N, int64_t K, c
                                             (cudaStream_t)stream);
   if (e == cudaErrorNotSupported) return FP8Q_ERR_UNSUPPORTED;
   return from_cuda(e);
+}
+
+fp8q_status fp8_gemm_mx(const uint8_t* A, const uint8_t* sA, fp8q_format fa, const uint8_t* B, const uint8_t* sB,
+                        fp8q_format fb, int64_t M, int64_t N, int64_t K, void* C, fp8q_stream_t stream) {
+  if (M < 0 || N < 0 || K < 0 || !valid_fmt(fa) || !valid_fmt(fb)) return FP8Q_ERR_INVALID_ARGUMENT;
+  if (M == 0 || N == 0) return FP8Q_OK;
+  if (N % 128 != 0 || K % 128 != 0 || K == 0) return FP8Q_ERR_UNSUPPORTED;
+  if (checked_elems(M, K) < 0 || checked_elems(N, K) < 0 || checked_elems(M, N) < 0) return FP8Q_ERR_UNSUPPORTED;
+  if (M > (int64_t(1) << 31) - 1 || N > (int64_t(1) << 31) - 1) return FP8Q_ERR_UNSUPPORTED;
+  if (!A || !B || !C || !sA || !sB || !aligned(A, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(sA, 16) ||
+      !aligned(sB, 16))
+    return FP8Q_ERR_INVALID_ARGUMENT;
+  return from_cuda(fp8q::launch_gemm_mx(A, sA, fa, B, sB, fb, M, N, K, static_cast<uint16_t*>(C),
+                                        (cudaStream_t)stream));
 }
 
 }  // extern "C"

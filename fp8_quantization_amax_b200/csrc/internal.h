@@ -79,9 +79,11 @@ cudaError_t launch_quant_delayed(const uint16_t* x0, const uint16_t* x1, uint8_t
                                  float* h0, float* h1, int64_t hlen, int64_t step, unsigned long long* counters,
                                  float* ws, cudaStream_t st);
 
-// MXFP8: 1x32 groups along rows (cols % 32 == 0), scales as byte exponents [rows][cols / 32]
+// MXFP8: 1x32 groups along rows (cols % 32 == 0), scales as byte exponents, row-major
+// [rows][cols / 32] (blocked = 0) or in the blocked layout of the block-scaled MMA (blocked = 1:
+// ceil(rows / 128) x ceil(cols / 128) chunks of 512 bytes)
 cudaError_t launch_quant_mx(const uint16_t* x, int64_t rows, int64_t cols, int fmt, uint8_t* codes, uint8_t* scales,
-                            cudaStream_t st);
+                            int blocked, cudaStream_t st);
 
 // y = bf16(decode(code) * s) under a granularity (0 tensor, 1 1x128, 2 128x128, 3 MX 1x32 with
 // byte exponents passed through `scales`)
@@ -93,6 +95,11 @@ cudaError_t launch_gemm(const uint8_t* A, const float* sA, int gA, const uint8_t
                         int64_t M, int64_t N, int64_t K, uint16_t* C, void* ws, size_t ws_bytes,
                         cudaStream_t st);
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+// MXFP8 GEMM on the block-scaled MMA: A [M][K], B [N][K] codes (formats fa, fb), scales in the
+// blocked layout; N % 128 == 0, K % 128 == 0
+cudaError_t launch_gemm_mx(const uint8_t* A, const uint8_t* sfa, int fa, const uint8_t* B, const uint8_t* sfb, int fb,
+                           int64_t M, int64_t N, int64_t K, uint16_t* C, cudaStream_t st);
 
 // C = GEMM(quantize_1x128_E4M3(X), B) for bf16 X [M][K]: the 1x128 quantizer into act_ws
 // (linear_act_workspace_bytes) and the block-scaled GEMM with gemm_ws

@@ -123,7 +123,8 @@ constexpr uint32_t kGroupStage = kGroupBoxRows * 128 * 2;
 struct GroupParams {
   uint8_t* codes;
   float* scales;
-  uint8_t* mx_scales;  // MX: [rows][cols / 32] power-of-two exponents (k + 127)
+  uint8_t* mx_scales;  // MX: power-of-two exponents (k + 127), row-major [rows][cols / 32] or blocked
+  int mx_blocked;      // MX: 1 = the blocked layout (one 512-byte chunk per 128 x 128 box)
   int64_t rows, cols;
   uint32_t nitems;
   FastDiv ngc;        // 128-column groups per row
@@ -229,13 +230,20 @@ __global__ void __launch_bounds__(kThreads, 2) k_group128(const __grid_constant_
         const float mul = e == 128 ? __uint_as_float(0x7FC00000u) : __uint_as_float((uint32_t)(127 - e) << 23);
         const int64_t row = (int64_t)rb * kGroupBoxRows + grp + h * 64;
         const int64_t col0 = (int64_t)g * 128 + q * 32;
+        if (p.mx_blocked) {
+          // the box's 128 rows x 4 groups are one 512-byte chunk: row r of the box at byte
+          // 16 (r % 32) + 4 (r / 32), group q beside it; rows and groups past the edge read zeros
+          // (the TMA fill), so they store byte 0
+          const int r = grp + h * 64;
+          p.mx_scales[((int64_t)rb * p.ngc.d + g) * 512 + (r & 31) * 16 + (r >> 5) * 4 + q] = (uint8_t)(e + 127);
+        }
         if (row >= p.rows || col0 >= p.cols) continue;
         uint8_t* dst = p.codes + row * p.cols + col0;
         const uint2 c0 = mx_quant8<FMT>(v[h][0], mul), c1 = mx_quant8<FMT>(v[h][1], mul),
                     c2 = mx_quant8<FMT>(v[h][2], mul), c3 = mx_quant8<FMT>(v[h][3], mul);
         st_stream_v4(dst, make_uint4(c0.x, c0.y, c1.x, c1.y));
         st_stream_v4(dst + 16, make_uint4(c2.x, c2.y, c3.x, c3.y));
-        p.mx_scales[row * ngroups + g * 4 + q] = (uint8_t)(e + 127);
+        if (!p.mx_blocked) p.mx_scales[row * ngroups + g * 4 + q] = (uint8_t)(e + 127);
       }
     }
     return;
@@ -290,7 +298,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_group128(const __grid_constant_
 
 template <int FMT, bool MX>
 static cudaError_t launch_group128_fmt(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* codes,
-                                       float* scales, uint8_t* mx_scales, cudaStream_t st) {
+                                       float* scales, uint8_t* mx_scales, int mx_blocked, cudaStream_t st) {
   const int64_t ngc = (cols + 127) / 128, nrb = (rows + kGroupBoxRows - 1) / kGroupBoxRows;
   const int64_t nitems = ngc * nrb;
   if (nitems == 0) return cudaSuccess;
@@ -302,6 +310,7 @@ static cudaError_t launch_group128_fmt(const uint16_t* x, int64_t rows, int64_t 
   p.codes = codes;
   p.scales = scales;
   p.mx_scales = mx_scales;
+  p.mx_blocked = mx_blocked;
   p.rows = rows;
   p.cols = cols;
   p.nitems = (uint32_t)nitems;
@@ -321,14 +330,14 @@ static cudaError_t launch_group128_fmt(const uint16_t* x, int64_t rows, int64_t 
 
 cudaError_t launch_quant_1x128(const uint16_t* x, int64_t rows, int64_t cols, int fmt, uint8_t* codes,
                                float* scales, cudaStream_t st) {
-  return fmt == kE4M3 ? launch_group128_fmt<kE4M3, false>(x, rows, cols, codes, scales, nullptr, st)
-                      : launch_group128_fmt<kE5M2, false>(x, rows, cols, codes, scales, nullptr, st);
+  return fmt == kE4M3 ? launch_group128_fmt<kE4M3, false>(x, rows, cols, codes, scales, nullptr, 0, st)
+                      : launch_group128_fmt<kE5M2, false>(x, rows, cols, codes, scales, nullptr, 0, st);
 }
 
 cudaError_t launch_quant_mx(const uint16_t* x, int64_t rows, int64_t cols, int fmt, uint8_t* codes, uint8_t* scales,
-                            cudaStream_t st) {
-  return fmt == kE4M3 ? launch_group128_fmt<kE4M3, true>(x, rows, cols, codes, nullptr, scales, st)
-                      : launch_group128_fmt<kE5M2, true>(x, rows, cols, codes, nullptr, scales, st);
+                            int blocked, cudaStream_t st) {
+  return fmt == kE4M3 ? launch_group128_fmt<kE4M3, true>(x, rows, cols, codes, nullptr, scales, blocked, st)
+                      : launch_group128_fmt<kE5M2, true>(x, rows, cols, codes, nullptr, scales, blocked, st);
 }
 
 // ============================================================================ 128-row tiles

@@ -212,11 +212,23 @@ FP8Q_API fp8q_status fp8_kv_quantize_noalloc(const void *k, const void *v, int64
  *   x       bf16 [rows][cols] (device, 16-byte aligned), cols % 32 == 0
  *   codes   uint8 [rows][cols] (device, written)
  *   scales  uint8 [rows][cols / 32] (device, written)
- * Only the format: no GEMM consumes these scales here (a native block-scaled tensor-core
- * product is not part of this library).
  */
 FP8Q_API fp8q_status fp8_quantize_mx(const void *x, int64_t rows, int64_t cols, fp8q_format f, uint8_t *codes,
                                      uint8_t *scales, fp8q_stream_t stream);
+
+/*
+ * The same quantization with the scales written in the BLOCKED layout that fp8_gemm_mx reads
+ * (the tensor cores' block-scaled MMA takes one 512-byte chunk per 128 rows x 128 columns):
+ *   chunk (rb, cb) = rows [128 rb, 128 rb + 128) x columns [128 cb, 128 cb + 128) starts at byte
+ *   512 * (rb * ceil(cols / 128) + cb); inside it the scale of row r and 32-column group j
+ *   (j = 0..3 within the chunk) sits at byte 16 * (r % 32) + 4 * ((r % 128) / 32) + j.
+ * Rows past `rows` and groups past cols / 32 in the last chunks are written as 0.
+ *   scales  uint8, fp8q_mx_blocked_scale_bytes(rows, cols) bytes (device, written)
+ * Other arguments and the codes as fp8_quantize_mx.
+ */
+FP8Q_API size_t fp8q_mx_blocked_scale_bytes(int64_t rows, int64_t cols);
+FP8Q_API fp8q_status fp8_quantize_mx_blocked(const void *x, int64_t rows, int64_t cols, fp8q_format f,
+                                             uint8_t *codes, uint8_t *scales, fp8q_stream_t stream);
 
 /* y = bf16_rne(fp32(decode(code) * 2^(scale - 127))), layouts as fp8_quantize_mx. */
 FP8Q_API fp8q_status fp8_dequantize_mx(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t cols,
@@ -315,6 +327,25 @@ FP8Q_API fp8q_status fp8_linear_dynamic(const void *X, int64_t M, int64_t N, int
                                         const float *sB, fp8q_granularity gB, void *C, void *act_ws,
                                         size_t act_ws_bytes, void *gemm_ws, size_t gemm_ws_bytes,
                                         fp8q_stream_t stream);
+
+/*
+ * MXFP8 GEMM on the tensor cores' native block-scaled MMA ([M] section on Microscaling: blocks
+ * of 32 with power-of-two scales, native on Blackwell; [W] "FP8 矩阵乘": FP8 products, fp32
+ * accumulation):
+ *   C[m][n] = bf16_rne( sum_k decode(A[m][k]) 2^(sA(m,k/32) - 127) * decode(B[n][k]) 2^(sB(n,k/32) - 127) )
+ * The tensor core applies the scales inside each MMA, so all of K accumulates in fp32 without
+ * a promotion step.
+ *   A    uint8 codes [M][K] in format fa (device, K-major), e.g. fp8_quantize_mx_blocked(X)
+ *   sA   blocked scales of A: fp8q_mx_blocked_scale_bytes(M, K) bytes (device)
+ *   B    uint8 codes [N][K] in format fb (W in R^{N x K}); sB: fp8q_mx_blocked_scale_bytes(N, K)
+ *   C    bf16 [M][N] (device, written)
+ * E4M3 and E5M2 mix freely (fa, fb).  A scale byte of 255 (NaN) gives NaN in the outputs it
+ * touches.  Requirements: M >= 1; N % 128 == 0; K % 128 == 0 (else FP8Q_ERR_UNSUPPORTED);
+ * A, B, C, sA, sB 16-byte aligned.  No workspace.
+ */
+FP8Q_API fp8q_status fp8_gemm_mx(const uint8_t *A, const uint8_t *sA, fp8q_format fa, const uint8_t *B,
+                                 const uint8_t *sB, fp8q_format fb, int64_t M, int64_t N, int64_t K, void *C,
+                                 fp8q_stream_t stream);
 
 #ifdef __cplusplus
 }

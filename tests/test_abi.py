@@ -134,3 +134,21 @@ def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(ValueError):
         fq.fp8_quantize(torch.zeros(4, 8, dtype=torch.bfloat16))
+
+
+def test_mx_blocked_and_gemm_mx_rejects(L):
+    a, m = ALIGNED, MISALIGNED
+    assert L.fp8q_mx_blocked_scale_bytes(130, 256) == 2 * 2 * 512
+    assert L.fp8q_mx_blocked_scale_bytes(128, 96) == 512
+    assert L.fp8q_mx_blocked_scale_bytes(-1, 32) == 0
+    assert L.fp8_quantize_mx_blocked(a, 4, 48, 0, a, a, None) == 1          # cols % 32
+    assert L.fp8_quantize_mx_blocked(a, 4, 64, 2, a, a, None) == 1          # bad format
+    assert L.fp8_quantize_mx_blocked(a, 4, 64, 0, a, None, None) == 1       # null scales
+    assert L.fp8_quantize_mx_blocked(None, 0, 64, 0, None, None, None) == 0  # empty
+    # (A, sA, fa, B, sB, fb, M, N, K, C, stream)
+    assert L.fp8_gemm_mx(a, a, 0, a, a, 2, 16, 256, 256, a, None) == 1      # bad format
+    assert L.fp8_gemm_mx(a, a, 0, a, a, 0, 16, 200, 256, a, None) == 2     # N % 128
+    assert L.fp8_gemm_mx(a, a, 0, a, a, 0, 16, 256, 96, a, None) == 2      # K % 128
+    assert L.fp8_gemm_mx(a, m, 0, a, a, 0, 16, 256, 256, a, None) == 1     # misaligned scales
+    assert L.fp8_gemm_mx(a, a, 0, a, None, 1, 16, 256, 256, a, None) == 1  # null scales
+    assert L.fp8_gemm_mx(None, None, 0, None, None, 0, 0, 256, 256, None, None) == 0
