@@ -363,7 +363,8 @@ def supplementary(device, stream, peaks, flush):
 
         def gemm_entry(m, n, k, ms, a, sa, wscale, c):
             flops = 2.0 * m * n * k
-            nbytes = a.numel() + n * k + c.numel() * 2 + sa.numel() * 4 + wscale.numel() * 4
+            nbytes = a.numel() + n * k + c.numel() * 2 + sa.numel() * sa.element_size() + \
+                wscale.numel() * wscale.element_size()
             return {"us": round(ms * 1e3, 2), "TFLOP/s": round(flops / ms / 1e9, 1),
                     "frac_fp8_peak": round(flops / ms / 1e9 / fp8_peak, 3),
                     "frac_fp8_peak_sustained": round(flops / ms / 1e9 / fp8_peak_sustained, 3),
@@ -377,7 +378,14 @@ def supplementary(device, stream, peaks, flush):
             fq.fp8_gemm_blockscaled(a, sa, wc, ws, out=cbuf)
             ms = timed(lambda: fq.fp8_gemm_blockscaled(a, sa, wc, ws, out=cbuf), 10, stream, flush)
             out["gemm_8b_up_m8192"] = gemm_entry(m, W_SHAPE[0], W_SHAPE[1], ms, a, sa, ws, cbuf)
-            del cbuf
+            # MXFP8 on the native block-scaled MMA, same shape: both operands quantized in 1x32
+            # groups with power-of-two scales (blocked layout)
+            am, sam = fq.fp8_quantize_mx_blocked(dev_bf16(synth.activations(seed=1), device))
+            bm, sbm = fq.fp8_quantize_mx_blocked(dev_bf16(synth.weight_8b(seed=1), device))
+            fq.fp8_gemm_mx(am, sam, bm, sbm, out=cbuf)
+            ms = timed(lambda: fq.fp8_gemm_mx(am, sam, bm, sbm, out=cbuf), 10, stream, flush)
+            out["gemm_mx_8b_up_m8192"] = gemm_entry(m, W_SHAPE[0], W_SHAPE[1], ms, am, sam, sbm, cbuf)
+            del cbuf, am, sam, bm, sbm
             # decode: back-to-back calls as in a decode step, each on one of four copies of the
             # weight codes (4 x 58.7 MB > L2), so every call streams its weights from HBM
             m = 16
@@ -418,6 +426,7 @@ def supplementary(device, stream, peaks, flush):
             # decode on the 70B up-projection (one weight, 235 MB > L2)
             w70 = dev_bf16(synth.weight_70b(seed=4, which="up"), device)
             b70, s70 = fq.fp8_quantize(w70, fq.E4M3, fq.BLOCK_128x128)
+            b70m, s70m = fq.fp8_quantize_mx_blocked(w70)
             del w70
             x70 = dev_bf16(synth.activations_70b(seed=4, m=64, which="up"), device)
             a70, sa70 = fq.fp8_quantize(x70, fq.E4M3, fq.GROUP_1x128)
@@ -442,6 +451,8 @@ def supplementary(device, stream, peaks, flush):
                     del w70
                 x70 = dev_bf16(synth.activations_70b(seed=4, m=16384, which=which), device)
                 a70, sa70 = fq.fp8_quantize(x70, fq.E4M3, fq.GROUP_1x128)
+                if which == "up":
+                    a70m, sa70m = fq.fp8_quantize_mx_blocked(x70)
                 del x70
                 c70 = torch.empty((16384, b70.shape[0]), dtype=torch.bfloat16, device=device)
                 fq.fp8_gemm_blockscaled(a70, sa70, b70, s70, out=c70)
@@ -454,6 +465,11 @@ def supplementary(device, stream, peaks, flush):
                                                                out=c70), 3, stream, flush)
                     out["gemm_70b_up_m16384_per_tensor"] = gemm_entry(16384, b70.shape[0], b70.shape[1], ms, a70, one,
                                                                       one, c70)
+                    fq.fp8_gemm_mx(a70m, sa70m, b70m, s70m, out=c70)
+                    ms = timed(lambda: fq.fp8_gemm_mx(a70m, sa70m, b70m, s70m, out=c70), 3, stream, flush)
+                    out["gemm_mx_70b_up_m16384"] = gemm_entry(16384, b70.shape[0], b70.shape[1], ms, a70m, sa70m,
+                                                              s70m, c70)
+                    del a70m, sa70m, b70m, s70m
                 del a70, sa70, c70
             del b70, s70
         except fq.Fp8qError as err:
@@ -679,7 +695,7 @@ def profile_target(name, reps):
     torch.cuda.set_device(device)
     stream = torch.cuda.Stream(device)
     with torch.cuda.stream(stream):
-        if name.startswith("gemm"):
+        if name.startswith("gemm") and not name.startswith("gemm_mx"):
             if name == "gemm_70b_up_m16384":
                 w = dev_bf16(synth.weight_70b(seed=4, which="up"), device)
                 x = dev_bf16(synth.activations_70b(seed=4, m=16384, which="up"), device)
@@ -692,6 +708,11 @@ def profile_target(name, reps):
             b, sb = fq.fp8_quantize(w, fq.E4M3, fq.BLOCK_128x128)
             c = torch.empty((a.shape[0], b.shape[0]), dtype=torch.bfloat16, device=device)
             fn = lambda: fq.fp8_gemm_blockscaled(a, sa, b, sb, out=c)  # noqa: E731
+        elif name == "gemm_mx_8b_m8192":
+            a, sa = fq.fp8_quantize_mx_blocked(dev_bf16(synth.activations(seed=1), device))
+            b, sb = fq.fp8_quantize_mx_blocked(dev_bf16(synth.weight_8b(seed=1), device))
+            c = torch.empty((a.shape[0], b.shape[0]), dtype=torch.bfloat16, device=device)
+            fn = lambda: fq.fp8_gemm_mx(a, sa, b, sb, out=c)  # noqa: E731
         elif name == "kv_delayed":
             k, v = synth.kv_70b(seed=3)
             kd, vd = dev_bf16(k, device), dev_bf16(v, device)
@@ -735,7 +756,7 @@ def main():
     ap.add_argument("--skip-extras", action="store_true",
                     help="time the steps only: no e2e, CPU baseline or supplementary kernels (for profiling)")
     ap.add_argument("--profile-target", default=None,
-                    choices=["gemm_8b_m8192", "gemm_8b_m16", "gemm_70b_up_m16384", "kv_tok128", "kv_head",
+                    choices=["gemm_8b_m8192", "gemm_8b_m16", "gemm_mx_8b_m8192", "gemm_70b_up_m16384", "kv_tok128", "kv_head",
                              "kv_delayed", "mx_8b", "dequant_8b"],
                     help="run one workload a few times and exit (a small target for ncu)")
     args = ap.parse_args()
