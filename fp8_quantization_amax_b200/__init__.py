@@ -23,7 +23,8 @@ __all__ = [
     "fp8_encode", "fp8_decode", "fp8_quantize", "fp8_dequantize", "fp8_kv_quantize",
     "fp8_kv_quantize_noalloc", "fp8_gemm_blockscaled", "fp8_quantize_delayed", "fp8_kv_quantize_delayed",
     "linear_act_workspace_bytes", "fp8_linear_dynamic", "fp8_quantize_mx", "fp8_dequantize_mx",
-    "mx_blocked_scale_bytes", "fp8_quantize_mx_blocked", "fp8_gemm_mx",
+    "mx_blocked_scale_bytes", "fp8_quantize_mx_blocked", "fp8_gemm_mx", "fp8_pack_b_tiles",
+    "fp8_gemm_blockscaled_packed",
 ]
 
 E4M3, E5M2 = 0, 1
@@ -76,6 +77,8 @@ def lib() -> ctypes.CDLL:
             L.fp8q_mx_blocked_scale_bytes.restype = sz
             L.fp8_quantize_mx_blocked.argtypes = [vp, i64, i64, i32, vp, vp, vp]
             L.fp8_gemm_mx.argtypes = [vp, vp, i32, vp, vp, i32, i64, i64, i64, vp, vp]
+            L.fp8_pack_b_tiles.argtypes = [vp, i64, i64, vp, vp]
+            L.fp8_gemm_blockscaled_packed.argtypes = [vp, vp, i32, vp, vp, i32, i64, i64, i64, vp, vp, sz, vp]
             L.fp8q_linear_act_workspace_bytes.argtypes = [i64, i64]
             L.fp8q_linear_act_workspace_bytes.restype = sz
             L.fp8_linear_dynamic.argtypes = [vp, i64, i64, i64, vp, vp, i32, vp, vp, sz, vp, sz, vp]
@@ -92,7 +95,8 @@ def lib() -> ctypes.CDLL:
             for fn in ("fp8_encode", "fp8_decode", "fp8_quantize", "fp8_dequantize", "fp8_kv_quantize",
                        "fp8_gemm_blockscaled", "fp8_kv_quantize_noalloc", "fp8_quantize_delayed",
                        "fp8_kv_quantize_delayed", "fp8_linear_dynamic", "fp8_quantize_mx", "fp8_dequantize_mx",
-                       "fp8_quantize_mx_blocked", "fp8_gemm_mx"):
+                       "fp8_quantize_mx_blocked", "fp8_gemm_mx", "fp8_pack_b_tiles",
+                       "fp8_gemm_blockscaled_packed"):
                 getattr(L, fn).restype = i32
             _lib = L
     return _lib
@@ -400,6 +404,44 @@ def fp8_gemm_blockscaled(a: torch.Tensor, sa: torch.Tensor, b: torch.Tensor, sb:
     if st != 0 and cached:
         _gemm_ws.clear()
     _check("fp8_gemm_blockscaled", st)
+    return out
+
+
+def fp8_pack_b_tiles(b: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """B codes [N][K] (N, K multiples of 128) -> packed tiles (uint8 [N * K]): one 16 KB block per
+    128 x 128 tile in the tensor cores' swizzled shared-memory image (see fp8_gemm_blockscaled_packed)."""
+    _dev(b, "b", torch.uint8)
+    N, K = b.shape
+    out = torch.empty(N * K, dtype=torch.uint8, device=b.device) if out is None else _dev(out, "out", torch.uint8)
+    if out.numel() < N * K:
+        raise ValueError(f"out needs {N * K} bytes")
+    _check("fp8_pack_b_tiles", lib().fp8_pack_b_tiles(_ptr(b), N, K, _ptr(out), _stream(b.device)))
+    return out
+
+
+def fp8_gemm_blockscaled_packed(a: torch.Tensor, sa: torch.Tensor, bp: torch.Tensor, sb: torch.Tensor, N: int,
+                                ga: int = GROUP_1x128, gb: int = BLOCK_128x128, out: torch.Tensor | None = None,
+                                ws: torch.Tensor | None = None) -> torch.Tensor:
+    """fp8_gemm_blockscaled with B as packed tiles (fp8_pack_b_tiles of the [N][K] codes): the same
+    result; each weight tile arrives with one bulk copy.  Workspace handling as fp8_gemm_blockscaled."""
+    _dev(a, "a", torch.uint8)
+    _dev(bp, "bp", torch.uint8)
+    _dev(sa, "sa", torch.float32)
+    _dev(sb, "sb", torch.float32)
+    M, K = a.shape
+    if bp.numel() < N * K:
+        raise ValueError("bp holds fewer than N * K bytes")
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device) if out is None else _dev(out, "out", torch.bfloat16)
+    need = gemm_workspace_bytes(M, N, K)
+    cached = ws is None
+    if cached:
+        ws = _gemm_workspace(need, a.device)
+    st = lib().fp8_gemm_blockscaled_packed(_ptr(a), _ptr(sa), ga, _ptr(bp), _ptr(sb), gb, M, N, K, _ptr(out),
+                                           _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+                                           _stream(a.device))
+    if st != 0 and cached:
+        _gemm_ws.clear()
+    _check("fp8_gemm_blockscaled_packed", st)
     return out
 
 

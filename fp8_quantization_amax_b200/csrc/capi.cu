@@ -267,8 +267,38 @@ fp8q_status fp8_gemm_blockscaled(const uint8_t* A, const float* sA, fp8q_granula
     return FP8Q_ERR_INVALID_ARGUMENT;
   const size_t need = fp8q::gemm_workspace_bytes(M, N, K);
   if (need > 0 && (!ws || ws_bytes < need || !aligned(ws, 16))) return FP8Q_ERR_WORKSPACE;
-  const cudaError_t e = fp8q::launch_gemm(A, sA, gA, B, sB, gB, M, N, K, static_cast<uint16_t*>(C), ws, ws_bytes,
-                                          (cudaStream_t)stream);
+  const cudaError_t e = fp8q::launch_gemm(A, sA, gA, B, false, sB, gB, M, N, K, static_cast<uint16_t*>(C), ws,
+                                          ws_bytes, (cudaStream_t)stream);
+  if (e == cudaErrorNotSupported) return FP8Q_ERR_UNSUPPORTED;
+  return from_cuda(e);
+}
+
+fp8q_status fp8_pack_b_tiles(const uint8_t* B, int64_t N, int64_t K, uint8_t* packed, fp8q_stream_t stream) {
+  if (N < 0 || K < 0) return FP8Q_ERR_INVALID_ARGUMENT;
+  if (N % 128 != 0 || K % 128 != 0) return FP8Q_ERR_UNSUPPORTED;
+  if (checked_elems(N, K) < 0) return FP8Q_ERR_UNSUPPORTED;
+  if (N == 0 || K == 0) return FP8Q_OK;
+  if (!B || !packed || !aligned(B, 16) || !aligned(packed, 16) || B == packed) return FP8Q_ERR_INVALID_ARGUMENT;
+  return from_cuda(fp8q::launch_pack_b_tiles(B, N, K, packed, (cudaStream_t)stream));
+}
+
+fp8q_status fp8_gemm_blockscaled_packed(const uint8_t* A, const float* sA, fp8q_granularity gA, const uint8_t* Bp,
+                                        const float* sB, fp8q_granularity gB, int64_t M, int64_t N, int64_t K,
+                                        void* C, void* ws, size_t ws_bytes, fp8q_stream_t stream) {
+  if (M < 0 || N < 0 || K < 0) return FP8Q_ERR_INVALID_ARGUMENT;
+  if (!(gA == FP8Q_GROUP_1x128 || gA == FP8Q_PER_TENSOR)) return FP8Q_ERR_INVALID_ARGUMENT;
+  if (!(gB == FP8Q_BLOCK_128x128 || gB == FP8Q_PER_TENSOR)) return FP8Q_ERR_INVALID_ARGUMENT;
+  if (M == 0 || N == 0) return FP8Q_OK;
+  if (N % 128 != 0 || K % 128 != 0 || K == 0) return FP8Q_ERR_UNSUPPORTED;
+  if (checked_elems(M, K) < 0 || checked_elems(N, K) < 0 || checked_elems(M, N) < 0) return FP8Q_ERR_UNSUPPORTED;
+  if (M > (int64_t(1) << 31) - 1 || N > (int64_t(1) << 31) - 1) return FP8Q_ERR_UNSUPPORTED;
+  if (!A || !Bp || !C || !sA || !sB || !aligned(A, 16) || !aligned(Bp, 16) || !aligned(C, 16) || !aligned(sA, 4) ||
+      !aligned(sB, 4))
+    return FP8Q_ERR_INVALID_ARGUMENT;
+  const size_t need = fp8q::gemm_workspace_bytes(M, N, K);
+  if (need > 0 && (!ws || ws_bytes < need || !aligned(ws, 16))) return FP8Q_ERR_WORKSPACE;
+  const cudaError_t e = fp8q::launch_gemm(A, sA, gA, Bp, true, sB, gB, M, N, K, static_cast<uint16_t*>(C), ws,
+                                          ws_bytes, (cudaStream_t)stream);
   if (e == cudaErrorNotSupported) return FP8Q_ERR_UNSUPPORTED;
   return from_cuda(e);
 }

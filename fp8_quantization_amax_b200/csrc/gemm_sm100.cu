@@ -75,6 +75,7 @@ struct Params {
   const float* sB;
   int gA_group;       // 1: sA is [K/128][M]; 0: one scale
   int gB_block;       // 1: sB is [N/128][K/128]; 0: one scale
+  const uint8_t* Bp;  // packed B tiles (16 KB each, tile (nb, kb) at nb * num_kb + kb), or null: B via TMA
   uint16_t* C;
   uint32_t* err;
 };
@@ -139,7 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ CU
     // ------------------------------------------------------------ TMA producer
     if (lane == 0 && my_tiles > 0) {
       tma_prefetch_desc(&tA);
-      tma_prefetch_desc(&tB);
+      if (!p.Bp) tma_prefetch_desc(&tB);
       int s = 0;
       uint32_t ph = 0;
       uint32_t it = 0;
@@ -147,14 +148,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ CU
       for (int k = 0; k < my_tiles && ok; ++k) {
         int m0, n0;
         tile_coords((int)blockIdx.x + k * (int)gridDim.x, p, &m0, &n0);
+        // packed B: one bulk copy per 128-row half inside N (a half past N is not loaded; its
+        // accumulator columns are never stored)
+        const int halves = p.Bp ? min(2, (p.N - n0) / 128) : 0;
+        const uint8_t* bp = p.Bp ? p.Bp + (size_t)(n0 / 128) * p.num_kb * 16384u : nullptr;
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
           if (it >= (uint32_t)kStages && !mbar_wait(&empty[s], ph ^ 1u, p.err)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[s], kStageBytes);
+          mbar_arrive_expect_tx(&full[s], p.Bp ? kStageA + 16384u * halves : kStageBytes);
           tma_load_2d(sm_a + s * kStageA, &tA, kb * BK, m0, &full[s]);
-          tma_load_2d(sm_b + s * kStageB, &tB, kb * BK, n0, &full[s]);
+          if (p.Bp) {
+            for (int h = 0; h < halves; ++h)
+              bulk_load(sm_b + s * kStageB + h * 16384u, bp + ((size_t)h * p.num_kb + kb) * 16384u, 16384u, &full[s]);
+          } else {
+            tma_load_2d(sm_b + s * kStageB, &tB, kb * BK, n0, &full[s]);
+          }
           if (++s == kStages) {
             s = 0;
             ph ^= 1u;
@@ -422,6 +432,7 @@ struct Params {
   uint16_t* C;
   int stages;
   uint32_t stage_bytes;
+  const uint8_t* Bp;  // packed weight tiles (tile t, K block kb at t * nkb + kb), or null: TMA
   uint32_t* err;
 };
 
@@ -463,11 +474,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
   if (warp == 0 && lane == 0 && n_units > 0) {
     // the weights are read once: start their first tiles towards L2 before waiting on the
     // previous grid (a prefetch only warms L2, which stays coherent with any later write)
-    tma_prefetch_desc(&tW);
+    if (!p.Bp) tma_prefetch_desc(&tW);
     tma_prefetch_desc(&tX);
     for (uint32_t i = 0; i < n_units && i < (uint32_t)S; ++i) {
       const uint32_t u = lo + i, t = u / nkb;
-      tma_prefetch_l2_2d(&tW, (int32_t)((u - t * nkb) * BK), (int32_t)(t * BM));
+      if (p.Bp)
+        bulk_prefetch_l2(p.Bp + (size_t)u * kStageW, kStageW);
+      else
+        tma_prefetch_l2_2d(&tW, (int32_t)((u - t * nkb) * BK), (int32_t)(t * BM));
     }
   }
   if (threadIdx.x == 0) {
@@ -509,7 +523,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
         if (i >= (uint32_t)S && !mbar_wait(&empty[s], ph ^ 1u, p.err)) break;
         uint8_t* st = smem + s * p.stage_bytes;
         mbar_arrive_expect_tx(&full[s], p.stage_bytes);
-        tma_load_2d(st, &tW, (int32_t)(kb * BK), (int32_t)(t * BM), &full[s]);
+        if (p.Bp)
+          bulk_load(st, p.Bp + (size_t)u * kStageW, kStageW, &full[s]);   // unit u = tile t, K block kb
+        else
+          tma_load_2d(st, &tW, (int32_t)(kb * BK), (int32_t)(t * BM), &full[s]);
         tma_load_2d(st + kStageW, &tX, (int32_t)(kb * BK), 0, &full[s]);
         if (++s == S) {
           s = 0;
@@ -759,15 +776,16 @@ cudaError_t launch_decode(const CUtensorMap& mW, const CUtensorMap& mX, gemm::de
 }
 
 cudaError_t launch_decode_gemm(const DecodePlan& plan, const uint8_t* A, const float* sA, int gA, const uint8_t* B,
-                               const float* sB, int gB, int64_t M, int64_t N, int64_t K, uint16_t* C, void* ws,
-                               size_t ws_bytes, cudaStream_t st) {
+                               bool b_packed, const float* sB, int gB, int64_t M, int64_t N, int64_t K, uint16_t* C,
+                               void* ws, size_t ws_bytes, cudaStream_t st) {
   using namespace gemm::dec;
   using gemm::BK;
   if (!ws || ws_bytes < plan.ws_bytes) return cudaErrorInvalidValue;
   CUtensorMap mW, mX;
   std::memset(&mW, 0, sizeof(mW));
   std::memset(&mX, 0, sizeof(mX));
-  if (!make_tmap_2d(&mW, 1, B, (uint64_t)K, (uint64_t)N, (uint64_t)K, BK, BM, 1)) return cudaErrorInvalidValue;
+  if (!b_packed && !make_tmap_2d(&mW, 1, B, (uint64_t)K, (uint64_t)N, (uint64_t)K, BK, BM, 1))
+    return cudaErrorInvalidValue;
   if (!make_tmap_2d(&mX, 1, A, (uint64_t)K, (uint64_t)M, (uint64_t)K, BK, (uint32_t)plan.mp, 1))
     return cudaErrorInvalidValue;
   gemm::dec::Params d;
@@ -787,6 +805,7 @@ cudaError_t launch_decode_gemm(const DecodePlan& plan, const uint8_t* A, const f
   d.C = C;
   d.stage_bytes = kStageW + (uint32_t)plan.mp * BK;
   d.stages = (int)std::max<uint32_t>(2, std::min<uint32_t>(kMaxStages, (200u * 1024u) / d.stage_bytes));
+  d.Bp = b_packed ? B : nullptr;
   d.err = device_error_word();
   switch (plan.mp) {
     case 16: return launch_decode<16>(mW, mX, d, st);
@@ -800,17 +819,19 @@ cudaError_t launch_decode_gemm(const DecodePlan& plan, const uint8_t* A, const f
 
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) { return decode_plan(M, N, K).ws_bytes; }
 
-cudaError_t launch_gemm(const uint8_t* A, const float* sA, int gA, const uint8_t* B, const float* sB, int gB,
-                        int64_t M, int64_t N, int64_t K, uint16_t* C, void* ws, size_t ws_bytes, cudaStream_t st) {
+cudaError_t launch_gemm(const uint8_t* A, const float* sA, int gA, const uint8_t* B, bool b_packed, const float* sB,
+                        int gB, int64_t M, int64_t N, int64_t K, uint16_t* C, void* ws, size_t ws_bytes,
+                        cudaStream_t st) {
   using namespace gemm;
   if (M == 0 || N == 0) return cudaSuccess;
   const DecodePlan plan = decode_plan(M, N, K);
-  if (plan.mp > 0) return launch_decode_gemm(plan, A, sA, gA, B, sB, gB, M, N, K, C, ws, ws_bytes, st);
+  if (plan.mp > 0) return launch_decode_gemm(plan, A, sA, gA, B, b_packed, sB, gB, M, N, K, C, ws, ws_bytes, st);
   CUtensorMap mA, mB;
   std::memset(&mA, 0, sizeof(mA));
   std::memset(&mB, 0, sizeof(mB));
   if (!make_tmap_2d(&mA, 1, A, (uint64_t)K, (uint64_t)M, (uint64_t)K, BK, BM, 1)) return cudaErrorInvalidValue;
-  if (!make_tmap_2d(&mB, 1, B, (uint64_t)K, (uint64_t)N, (uint64_t)K, BK, BN, 1)) return cudaErrorInvalidValue;
+  if (!b_packed && !make_tmap_2d(&mB, 1, B, (uint64_t)K, (uint64_t)N, (uint64_t)K, BK, BN, 1))
+    return cudaErrorInvalidValue;
   Params p;
   p.M = (int)M;
   p.N = (int)N;
@@ -823,6 +844,7 @@ cudaError_t launch_gemm(const uint8_t* A, const float* sA, int gA, const uint8_t
   p.sB = sB;
   p.gA_group = gA == 1;
   p.gB_block = gB == 2;
+  p.Bp = b_packed ? B : nullptr;
   p.C = C;
   p.err = device_error_word();
   const bool promote = p.gA_group || p.gB_block;
@@ -861,7 +883,7 @@ cudaError_t launch_linear(const uint16_t* X, const uint8_t* B, const float* sB, 
   float* scales = reinterpret_cast<float*>(codes + ((size_t)M * (size_t)K + 255) / 256 * 256);
   const cudaError_t e = launch_quant_1x128(X, M, K, 0, codes, scales, st);
   if (e != cudaSuccess) return e;
-  return launch_gemm(codes, scales, 1, B, sB, gB, M, N, K, C, gemm_ws, gemm_ws_bytes, st);
+  return launch_gemm(codes, scales, 1, B, false, sB, gB, M, N, K, C, gemm_ws, gemm_ws_bytes, st);
 }
 
 }  // namespace fp8q

@@ -91,9 +91,14 @@ cudaError_t launch_dequant(const uint8_t* codes, const float* scales, int64_t ro
                            int gran, uint16_t* y, cudaStream_t st);
 
 // block-scaled / per-tensor FP8 GEMM on tcgen05
-cudaError_t launch_gemm(const uint8_t* A, const float* sA, int gA, const uint8_t* B, const float* sB, int gB,
-                        int64_t M, int64_t N, int64_t K, uint16_t* C, void* ws, size_t ws_bytes,
+// (b_packed: B holds packed tiles, launch_pack_b_tiles, instead of row-major codes)
+cudaError_t launch_gemm(const uint8_t* A, const float* sA, int gA, const uint8_t* B, bool b_packed, const float* sB,
+                        int gB, int64_t M, int64_t N, int64_t K, uint16_t* C, void* ws, size_t ws_bytes,
                         cudaStream_t st);
+
+// B codes [N][K] (N, K multiples of 128) -> packed 16 KB tiles in the 128-byte-swizzled image of
+// a TMA load, tile (nb, kb) at 16384 (nb K/128 + kb)
+cudaError_t launch_pack_b_tiles(const uint8_t* B, int64_t N, int64_t K, uint8_t* packed, cudaStream_t st);
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 // MXFP8 GEMM on the block-scaled MMA: A [M][K], B [N][K] codes (formats fa, fb), scales in the

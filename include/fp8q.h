@@ -309,6 +309,31 @@ FP8Q_API fp8q_status fp8_gemm_blockscaled(const uint8_t *A, const float *sA, fp8
                                  void *ws, size_t ws_bytes, fp8q_stream_t stream);
 
 /*
+ * Packed weight tiles for the GEMMs.  Repacks B codes [N][K] (row-major, K-major rows) so
+ * that each 128 x 128 tile is one contiguous 16384-byte block: tile (nb, kb) = rows
+ * [128 nb, +128) x columns [128 kb, +128) starts at byte 16384 * (nb * K/128 + kb); inside it
+ * row r occupies bytes [128 r, 128 r + 128) with its eight 16-byte pieces in swizzled order
+ * (piece j at position j XOR (r % 8)).  This is the shared-memory image the tensor cores read,
+ * so the GEMMs fetch a tile with one bulk copy instead of 128 row requests (decode shapes
+ * stream the weights at the DRAM rate).  A one-time step per weight, like the quantization.
+ *   B       uint8 [N][K] codes (device, 16-byte aligned);  packed: N * K bytes (device, written,
+ *           16-byte aligned, not overlapping B)
+ * Requirements: N % 128 == 0, K % 128 == 0 (else FP8Q_ERR_UNSUPPORTED).
+ */
+FP8Q_API fp8q_status fp8_pack_b_tiles(const uint8_t *B, int64_t N, int64_t K, uint8_t *packed,
+                                      fp8q_stream_t stream);
+
+/*
+ * fp8_gemm_blockscaled with B given as packed tiles (fp8_pack_b_tiles): the same product, the
+ * same scales, workspace rules and requirements; the results are identical to
+ * fp8_gemm_blockscaled on the unpacked codes.
+ */
+FP8Q_API fp8q_status fp8_gemm_blockscaled_packed(const uint8_t *A, const float *sA, fp8q_granularity gA,
+                                                 const uint8_t *Bp, const float *sB, fp8q_granularity gB,
+                                                 int64_t M, int64_t N, int64_t K, void *C,
+                                                 void *ws, size_t ws_bytes, fp8q_stream_t stream);
+
+/*
  * Linear layer with dynamic activation quantization ([W] "激活动态量化": per-token 1x128
  * groups computed at run time, then "FP8 矩阵乘"):
  *   C = fp8_gemm_blockscaled(codes, scales, FP8Q_GROUP_1x128, B, sB, gB)  with

@@ -328,6 +328,21 @@ def gemm_mx_rows(a_codes, sa, b_codes, sb, rows, fmt_a: int = E4M3, fmt_b: int =
     return out
 
 
+def pack_b_tiles(codes: np.ndarray) -> np.ndarray:
+    """B codes [N][K] (N, K multiples of 128) -> the packed tile layout: tile (nb, kb) = rows
+    [128 nb, 128 nb + 128) x columns [128 kb, 128 kb + 128) is one 16384-byte block at
+    16384 * (nb * K/128 + kb); inside it row r takes bytes [128 r, 128 r + 128) with its eight
+    16-byte pieces in the order piece j at position j XOR (r % 8) (the 128-byte swizzle)."""
+    b = np.ascontiguousarray(codes, np.uint8)
+    N, K = b.shape
+    assert N % 128 == 0 and K % 128 == 0
+    n, k = np.indices((N, K))
+    off = ((n // 128) * (K // 128) + k // 128) * 16384 + (n % 128) * 128 + (((k % 128) // 16) ^ (n % 8)) * 16 + k % 16
+    out = np.empty(N * K, np.uint8)
+    out[off] = b
+    return out
+
+
 # ---------------------------------------------------------------- GEMM
 
 def gemm_rows(a_codes, sa, ga, b_codes, sb, gb, rows, fmt_a: int = E4M3, fmt_b: int = E4M3,

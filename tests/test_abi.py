@@ -67,6 +67,7 @@ def test_sizes(L):
 P = ctypes.c_void_p
 ALIGNED = P(1 << 20)          # never dereferenced: every call below fails validation first
 MISALIGNED = P((1 << 20) + 4)
+ALIGNED2 = P(1 << 24)
 
 
 @pytest.mark.parametrize("args,status", [
@@ -152,3 +153,17 @@ def test_mx_blocked_and_gemm_mx_rejects(L):
     assert L.fp8_gemm_mx(a, m, 0, a, a, 0, 16, 256, 256, a, None) == 1     # misaligned scales
     assert L.fp8_gemm_mx(a, a, 0, a, None, 1, 16, 256, 256, a, None) == 1  # null scales
     assert L.fp8_gemm_mx(None, None, 0, None, None, 0, 0, 256, 256, None, None) == 0
+
+
+def test_packed_b_rejects(L):
+    a, m = ALIGNED, MISALIGNED
+    assert L.fp8_pack_b_tiles(a, 256, 200, ALIGNED2, None) == 2       # K % 128
+    assert L.fp8_pack_b_tiles(a, 100, 256, ALIGNED2, None) == 2       # N % 128
+    assert L.fp8_pack_b_tiles(a, 256, 256, a, None) == 1              # in place
+    assert L.fp8_pack_b_tiles(a, 256, 256, m, None) == 1              # misaligned output
+    assert L.fp8_pack_b_tiles(None, 0, 256, None, None) == 0
+    # (A, sA, gA, Bp, sB, gB, M, N, K, C, ws, ws_bytes, stream)
+    assert L.fp8_gemm_blockscaled_packed(a, a, 2, a, a, 2, 16, 256, 256, a, a, 1 << 20, None) == 1   # gA
+    assert L.fp8_gemm_blockscaled_packed(a, a, 1, a, a, 2, 16, 200, 256, a, a, 1 << 20, None) == 2   # N
+    assert L.fp8_gemm_blockscaled_packed(a, a, 1, m, a, 2, 16, 256, 256, a, a, 1 << 20, None) == 1   # Bp
+    assert L.fp8_gemm_blockscaled_packed(a, a, 1, a, a, 2, 16, 256, 256, a, None, 0, None) == 3      # ws

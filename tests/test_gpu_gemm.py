@@ -213,3 +213,36 @@ def test_gemm_config4_per_tensor_variant(orc):
     rows = sample_rows(1024)
     ref = orc.gemm_rows(a, sa, 0, b, sb, 0, rows)
     check_tolerance(got[rows], ref, "config 4 per-tensor")
+
+
+# ---------------------------------------------------------------- packed weight tiles
+
+@pytest.mark.parametrize("shape", [(128, 128), (256, 384), (14336, 4096)])
+def test_pack_b_tiles_matches_oracle(orc, shape):
+    N, K = shape
+    b = np.random.default_rng(N + K).integers(0, 256, (N, K)).astype(np.uint8)
+    got = fq.fp8_pack_b_tiles(dev(b))
+    torch.cuda.synchronize()
+    assert np.array_equal(host(got), orc.pack_b_tiles(b))
+
+
+@pytest.mark.parametrize("ga,gb", [(1, 2), (0, 0)])
+@pytest.mark.parametrize("shape", [(1, 128, 128), (16, 256, 256), (64, 384, 512), (130, 384, 512), (300, 512, 384),
+                                   (16, 14336, 4096)])
+def test_packed_gemm_bit_identical(orc, ga, gb, shape):
+    """The packed path feeds the MMAs the same shared-memory bytes: identical bf16 output."""
+    M, N, K = shape
+    a, sa, b, sb = operands(orc, M, N, K, ga, gb, seed=M + N + K + 7)
+    want = run_gpu(a, sa, b, sb, ga, gb)
+    bp = fq.fp8_pack_b_tiles(dev(b))
+    got = fq.fp8_gemm_blockscaled_packed(dev(a), dev(sa), bp, dev(sb), N, ga, gb)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(got), want)
+
+
+def test_packed_gemm_against_oracle(orc):
+    M, N, K = 200, 384, 640
+    a, sa, b, sb = operands(orc, M, N, K, 1, 2, seed=41)
+    got = fq.fp8_gemm_blockscaled_packed(dev(a), dev(sa), dev(orc.pack_b_tiles(b)), dev(sb), N)
+    torch.cuda.synchronize()
+    check_tolerance(host(got), orc.gemm_rows(a, sa, 1, b, sb, 2, np.arange(M)), "packed")

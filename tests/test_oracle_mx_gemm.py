@@ -13,7 +13,9 @@ Pins, none of which retypes that sum:
     (catches a group index of k/128, k%32 or a transposed scale array);
   * raising every scale byte of one row (one column) by one doubles exactly that row (column);
   * a NaN scale byte (255) turns exactly its row into NaN;
-  * hand-worked byte positions of the blocked layout, and that it is a permutation.
+  * hand-worked byte positions of the blocked layout, and that it is a permutation;
+  * hand-worked byte positions of the packed B tile layout (the GEMM's bulk-copy weight format),
+    and that each packed row is its tile row with the 16-byte pieces XOR-permuted by row % 8.
 """
 import numpy as np
 import pytest
@@ -135,3 +137,32 @@ def test_blocked_layout_is_a_permutation(orc):
     np.testing.assert_array_equal(np.sort(b), np.sort(s.ravel()))
     # one chunk holds 128 rows x 4 groups: the first chunk is exactly rows 0..127, groups 0..3
     np.testing.assert_array_equal(np.sort(b[:512]), np.sort(s[:128, :4].ravel()))
+
+
+def test_packed_b_tiles_hand_worked(orc):
+    N, K = 256, 384                                          # 2 x 3 tiles
+    b = np.zeros((N, K), np.uint8)
+    marks = {(0, 0): 1, (0, 16): 2, (1, 0): 3, (1, 16): 4, (9, 5): 5, (0, 128): 6, (128, 0): 7, (135, 300): 8}
+    for (n, k), v in marks.items():
+        b[n, k] = v
+    p = orc.pack_b_tiles(b)
+    assert p.size == N * K
+    # tile (nb, kb) at 16384 (3 nb + kb); row r at 128 r; piece j of the row at 16 (j ^ (r % 8))
+    expect = {0: 1, 16: 2, 128 + 16: 3, 128 + 0: 4, 9 * 128 + 16 + 5: 5, 16384: 6, 3 * 16384: 7,
+              (3 + 2) * 16384 + 7 * 128 + 16 * ((300 - 256) // 16 ^ 7) + (300 % 16): 8}
+    for off, v in expect.items():
+        assert p[off] == v, off
+    assert np.count_nonzero(p) == len(marks)
+
+
+def test_packed_b_tiles_is_a_permutation_of_whole_tiles(orc):
+    rng = np.random.default_rng(31)
+    b = rng.integers(0, 256, (256, 256)).astype(np.uint8)
+    p = orc.pack_b_tiles(b)
+    for nb in range(2):
+        for kb in range(2):
+            blk = p[(nb * 2 + kb) * 16384:(nb * 2 + kb + 1) * 16384].reshape(128, 128)
+            tile = b[nb * 128:(nb + 1) * 128, kb * 128:(kb + 1) * 128]
+            for r in range(128):                             # each packed row is its tile row, pieces permuted
+                assert np.array_equal(np.sort(blk[r]), np.sort(tile[r]))
+                assert np.array_equal(blk[r].reshape(8, 16)[np.arange(8) ^ (r % 8)], tile[r].reshape(8, 16))
