@@ -78,6 +78,10 @@ def _load():
             lib.orc_dequantize_mx.restype = i32
             lib.orc_gemm_mx_rows.argtypes = [vp, vp, vp, vp, i32, i32, i64, i64, i64, vp, i64, vp]
             lib.orc_gemm_mx_rows.restype = i32
+            lib.orc_scale_histogram.argtypes = [vp, i64, i32, vp]
+            lib.orc_scale_histogram.restype = i32
+            lib.orc_count_underflow.argtypes = [vp, vp, i64, vp]
+            lib.orc_count_underflow.restype = i32
             _lib = lib
     return _lib
 
@@ -326,6 +330,28 @@ def gemm_mx_rows(a_codes, sa, b_codes, sb, rows, fmt_a: int = E4M3, fmt_b: int =
                                     _p(rows[i0:i0 + n]), n, _p(out[i0:i0 + n])) == 0
     _parallel(rows.size, run, threads, 4)
     return out
+
+
+def scale_histogram(scales: np.ndarray) -> np.ndarray:
+    """256-bucket histogram of scales by power of two: fp32 scales by their biased exponent
+    field, MX scale bytes (uint8) by value."""
+    s = np.ascontiguousarray(scales)
+    kind = 1 if s.dtype == np.uint8 else 0
+    if kind == 0:
+        s = np.ascontiguousarray(s, np.float32)
+    hist = np.zeros(256, np.uint32)
+    assert _load().orc_scale_histogram(_p(s), s.size, kind, _p(hist)) == 0
+    return hist
+
+
+def count_underflow(x_bf16: np.ndarray, codes: np.ndarray) -> int:
+    """Nonzero, non-NaN inputs whose code is +-0."""
+    x = np.ascontiguousarray(x_bf16, np.uint16)
+    c = np.ascontiguousarray(codes, np.uint8)
+    assert x.size == c.size
+    out = np.zeros(1, np.uint64)
+    assert _load().orc_count_underflow(_p(x), _p(c), x.size, _p(out)) == 0
+    return int(out[0])
 
 
 def pack_b_tiles(codes: np.ndarray) -> np.ndarray:

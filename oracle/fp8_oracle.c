@@ -576,3 +576,41 @@ int orc_gemm_mx_rows(const uint8_t *A, const uint8_t *sA, const uint8_t *B, cons
     FPENV_LEAVE;
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* scale health                                                              */
+/*
+ * [C] "scale 是控制面": the scales and the overflow / underflow they cause
+ * should be observable.  Two plain counts:
+ *   - a histogram of scales by power of two: kind 0 takes fp32 scales and
+ *     counts each in the bucket of its biased exponent field (bucket 0: zero
+ *     or subnormal, 255: Inf or NaN; so amax = s * FMAX falls in a known
+ *     octave); kind 1 takes MX scale bytes (the biased exponent itself);
+ *     hist[256] is added to;
+ *   - underflow to zero: nonzero, non-NaN inputs whose code is +-0 (added to
+ *     *count).
+ */
+int orc_scale_histogram(const void *scales, int64_t n, int kind, uint32_t *hist) {
+    if (kind != 0 && kind != 1) return -1;
+    for (int64_t i = 0; i < n; ++i) {
+        int b;
+        if (kind == 0) {
+            float s = ((const float *)scales)[i];
+            uint32_t bits;
+            memcpy(&bits, &s, 4);
+            b = (int)((bits >> 23) & 0xFF);
+        } else {
+            b = ((const uint8_t *)scales)[i];
+        }
+        hist[b] += 1;
+    }
+    return 0;
+}
+
+int orc_count_underflow(const uint16_t *x, const uint8_t *codes, int64_t n, uint64_t *count) {
+    for (int64_t i = 0; i < n; ++i) {
+        float xv = bf16_value(x[i]);
+        if (!isnan(xv) && xv != 0.0f && (codes[i] & 0x7F) == 0) *count += 1;
+    }
+    return 0;
+}

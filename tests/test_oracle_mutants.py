@@ -16,6 +16,7 @@ import test_oracle_codec as tc
 import test_oracle_delayed as td
 import test_oracle_mx as tmx
 import test_oracle_mx_gemm as tmg
+import test_oracle_health as th
 import test_oracle_gemm as tg
 import test_oracle_quantize as tq
 
@@ -59,6 +60,10 @@ MUTANTS = {
     "mx_gemm_b_format_of_a": ("b[k] = (double)orc_decode(fmtB, B[n * K + k]) * mx_scale_value",
                               "b[k] = (double)orc_decode(fmtA, B[n * K + k]) * mx_scale_value"),
     "mx_gemm_nan_scale_ignored": ("return b == 255 ? NAN : ldexp", "return b == 255 ? 1.0 : ldexp"),
+    "hist_bucket_shift": ("b = (int)((bits >> 23) & 0xFF);", "b = (int)((bits >> 24) & 0xFF);"),
+    "hist_sign_in_bucket": ("b = (int)((bits >> 23) & 0xFF);", "b = (int)(((bits >> 23) + (bits >> 31)) & 0xFF);"),
+    "underflow_counts_zero_inputs": ("if (!isnan(xv) && xv != 0.0f && (codes[i] & 0x7F) == 0) *count += 1;",
+                                     "if (!isnan(xv) && (codes[i] & 0x7F) == 0) *count += 1;"),
     "mx_dequant_drops_scale": ("y[r * cols + c] = bf16_round(orc_decode(fmt, codes[r * cols + c]) * s);",
                                "y[r * cols + c] = bf16_round(orc_decode(fmt, codes[r * cols + c]));"),
 }
@@ -91,6 +96,9 @@ def _pins(m):
         lambda: tmx.test_exponent_at_powers_of_two_of_fmax(m, 0),
         lambda: tmx.test_bruteforce_tiny(m, 0, (3, 96)),
         lambda: tmx.test_dequantize_matches_torch(m, 0),
+        lambda: th.test_histogram_hand_worked(m),
+        lambda: th.test_histogram_matches_frexp(m),
+        lambda: th.test_underflow_hand_worked(m),
         lambda: tmg.test_uniform_scales_reduce_to_matmul(m, 0, 1),
         lambda: tmg.test_one_group_special_case(m),
         lambda: tmg.test_row_and_column_doubling(m),
