@@ -24,7 +24,7 @@ __all__ = [
     "fp8_kv_quantize_noalloc", "fp8_gemm_blockscaled", "fp8_quantize_delayed", "fp8_kv_quantize_delayed",
     "linear_act_workspace_bytes", "fp8_linear_dynamic", "fp8_quantize_mx", "fp8_dequantize_mx",
     "mx_blocked_scale_bytes", "fp8_quantize_mx_blocked", "fp8_gemm_mx", "fp8_pack_b_tiles",
-    "fp8_gemm_blockscaled_packed",
+    "fp8_gemm_blockscaled_packed", "fp8_scale_histogram", "fp8_count_underflow",
 ]
 
 E4M3, E5M2 = 0, 1
@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
             L.fp8_quantize_mx_blocked.argtypes = [vp, i64, i64, i32, vp, vp, vp]
             L.fp8_gemm_mx.argtypes = [vp, vp, i32, vp, vp, i32, i64, i64, i64, vp, vp]
             L.fp8_pack_b_tiles.argtypes = [vp, i64, i64, vp, vp]
+            L.fp8_scale_histogram.argtypes = [vp, i64, i32, vp, vp]
+            L.fp8_count_underflow.argtypes = [vp, vp, i64, vp, vp]
             L.fp8_gemm_blockscaled_packed.argtypes = [vp, vp, i32, vp, vp, i32, i64, i64, i64, vp, vp, sz, vp]
             L.fp8q_linear_act_workspace_bytes.argtypes = [i64, i64]
             L.fp8q_linear_act_workspace_bytes.restype = sz
@@ -96,7 +98,7 @@ def lib() -> ctypes.CDLL:
                        "fp8_gemm_blockscaled", "fp8_kv_quantize_noalloc", "fp8_quantize_delayed",
                        "fp8_kv_quantize_delayed", "fp8_linear_dynamic", "fp8_quantize_mx", "fp8_dequantize_mx",
                        "fp8_quantize_mx_blocked", "fp8_gemm_mx", "fp8_pack_b_tiles",
-                       "fp8_gemm_blockscaled_packed"):
+                       "fp8_gemm_blockscaled_packed", "fp8_scale_histogram", "fp8_count_underflow"):
                 getattr(L, fn).restype = i32
             _lib = L
     return _lib
@@ -443,6 +445,33 @@ def fp8_gemm_blockscaled_packed(a: torch.Tensor, sa: torch.Tensor, bp: torch.Ten
         _gemm_ws.clear()
     _check("fp8_gemm_blockscaled_packed", st)
     return out
+
+
+def fp8_scale_histogram(scales: torch.Tensor, hist: torch.Tensor | None = None) -> torch.Tensor:
+    """Add a 256-bucket histogram of the scales by power of two to `hist` (int32 [256] on the
+    device, created zeroed when not given): fp32 scales by their biased exponent field, MX scale
+    bytes (uint8) by value."""
+    if scales.dtype not in (torch.float32, torch.uint8):
+        raise TypeError("scales must be float32 (fp32 scales) or uint8 (MX bytes)")
+    _dev(scales, "scales", scales.dtype)
+    hist = torch.zeros(256, dtype=torch.int32, device=scales.device) if hist is None else _dev(hist, "hist", torch.int32)
+    kind = 0 if scales.dtype == torch.float32 else 1
+    _check("fp8_scale_histogram", lib().fp8_scale_histogram(_ptr(scales), scales.numel(), kind, _ptr(hist),
+                                                           _stream(scales.device)))
+    return hist
+
+
+def fp8_count_underflow(x: torch.Tensor, codes: torch.Tensor, count: torch.Tensor | None = None) -> torch.Tensor:
+    """Add to `count` (int64 [1] on the device, created zeroed when not given) the number of
+    nonzero, non-NaN bf16 inputs whose FP8 code is +-0."""
+    _dev(x, "x", torch.bfloat16)
+    _dev(codes, "codes", torch.uint8)
+    if x.numel() != codes.numel():
+        raise ValueError("x and codes differ in size")
+    count = torch.zeros(1, dtype=torch.int64, device=x.device) if count is None else _dev(count, "count", torch.int64)
+    _check("fp8_count_underflow", lib().fp8_count_underflow(_ptr(x), _ptr(codes), x.numel(), _ptr(count),
+                                                           _stream(x.device)))
+    return count
 
 
 def linear_act_workspace_bytes(M: int, K: int) -> int:

@@ -273,6 +273,27 @@ fp8q_status fp8_gemm_blockscaled(const uint8_t* A, const float* sA, fp8q_granula
   return from_cuda(e);
 }
 
+fp8q_status fp8_scale_histogram(const void* scales, int64_t n, fp8q_scale_kind kind, uint32_t* hist,
+                                fp8q_stream_t stream) {
+  if (n < 0 || !(kind == FP8Q_SCALES_F32 || kind == FP8Q_SCALES_MX)) return FP8Q_ERR_INVALID_ARGUMENT;
+  if (n > kMaxElems) return FP8Q_ERR_UNSUPPORTED;
+  if (n == 0) return FP8Q_OK;
+  if (!scales || !hist || !aligned(hist, 4) || (kind == FP8Q_SCALES_F32 && !aligned(scales, 4)))
+    return FP8Q_ERR_INVALID_ARGUMENT;
+  return from_cuda(fp8q::launch_scale_histogram(scales, n, kind, hist, (cudaStream_t)stream));
+}
+
+fp8q_status fp8_count_underflow(const void* x, const uint8_t* codes, int64_t n, unsigned long long* count,
+                                fp8q_stream_t stream) {
+  if (n < 0) return FP8Q_ERR_INVALID_ARGUMENT;
+  if (n > kMaxElems) return FP8Q_ERR_UNSUPPORTED;
+  if (n == 0) return FP8Q_OK;
+  if (!x || !codes || !count || !aligned(x, 16) || !aligned(codes, 16) || !aligned(count, 8))
+    return FP8Q_ERR_INVALID_ARGUMENT;
+  return from_cuda(fp8q::launch_count_underflow(static_cast<const uint16_t*>(x), codes, n, count,
+                                                (cudaStream_t)stream));
+}
+
 fp8q_status fp8_pack_b_tiles(const uint8_t* B, int64_t N, int64_t K, uint8_t* packed, fp8q_stream_t stream) {
   if (N < 0 || K < 0) return FP8Q_ERR_INVALID_ARGUMENT;
   if (N % 128 != 0 || K % 128 != 0) return FP8Q_ERR_UNSUPPORTED;

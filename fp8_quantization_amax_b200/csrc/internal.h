@@ -96,6 +96,13 @@ cudaError_t launch_gemm(const uint8_t* A, const float* sA, int gA, const uint8_t
                         int gB, int64_t M, int64_t N, int64_t K, uint16_t* C, void* ws, size_t ws_bytes,
                         cudaStream_t st);
 
+// scale health: a 256-bucket histogram of scales by power of two (kind 0: fp32 scales by their
+// exponent field; 1: MX bytes), added to hist; and the count of nonzero non-NaN inputs whose
+// code is +-0, added to *count
+cudaError_t launch_scale_histogram(const void* scales, int64_t n, int kind, uint32_t* hist, cudaStream_t st);
+cudaError_t launch_count_underflow(const uint16_t* x, const uint8_t* codes, int64_t n, unsigned long long* count,
+                                   cudaStream_t st);
+
 // B codes [N][K] (N, K multiples of 128) -> packed 16 KB tiles in the 128-byte-swizzled image of
 // a TMA load, tile (nb, kb) at 16384 (nb K/128 + kb)
 cudaError_t launch_pack_b_tiles(const uint8_t* B, int64_t N, int64_t K, uint8_t* packed, cudaStream_t st);

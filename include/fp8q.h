@@ -308,6 +308,30 @@ FP8Q_API fp8q_status fp8_gemm_blockscaled(const uint8_t *A, const float *sA, fp8
                                  int64_t M, int64_t N, int64_t K, void *C,
                                  void *ws, size_t ws_bytes, fp8q_stream_t stream);
 
+/* ---------------------------------------------------------------- scale health */
+
+/*
+ * Observability of the scales and of the values they lose ([C] "scale 是控制面": scales,
+ * overflow and underflow should be observable; saturation counts come with the delayed-scaling
+ * calls, the only path where a value can exceed the scale's range).
+ *
+ * fp8_scale_histogram adds to hist[256] (uint32, device) a histogram of n scales by power of
+ * two: FP8Q_SCALES_F32 takes fp32 scales (4-byte aligned) and counts each in the bucket of its
+ * biased exponent field (bucket e holds scales in [2^(e-127), 2^(e-126)); 0: zero or subnormal;
+ * 255: Inf or NaN), so amax = s * FMAX lies in a known octave; FP8Q_SCALES_MX takes MX scale
+ * bytes and counts each by value (the biased exponent itself).  Any layout works: scales are
+ * counted, not located.
+ *
+ * fp8_count_underflow adds to *count (uint64, device, 8-byte aligned) the number of elements of
+ * x (bf16 [n], 16-byte aligned) that are nonzero and not NaN while their code (uint8 [n],
+ * 16-byte aligned, any format) is +-0: values the quantization flushed to zero.
+ */
+typedef enum { FP8Q_SCALES_F32 = 0, FP8Q_SCALES_MX = 1 } fp8q_scale_kind;
+FP8Q_API fp8q_status fp8_scale_histogram(const void *scales, int64_t n, fp8q_scale_kind kind, uint32_t *hist,
+                                         fp8q_stream_t stream);
+FP8Q_API fp8q_status fp8_count_underflow(const void *x, const uint8_t *codes, int64_t n,
+                                         unsigned long long *count, fp8q_stream_t stream);
+
 /*
  * Packed weight tiles for the GEMMs.  Repacks B codes [N][K] (row-major, K-major rows) so
  * that each 128 x 128 tile is one contiguous 16384-byte block: tile (nb, kb) = rows

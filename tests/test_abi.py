@@ -65,6 +65,12 @@ def test_sizes(L):
 
 
 P = ctypes.c_void_p
+# The rejection tests pass dummy device pointers that every call must refuse before launching
+# anything; they run only where no GPU is visible, so a validation slip can never launch a kernel
+# on those addresses.
+host_only = pytest.mark.skipif(__import__("torch").cuda.is_available(),
+                               reason="dummy device pointers: run on a host without a GPU")
+
 ALIGNED = P(1 << 20)          # never dereferenced: every call below fails validation first
 MISALIGNED = P((1 << 20) + 4)
 ALIGNED2 = P(1 << 24)
@@ -84,10 +90,12 @@ ALIGNED2 = P(1 << 24)
     ((ALIGNED, 1 << 40, 1 << 8, 0, 1, ALIGNED, ALIGNED, None, 0, None), 2),  # too large
     ((None, 0, 8, 0, 1, None, None, None, 0, None), 0),                  # empty: nothing to do
 ])
+@host_only
 def test_quantize_rejects(L, args, status):
     assert L.fp8_quantize(*args) == status
 
 
+@host_only
 def test_delayed_rejects(L):
     a, m = ALIGNED, MISALIGNED
     # (x, rows, cols, fmt, history, history_len, step, codes, scale, counts, ws, ws_bytes, stream)
@@ -104,6 +112,7 @@ def test_delayed_rejects(L):
     assert L.fp8_kv_quantize_delayed(a, a, 16, 0, 128, 0, 1, a, a, 4, 1, a, a, a, a, None, None, 0, None) == 0
 
 
+@host_only
 def test_dequantize_rejects(L):
     assert L.fp8_dequantize(ALIGNED, ALIGNED, 4, 12, 0, 1, ALIGNED, None) == 1
     assert L.fp8_dequantize(ALIGNED, None, 4, 8, 0, 1, ALIGNED, None) == 1
@@ -111,6 +120,7 @@ def test_dequantize_rejects(L):
     assert L.fp8_dequantize(None, None, 0, 8, 0, 1, None, None) == 0
 
 
+@host_only
 def test_kv_rejects(L):
     k = ALIGNED
     assert L.fp8_kv_quantize(k, k, 16, 8, 12, 0, 1, k, k, k, k, k, 1 << 20, None) == 1        # head_dim % 8
@@ -120,6 +130,7 @@ def test_kv_rejects(L):
     assert L.fp8_kv_quantize(k, None, 16, 8, 128, 0, 2, k, k, k, k, None, 0, None) == 1       # null v
 
 
+@host_only
 def test_gemm_rejects(L):
     a = ALIGNED
     assert L.fp8_gemm_blockscaled(a, a, 1, a, a, 2, 128, 100, 128, a, None, 0, None) == 2      # N % 128
@@ -137,6 +148,7 @@ def test_binding_refuses_cpu_tensors():
         fq.fp8_quantize(torch.zeros(4, 8, dtype=torch.bfloat16))
 
 
+@host_only
 def test_mx_blocked_and_gemm_mx_rejects(L):
     a, m = ALIGNED, MISALIGNED
     assert L.fp8q_mx_blocked_scale_bytes(130, 256) == 2 * 2 * 512
@@ -155,6 +167,7 @@ def test_mx_blocked_and_gemm_mx_rejects(L):
     assert L.fp8_gemm_mx(None, None, 0, None, None, 0, 0, 256, 256, None, None) == 0
 
 
+@host_only
 def test_packed_b_rejects(L):
     a, m = ALIGNED, MISALIGNED
     assert L.fp8_pack_b_tiles(a, 256, 200, ALIGNED2, None) == 2       # K % 128
@@ -167,3 +180,14 @@ def test_packed_b_rejects(L):
     assert L.fp8_gemm_blockscaled_packed(a, a, 1, a, a, 2, 16, 200, 256, a, a, 1 << 20, None) == 2   # N
     assert L.fp8_gemm_blockscaled_packed(a, a, 1, m, a, 2, 16, 256, 256, a, a, 1 << 20, None) == 1   # Bp
     assert L.fp8_gemm_blockscaled_packed(a, a, 1, a, a, 2, 16, 256, 256, a, None, 0, None) == 3      # ws
+
+
+@host_only
+def test_health_rejects(L):
+    a, m = ALIGNED, MISALIGNED
+    assert L.fp8_scale_histogram(a, 10, 2, a, None) == 1                # bad kind
+    assert L.fp8_scale_histogram(P((1 << 20) + 2), 10, 0, a, None) == 1  # fp32 scales not 4-byte aligned
+    assert L.fp8_scale_histogram(None, 0, 0, None, None) == 0           # empty
+    assert L.fp8_count_underflow(a, m, 64, a, None) == 1                # misaligned codes
+    assert L.fp8_count_underflow(a, a, -1, a, None) == 1
+    assert L.fp8_count_underflow(None, None, 0, None, None) == 0
