@@ -18,13 +18,15 @@
 //   warp 0      producer: per K block of 128, the A box 128 x 128 and the B box 256 x 128
 //               (128-byte swizzle, TMA) and the scale chunks of A (512 B) and of B's two
 //               128-row halves (bulk copies) into a 4-stage shared-memory ring.
-//   warp 1      allocates 512 TMEM columns (accumulator 0..255, A scales 256..259, B scales
-//               260..267); lane 0 copies each stage's scale chunks into TMEM (tcgen05.cp) and
+//   warp 1      allocates 512 TMEM columns: two 256-column accumulators that overlap by one
+//               32-column chunk (columns 0..255 and 224..479), A scales 480..483, B scales
+//               484..491; lane 0 copies each stage's scale chunks into TMEM (tcgen05.cp) and
 //               issues four block-scaled MMAs (M128 N256 K32).  tcgen05 operations of one thread
 //               run in issue order, so one set of scale columns serves every K block.
 //   warps 2-3   idle (they complete warpgroup 0, which hands its registers to the epilogue).
-//   warps 4-11  epilogue: TMEM -> registers -> bf16, release the accumulator, then store (the
-//               next tile's MMAs run while the stores drain).
+//   warps 4-11  epilogue: TMEM -> registers -> bf16, release the accumulator, then store.  The
+//               warps holding the shared chunk read it first and release it at once, so the
+//               next tile's MMAs (into the other accumulator) wait only for that one load.
 // Every mbarrier wait is bounded (sm100.cuh): on a timeout the kernel records an error in the
 // device error word and winds down instead of hanging.
 #include <cuda.h>
@@ -55,8 +57,9 @@ constexpr int kEpiWarps = 8;
 constexpr int kFirstEpiWarp = 4;
 constexpr int kThreads = 128 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSfaCol = 256;                     // 4 columns: rows 32c .. 32c + 31 in column c
-constexpr uint32_t kSfbCol = 260;                     // 8 columns for the tile's 256 B rows
+constexpr uint32_t kBuf1Col = 224;                    // second accumulator: shares columns 224..255
+constexpr uint32_t kSfaCol = 480;                     // 4 columns: rows 32c .. 32c + 31 in column c
+constexpr uint32_t kSfbCol = 484;                     // 8 columns for the tile's 256 B rows
 
 // the same register split as the block-scaled GEMM (the build checks the launch count)
 constexpr int kLaunchRegs = 168;
@@ -108,6 +111,17 @@ __device__ __forceinline__ void umma_mx(uint32_t tmem_d, uint64_t adesc, uint64_
       : "memory");
 }
 
+// one 32-column chunk of this thread's accumulator row -> 16 packed bf16 pairs
+template <int C>
+__device__ __forceinline__ void epi_chunk(uint32_t taddr, uint32_t (&out)[64]) {
+  uint32_t v[32];
+  tmem_ld32(taddr + C * 32, v);
+  tmem_ld_wait();
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+    out[C * 16 + i] = f32x2_to_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+}
+
 __global__ void __launch_bounds__(kThreads, 1) k_gemm_mx(const __grid_constant__ CUtensorMap tA,
                                                          const __grid_constant__ CUtensorMap tB, Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -117,9 +131,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_mx(const __grid_constant__
   uint8_t* sm_sf = smem + kStages * (kStageA + kStageB);     // kStages x 1.5 KB (A, B half 0, B half 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(sm_sf + kStages * kStageSf);
   uint64_t* empty = full + kStages;
-  uint64_t* tfull = empty + kStages;
-  uint64_t* tempty = tfull + 1;
-  uint64_t* drain = tempty + 1;
+  uint64_t* tfull = empty + kStages;                         // [2] per accumulator
+  uint64_t* tempty = tfull + 2;                              // [2]
+  uint64_t* ofree = tempty + 2;                              // shared chunk read, once per tile
+  uint64_t* drain = ofree + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -128,8 +143,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_mx(const __grid_constant__
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(tfull, 1);
-    mbar_init(tempty, kEpiWarps);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], kEpiWarps);
+    }
+    mbar_init(ofree, kEpiWarps / 2);
     mbar_init(drain, 1);
     fence_mbar_init();
   }
@@ -196,14 +214,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_mx(const __grid_constant__
         bool ok = true;
         const uint32_t tsfa = tmem_base + kSfaCol, tsfb = tmem_base + kSfbCol;
         for (int k = 0; k < my_tiles && ok; ++k) {
-          if (k > 0) {
-            // the epilogue has read the previous tile out of the accumulator
-            if (!mbar_wait(tempty, (uint32_t)(k - 1) & 1u, p.err)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
+          const uint32_t buf = (uint32_t)k & 1u;
+          // this accumulator's previous tile has been read out, and the previous tile (in the
+          // other accumulator) has released the shared chunk
+          if (k >= 2 && !mbar_wait(&tempty[buf], ((uint32_t)(k >> 1) - 1u) & 1u, p.err)) {
+            ok = false;
+            break;
           }
+          if (k >= 1 && !mbar_wait(ofree, (uint32_t)(k - 1) & 1u, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t tmem_d = tmem_base + (buf ? kBuf1Col : 0u);
           for (int kb = 0; kb < p.num_kb; ++kb) {
             if (!mbar_wait(&full[s], ph, p.err)) {
               ok = false;
@@ -221,12 +244,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_mx(const __grid_constant__
               // scale byte kk of each TMEM word: the address' top two bits and the descriptor's
               // selectors name it
               const uint32_t sel = (uint32_t)kk;
-              umma_mx(tmem_base, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2),
+              umma_mx(tmem_d, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2),
                       p.idesc | (sel << 4) | (sel << 29), tsfa | (sel << 30), tsfb | (sel << 30),
                       (kb > 0 || kk > 0) ? 1u : 0u);
             }
             umma_commit(&empty[s]);                       // frees the stage (codes and scales)
-            if (kb == p.num_kb - 1) umma_commit(tfull);   // tile accumulated
+            if (kb == p.num_kb - 1) umma_commit(&tfull[buf]);   // tile accumulated
             if (++s == kStages) {
               s = 0;
               ph ^= 1u;
@@ -245,26 +268,42 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_mx(const __grid_constant__
     const int quarter = warp & 3;            // TMEM lane quarter this warp may access
     const int half = ew >> 2;                // 128-column half of the tile
     const int row_in_tile = quarter * 32 + lane;
-    const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + half * 128;
+    const uint32_t lane_base = tmem_base + ((uint32_t)(quarter * 32) << 16) + half * 128;
     for (int k = 0; k < my_tiles; ++k) {
       const int t = (int)blockIdx.x + k * (int)gridDim.x;
       const int m = (t % p.m_tiles) * BM + row_in_tile;
       const int ncol0 = (t / p.m_tiles) * BN + half * 128;
-      if (!mbar_wait(tfull, (uint32_t)k & 1u, p.err)) break;
+      const uint32_t buf = (uint32_t)k & 1u;
+      if (!mbar_wait(&tfull[buf], (uint32_t)(k >> 1) & 1u, p.err)) break;
       tc_fence_after();
+      const uint32_t taddr = lane_base + (buf ? kBuf1Col : 0u);
       uint32_t out[64];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(taddr + c * 32, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          out[c * 16 + i] = f32x2_to_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+      // the shared chunk is accumulator 0's last (tile columns 224..255, held by half 1) and
+      // accumulator 1's first (tile columns 0..31, half 0): its holders read it first
+      const bool first_last = buf == 0 && half == 1;
+      const bool holds_shared = first_last || (buf == 1 && half == 0);
+      if (first_last) {
+        epi_chunk<3>(taddr, out);
+      } else {
+        epi_chunk<0>(taddr, out);
+      }
+      if (holds_shared) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ofree);
+      }
+      if (first_last) {
+        epi_chunk<0>(taddr, out);
+        epi_chunk<1>(taddr, out);
+        epi_chunk<2>(taddr, out);
+      } else {
+        epi_chunk<1>(taddr, out);
+        epi_chunk<2>(taddr, out);
+        epi_chunk<3>(taddr, out);
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(tempty);
+      if (lane == 0) mbar_arrive(&tempty[buf]);
       if (m < p.M && ncol0 < p.N) {
         uint16_t* dst = p.C + (size_t)m * p.N + ncol0;
 #pragma unroll
@@ -283,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_mx(const __grid_constant__
   }
 }
 
-constexpr size_t kSmemBytes = 1024 + kStages * (kStageA + kStageB + kStageSf) + (2 * kStages + 3) * sizeof(uint64_t) + 16;
+constexpr size_t kSmemBytes = 1024 + kStages * (kStageA + kStageB + kStageSf) + (2 * kStages + 6) * sizeof(uint64_t) + 16;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
 }  // namespace mx
