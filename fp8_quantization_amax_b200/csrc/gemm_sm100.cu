@@ -605,14 +605,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
     for (int m = 0; m < MP; ++m) acc[m] = 0.0f;
     uint32_t r = 0, sph = 0, seg_k = 0;
     const uint32_t first_tile = lo / nkb;
-    for (uint32_t i = 0; i < n_units; ++i) {
-      const uint32_t u = lo + i, t = u / nkb;
-      const uint32_t buf = i % kTBuf;
-      if (!mbar_wait(&sfull[r], sph, p.err)) break;
-      if (!mbar_wait(&tfull[buf], (i / kTBuf) & 1u, p.err)) break;
-      tc_fence_after();
-      const float sb = sc_b[r];
-      uint32_t v[MP];
+    // Units are taken in pairs when the next unit belongs to the same tile: one round of waits,
+    // both partials loaded before one tcgen05.wait, applied in unit order (the same fp32 sums as
+    // one at a time), both buffers and scale slots released together.
+    auto ld_partial = [&](uint32_t buf, uint32_t (&v)[MP]) {
 #pragma unroll
       for (int c = 0; c < MP / 16; ++c) {
         asm volatile(
@@ -624,19 +620,49 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
               "=r"(v[c * 16 + 12]), "=r"(v[c * 16 + 13]), "=r"(v[c * 16 + 14]), "=r"(v[c * 16 + 15])
             : "r"(tmem_base + lane_addr + buf * kMaxMp + c * 16));
       }
+    };
+    for (uint32_t i = 0; i < n_units;) {
+      const uint32_t u0 = lo + i, t = u0 / nkb;
+      const bool pair = i + 1 < n_units && (u0 + 1) % nkb != 0;   // unit i + 1 is in tile t too
+      const uint32_t buf0 = i % kTBuf, buf1 = (i + 1) % kTBuf;
+      const uint32_t r0 = r, ph0 = sph;
+      const uint32_t r1 = r0 + 1 == (uint32_t)kScaleSlots ? 0u : r0 + 1;
+      const uint32_t ph1 = r0 + 1 == (uint32_t)kScaleSlots ? sph ^ 1u : sph;
+      if (!mbar_wait(&sfull[r0], ph0, p.err)) break;
+      if (!mbar_wait(&tfull[buf0], (i / kTBuf) & 1u, p.err)) break;
+      if (pair && !mbar_wait(&sfull[r1], ph1, p.err)) break;
+      if (pair && !mbar_wait(&tfull[buf1], ((i + 1) / kTBuf) & 1u, p.err)) break;
+      tc_fence_after();
+      uint32_t v0[MP], v1[MP];
+      ld_partial(buf0, v0);
+      if (pair) ld_partial(buf1, v1);
       tmem_ld_wait();
+      const float sb0 = sc_b[r0];
 #pragma unroll
-      for (int m = 0; m < MP; ++m) acc[m] = __fmaf_rn(sc_a[r][m] * sb, __uint_as_float(v[m]), acc[m]);
+      for (int m = 0; m < MP; ++m) acc[m] = __fmaf_rn(sc_a[r0][m] * sb0, __uint_as_float(v0[m]), acc[m]);
+      if (pair) {
+        const float sb1 = sc_b[r1];
+#pragma unroll
+        for (int m = 0; m < MP; ++m) acc[m] = __fmaf_rn(sc_a[r1][m] * sb1, __uint_as_float(v1[m]), acc[m]);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&tempty[buf]);
-        mbar_arrive(&sempty[r]);
+        mbar_arrive(&tempty[buf0]);
+        mbar_arrive(&sempty[r0]);
+        if (pair) {
+          mbar_arrive(&tempty[buf1]);
+          mbar_arrive(&sempty[r1]);
+        }
       }
-      if (++r == kScaleSlots) {
-        r = 0;
+      const uint32_t used = pair ? 2u : 1u;
+      r += used;
+      if (r >= (uint32_t)kScaleSlots) {
+        r -= kScaleSlots;
         sph ^= 1u;
       }
+      i += used;
+      const uint32_t u = u0 + used - 1;   // the last unit taken
       if (u + 1 == hi || (u + 1) % nkb == 0) {
         // this CTA's segment of tile t ends
         const uint32_t c_first = cta_of(t * nkb, p.W, p.G), c_last = cta_of(t * nkb + nkb - 1, p.W, p.G);
