@@ -24,7 +24,7 @@ __all__ = [
     "fp8_kv_quantize_noalloc", "fp8_gemm_blockscaled", "fp8_quantize_delayed", "fp8_kv_quantize_delayed",
     "linear_act_workspace_bytes", "fp8_linear_dynamic", "fp8_quantize_mx", "fp8_dequantize_mx",
     "mx_blocked_scale_bytes", "fp8_quantize_mx_blocked", "fp8_gemm_mx", "fp8_pack_b_tiles",
-    "fp8_gemm_blockscaled_packed", "fp8_scale_histogram", "fp8_count_underflow",
+    "fp8_gemm_blockscaled_packed", "fp8_scale_histogram", "fp8_count_underflow", "fp8_quantize_many",
 ]
 
 E4M3, E5M2 = 0, 1
@@ -35,6 +35,12 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libfp8q.so")
 _lock = threading.Lock()
 _lib = None
+
+
+class _QuantTensor(ctypes.Structure):
+    """fp8q_quant_tensor of include/fp8q.h."""
+    _fields_ = [("x", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("g", ctypes.c_int),
+                ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
 
 
 class Fp8qError(RuntimeError):
@@ -79,6 +85,7 @@ def lib() -> ctypes.CDLL:
             L.fp8_gemm_mx.argtypes = [vp, vp, i32, vp, vp, i32, i64, i64, i64, vp, vp]
             L.fp8_pack_b_tiles.argtypes = [vp, i64, i64, vp, vp]
             L.fp8_scale_histogram.argtypes = [vp, i64, i32, vp, vp]
+            L.fp8_quantize_many.argtypes = [ctypes.POINTER(_QuantTensor), i32, i32, vp]
             L.fp8_count_underflow.argtypes = [vp, vp, i64, vp, vp]
             L.fp8_gemm_blockscaled_packed.argtypes = [vp, vp, i32, vp, vp, i32, i64, i64, i64, vp, vp, sz, vp]
             L.fp8q_linear_act_workspace_bytes.argtypes = [i64, i64]
@@ -98,7 +105,8 @@ def lib() -> ctypes.CDLL:
                        "fp8_gemm_blockscaled", "fp8_kv_quantize_noalloc", "fp8_quantize_delayed",
                        "fp8_kv_quantize_delayed", "fp8_linear_dynamic", "fp8_quantize_mx", "fp8_dequantize_mx",
                        "fp8_quantize_mx_blocked", "fp8_gemm_mx", "fp8_pack_b_tiles",
-                       "fp8_gemm_blockscaled_packed", "fp8_scale_histogram", "fp8_count_underflow"):
+                       "fp8_gemm_blockscaled_packed", "fp8_scale_histogram", "fp8_count_underflow",
+                       "fp8_quantize_many"):
                 getattr(L, fn).restype = i32
             _lib = L
     return _lib
@@ -444,6 +452,31 @@ def fp8_gemm_blockscaled_packed(a: torch.Tensor, sa: torch.Tensor, bp: torch.Ten
     if st != 0 and cached:
         _gemm_ws.clear()
     _check("fp8_gemm_blockscaled_packed", st)
+    return out
+
+
+def fp8_quantize_many(jobs, fmt: int = E4M3):
+    """Quantize several bf16 tensors in one launch.  jobs: sequence of (x, granularity) or
+    (x, granularity, codes, scales) with granularity GROUP_1x128 or BLOCK_128x128; returns a list
+    of (codes, scales) identical to fp8_quantize of each."""
+    if not 1 <= len(jobs) <= 8:
+        raise ValueError("1 to 8 tensors per call")
+    arr = (_QuantTensor * len(jobs))()
+    out = []
+    for j, job in enumerate(jobs):
+        x, gran = job[0], job[1]
+        _dev(x, "x", torch.bfloat16)
+        if x.dim() != 2:
+            raise ValueError("x must be 2-D [rows][cols]")
+        rows, cols = x.shape
+        codes = job[2] if len(job) > 2 and job[2] is not None else torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+        scales = job[3] if len(job) > 3 and job[3] is not None else torch.empty(scale_shape(rows, cols, gran),
+                                                                               dtype=torch.float32, device=x.device)
+        _dev(codes, "codes", torch.uint8)
+        _dev(scales, "scales", torch.float32)
+        arr[j] = _QuantTensor(_ptr(x), rows, cols, gran, _ptr(codes), _ptr(scales))
+        out.append((codes, scales))
+    _check("fp8_quantize_many", lib().fp8_quantize_many(arr, len(jobs), fmt, _stream(jobs[0][0].device)))
     return out
 
 

@@ -120,6 +120,28 @@ fp8q_status fp8_quantize(const void* x, int64_t rows, int64_t cols, fp8q_format 
       fp8q::launch_quant_tiles(xs, nullptr, codes, nullptr, scales, nullptr, 1, rows, cols, cols, 128, f, st));
 }
 
+fp8q_status fp8_quantize_many(const fp8q_quant_tensor* tensors, int n, fp8q_format f, fp8q_stream_t stream) {
+  if (!tensors || n < 1 || n > fp8q::kMaxManyJobs || !valid_fmt(f)) return FP8Q_ERR_INVALID_ARGUMENT;
+  fp8q::QuantJob jobs[fp8q::kMaxManyJobs];
+  for (int j = 0; j < n; ++j) {
+    const fp8q_quant_tensor& t = tensors[j];
+    const int64_t e = checked_elems(t.rows, t.cols);
+    if (t.rows < 0 || t.cols < 0 || !valid_gran(t.g) || t.cols % 8 != 0) return FP8Q_ERR_INVALID_ARGUMENT;
+    if (t.g == FP8Q_PER_TENSOR) return FP8Q_ERR_UNSUPPORTED;
+    if (e < 0) return FP8Q_ERR_UNSUPPORTED;
+    if (e > 0 && (!t.x || !t.codes || !t.scales || !aligned(t.x, 16) || !aligned(t.codes, 16) ||
+                  !aligned(t.scales, 4)))
+      return FP8Q_ERR_INVALID_ARGUMENT;
+    jobs[j].x = static_cast<const uint16_t*>(t.x);
+    jobs[j].rows = t.rows;
+    jobs[j].cols = t.cols;
+    jobs[j].block = t.g == FP8Q_BLOCK_128x128 ? 1 : 0;
+    jobs[j].codes = t.codes;
+    jobs[j].scales = t.scales;
+  }
+  return from_cuda(fp8q::launch_quant_many(jobs, n, f, (cudaStream_t)stream));
+}
+
 fp8q_status fp8_quantize_mx(const void* x, int64_t rows, int64_t cols, fp8q_format f, uint8_t* codes,
                             uint8_t* scales, fp8q_stream_t stream) {
   const int64_t n = checked_elems(rows, cols);

@@ -79,6 +79,17 @@ cudaError_t launch_quant_delayed(const uint16_t* x0, const uint16_t* x1, uint8_t
                                  float* h0, float* h1, int64_t hlen, int64_t step, unsigned long long* counters,
                                  float* ws, cudaStream_t st);
 
+// several tensors, each in 1x128 groups (block = 0) or 128x128 blocks (block = 1), in one launch
+constexpr int kMaxManyJobs = 8;
+struct QuantJob {
+  const uint16_t* x;
+  int64_t rows, cols;
+  int block;
+  uint8_t* codes;
+  float* scales;
+};
+cudaError_t launch_quant_many(const QuantJob* jobs, int n, int fmt, cudaStream_t st);
+
 // MXFP8: 1x32 groups along rows (cols % 32 == 0), scales as byte exponents, row-major
 // [rows][cols / 32] (blocked = 0) or in the blocked layout of the block-scaled MMA (blocked = 1:
 // ceil(rows / 128) x ceil(cols / 128) chunks of 512 bytes)

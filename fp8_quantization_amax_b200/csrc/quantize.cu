@@ -818,4 +818,228 @@ cudaError_t launch_quant_delayed(const uint16_t* x0, const uint16_t* x1, uint8_t
                     ntens > 1 ? h1 : h0, step % hlen);
 }
 
+
+// ============================================================================ several tensors, one launch
+//
+// Up to kMaxJobs tensors, each quantized in 1x128 groups or 128x128 blocks, in one persistent
+// launch: every tensor is cut into 128 x 128 bf16 boxes (the 32 KB stages above), the boxes of
+// all tensors form one item list split over the CTAs with the grid stride, so one ring, one ramp
+// and one tail serve them all, and the work divides evenly however the tensors' box counts fall.
+// A box is consumed as its tensor's granularity requires, with the arithmetic of k_group128
+// (per-row amax, four threads per row) or of k_tile128's one-pass mode (CTA-wide amax): the
+// codes and scales are those of separate calls.
+
+struct ManyJob {
+  uint8_t* codes;
+  float* scales;
+  int64_t rows, cols;
+  uint32_t first;    // first item of this tensor in the combined list
+  FastDiv nbc;       // 128-column boxes across
+  int block;         // 1: 128x128 blocks; 0: 1x128 groups
+  int wide;          // cols % 16 == 0: 16-byte code stores
+};
+
+struct ManyMaps {
+  CUtensorMap m[kMaxManyJobs];
+};
+
+struct ManyParams {
+  ManyJob job[kMaxManyJobs];
+  int njobs;
+  uint32_t nitems;
+  int stages;
+  uint32_t* err;
+};
+
+__device__ __forceinline__ int many_job_of(uint32_t i, const ManyParams& p) {
+  int j = 0;
+  while (j + 1 < p.njobs && i >= p.job[j + 1].first) ++j;
+  return j;
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(kThreads, 2) k_quant_many(const __grid_constant__ ManyMaps maps,
+                                                             const __grid_constant__ ManyParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = ring_base(smem_raw);
+  __shared__ uint32_t red[2][kConsumerWarps];
+  const int S = p.stages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * kGroupStage);
+  uint64_t* empty = full + kMaxStages;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
+    }
+    fence_mbar_init();
+  }
+  const uint32_t nk = items_of_cta(p.nitems);
+  if (warp == kConsumerWarps && lane == 0 && nk > 0) {
+    // warm L2 with this CTA's first boxes while the previous grid on the stream finishes
+    for (int j = 0; j < p.njobs; ++j)
+      if (p.job[j].rows > 0 && p.job[j].cols > 0) tma_prefetch_desc(&maps.m[j]);
+    for (uint32_t k = 0; k < nk && k < (uint32_t)S; ++k) {
+      const uint32_t i = blockIdx.x + k * gridDim.x;
+      const int j = many_job_of(i, p);
+      const uint32_t local = i - p.job[j].first, rb = fdiv(local, p.job[j].nbc), g = local - rb * p.job[j].nbc.d;
+      tma_prefetch_l2_2d(&maps.m[j], (int32_t)(g * 128), (int32_t)(rb * 128));
+    }
+  }
+  __syncthreads();
+  allow_dependent_launch();
+  grid_dependency_wait();
+  if (warp == kConsumerWarps) {
+    if (lane == 0 && nk > 0) {
+      run_producer(
+          full, empty, S, nk, kGroupStage, p.err, [&](uint32_t k) { return blockIdx.x + k * gridDim.x; },
+          [&](uint32_t i, int s, uint64_t* bar) {
+            const int j = many_job_of(i, p);
+            const uint32_t local = i - p.job[j].first, rb = fdiv(local, p.job[j].nbc), g = local - rb * p.job[j].nbc.d;
+            tma_load_2d(smem + s * kGroupStage, &maps.m[j], (int32_t)(g * 128), (int32_t)(rb * 128), bar);
+          });
+    }
+    return;
+  }
+  const int t = threadIdx.x;
+  int s = 0;
+  uint32_t ph = 0, nblock = 0;   // nblock: 128x128 items so far (their reduction slots alternate)
+  for (uint32_t k = 0; k < nk; ++k) {
+    const uint32_t i = blockIdx.x + k * gridDim.x;
+    const ManyJob& J = p.job[many_job_of(i, p)];
+    const uint32_t local = i - J.first, rb = fdiv(local, J.nbc), g = local - rb * J.nbc.d;
+    if (!mbar_wait(&full[s], ph, p.err)) break;
+    const uint8_t* stage = smem + s * kGroupStage;
+    if (J.block) {
+      // 128x128 block (k_tile128 one-pass, 16-byte pieces per row CPR = 16): thread t owns the
+      // 32-byte chunk pairs t + 256 jp, i.e. rows t / 8 + 32 jp, 16-column block t % 8
+      uint4 va[4], vb[4];
+      uint32_t m = 0u;
+#pragma unroll
+      for (int jp = 0; jp < 4; ++jp) {
+        const uint8_t* src = stage + (t + kConsumers * jp) * 32;
+        va[jp] = ld_shared_v4(src);
+        vb[jp] = ld_shared_v4(src + 16);
+        m = absmax_v4(absmax_v4(m, va[jp]), vb[jp]);
+      }
+      release_stage(&empty[s], lane);
+      if (++s == S) {
+        s = 0;
+        ph ^= 1u;
+      }
+#pragma unroll
+      for (int d = 16; d >= 1; d >>= 1) m = absmax2(m, __shfl_xor_sync(0xFFFFFFFFu, m, d));
+      const uint32_t slot = nblock++ & 1u;
+      if (lane == 0) red[slot][warp] = m;
+      named_barrier(1, kConsumers);
+      uint32_t mm = red[slot][0];
+#pragma unroll
+      for (int w = 1; w < kConsumerWarps; ++w) mm = absmax2(mm, red[slot][w]);
+      const GroupScale gs = make_group_scale<FMT>(packed_amax_to_f32(mm));
+      if (t == 0) J.scales[(size_t)rb * J.nbc.d + g] = gs.s;
+      const int r0 = t >> 3, cp = t & 7;
+      const int64_t row_base = (int64_t)rb * 128, col_base = (int64_t)g * 128;
+      if (gs.fast && J.wide && row_base + 128 <= J.rows && col_base + 128 <= J.cols) {
+        uint8_t* dst = J.codes + (row_base + r0) * J.cols + col_base + cp * 16;
+#pragma unroll
+        for (int jp = 0; jp < 4; ++jp) st_stream_v4(dst + jp * 32 * J.cols, quant16_fast<FMT>(va[jp], vb[jp], gs.d, gs.r));
+      } else {
+#pragma unroll
+        for (int jp = 0; jp < 4; ++jp) {
+          const int64_t row = row_base + r0 + jp * 32, col = col_base + cp * 16;
+          uint8_t* dst = J.codes + row * J.cols + col;
+          if (row < J.rows && col < J.cols) st_stream_v2(dst, quant8<FMT>(va[jp], gs));
+          if (row < J.rows && col + 8 < J.cols) st_stream_v2(dst + 8, quant8<FMT>(vb[jp], gs));
+        }
+      }
+    } else {
+      // 1x128 groups (k_group128): thread (grp, q) owns chunk pairs q and q + 4 of box rows grp
+      // and grp + 64
+      const int grp = t >> 2, q = t & 3;
+      const uint32_t soff = grp * 256 + q * 32;
+      uint4 v[kGroupRowsPerThread][4];
+      uint32_t m[kGroupRowsPerThread];
+#pragma unroll
+      for (int h = 0; h < kGroupRowsPerThread; ++h) {
+        const uint8_t* src = stage + soff + h * 64 * 256;
+        v[h][0] = ld_shared_v4(src);
+        v[h][1] = ld_shared_v4(src + 16);
+        v[h][2] = ld_shared_v4(src + 128);
+        v[h][3] = ld_shared_v4(src + 144);
+        m[h] = absmax_v4(absmax_v4(absmax_v4(absmax_v4(0u, v[h][0]), v[h][1]), v[h][2]), v[h][3]);
+      }
+      release_stage(&empty[s], lane);
+      if (++s == S) {
+        s = 0;
+        ph ^= 1u;
+      }
+#pragma unroll
+      for (int h = 0; h < kGroupRowsPerThread; ++h) {
+        uint32_t mh = absmax2(m[h], __shfl_xor_sync(0xFFFFFFFFu, m[h], 1));
+        mh = absmax2(mh, __shfl_xor_sync(0xFFFFFFFFu, mh, 2));
+        const GroupScale gs = make_group_scale<FMT>(packed_amax_to_f32(mh));
+        const int64_t row = (int64_t)rb * kGroupBoxRows + grp + h * 64;
+        if (row >= J.rows) continue;
+        const int64_t col0 = (int64_t)g * 128 + q * 16, col1 = col0 + 64;
+        uint8_t* dst = J.codes + row * J.cols;
+        if (gs.fast && J.wide && (int64_t)g * 128 + 128 <= J.cols) {
+          st_stream_v4(dst + col0, quant16_fast<FMT>(v[h][0], v[h][1], gs.d, gs.r));
+          st_stream_v4(dst + col1, quant16_fast<FMT>(v[h][2], v[h][3], gs.d, gs.r));
+        } else {
+          if (col0 < J.cols) st_stream_v2(dst + col0, quant8<FMT>(v[h][0], gs));
+          if (col0 + 8 < J.cols) st_stream_v2(dst + col0 + 8, quant8<FMT>(v[h][1], gs));
+          if (col1 < J.cols) st_stream_v2(dst + col1, quant8<FMT>(v[h][2], gs));
+          if (col1 + 8 < J.cols) st_stream_v2(dst + col1 + 8, quant8<FMT>(v[h][3], gs));
+        }
+        if (q == 0) J.scales[(int64_t)g * J.rows + row] = gs.s;
+      }
+    }
+  }
+}
+
+template <int FMT>
+static cudaError_t launch_many_fmt(const ManyMaps& maps, const ManyParams& p, cudaStream_t st) {
+  const size_t smem = ring_smem(p.stages, kGroupStage);
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(k_quant_many<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    attr = true;
+  }
+  const int grid = grid_for(k_quant_many<FMT>, smem, p.nitems);
+  return launch_pdl(k_quant_many<FMT>, dim3(grid), dim3(kThreads), smem, st, maps, p);
+}
+
+cudaError_t launch_quant_many(const QuantJob* jobs, int n, int fmt, cudaStream_t st) {
+  if (n < 1 || n > kMaxManyJobs) return cudaErrorInvalidValue;
+  ManyMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  ManyParams p;
+  std::memset(&p, 0, sizeof(p));
+  uint64_t items = 0;
+  for (int j = 0; j < n; ++j) {
+    const QuantJob& q = jobs[j];
+    ManyJob& J = p.job[j];
+    J.codes = q.codes;
+    J.scales = q.scales;
+    J.rows = q.rows;
+    J.cols = q.cols;
+    J.block = q.block;
+    J.wide = q.cols % 16 == 0;
+    const int64_t nbr = (q.rows + 127) / 128, nbc = (q.cols + 127) / 128;
+    J.nbc = make_fastdiv((uint32_t)std::max<int64_t>(nbc, 1));
+    J.first = (uint32_t)items;
+    items += (uint64_t)(nbr * nbc);
+    if (items >= (1ull << 32)) return cudaErrorInvalidValue;
+    if (nbr * nbc > 0 &&
+        !make_tmap_2d(&maps.m[j], 2, q.x, (uint64_t)q.cols, (uint64_t)q.rows, (uint64_t)q.cols * 2, 128, 128, 0))
+      return cudaErrorInvalidValue;
+  }
+  if (items == 0) return cudaSuccess;
+  p.njobs = n;
+  p.nitems = (uint32_t)items;
+  p.stages = (int)ring_stages(kGroupStage);
+  p.err = device_error_word();
+  return fmt == kE4M3 ? launch_many_fmt<kE4M3>(maps, p, st) : launch_many_fmt<kE5M2>(maps, p, st);
+}
+
 }  // namespace fp8q

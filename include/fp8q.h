@@ -201,6 +201,29 @@ FP8Q_API fp8q_status fp8_kv_quantize_noalloc(const void *k, const void *v, int64
                                              uint8_t *k_codes, uint8_t *v_codes, float *k_scales,
                                              float *v_scales, fp8q_stream_t stream);
 
+/*
+ * Several tensors in one launch ([W] "权重量化：128x128 分块 FP8" and "激活动态量化": e.g. a
+ * layer's weight blocks and its activations).  Each entry is quantized exactly as fp8_quantize
+ * with its granularity would (same codes, same scales, same layouts); one persistent kernel
+ * walks the 128 x 128 boxes of all entries, so the launch overhead, ramp and tail are paid once.
+ *   tensors  host array of n entries (1 <= n <= 8); each: x bf16 [rows][cols] (device, 16-byte
+ *            aligned, cols % 8 == 0), granularity FP8Q_GROUP_1x128 or FP8Q_BLOCK_128x128
+ *            (FP8Q_PER_TENSOR needs two passes: FP8Q_ERR_UNSUPPORTED), codes uint8
+ *            [rows][cols] (16-byte aligned), scales fp32, fp8q_num_scales(rows, cols, g)
+ *            entries (4-byte aligned).  Entries must not overlap one another's outputs.
+ *   f        one format for all entries
+ * The array is read during the call only.
+ */
+typedef struct {
+  const void *x;
+  int64_t rows, cols;
+  fp8q_granularity g;
+  uint8_t *codes;
+  float *scales;
+} fp8q_quant_tensor;
+FP8Q_API fp8q_status fp8_quantize_many(const fp8q_quant_tensor *tensors, int n, fp8q_format f,
+                                       fp8q_stream_t stream);
+
 /* ---------------------------------------------------------------- MXFP8 */
 
 /*

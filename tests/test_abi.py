@@ -191,3 +191,19 @@ def test_health_rejects(L):
     assert L.fp8_count_underflow(a, m, 64, a, None) == 1                # misaligned codes
     assert L.fp8_count_underflow(a, a, -1, a, None) == 1
     assert L.fp8_count_underflow(None, None, 0, None, None) == 0
+
+
+@host_only
+def test_quantize_many_rejects(L):
+    arr = (fq._QuantTensor * 9)()
+    arr[0] = fq._QuantTensor(1 << 20, 128, 128, 0, 1 << 20, 1 << 20)
+    assert L.fp8_quantize_many(arr, 1, 0, None) == 2                  # per-tensor needs two passes
+    arr[0] = fq._QuantTensor(1 << 20, 128, 100, 1, 1 << 20, 1 << 20)
+    assert L.fp8_quantize_many(arr, 1, 0, None) == 1                  # cols % 8
+    assert L.fp8_quantize_many(arr, 9, 0, None) == 1                  # more than 8 tensors
+    assert L.fp8_quantize_many(arr, 0, 0, None) == 1
+    assert L.fp8_quantize_many(None, 1, 0, None) == 1
+    arr[0] = fq._QuantTensor((1 << 20) + 8, 128, 128, 2, 1 << 20, 1 << 20)
+    assert L.fp8_quantize_many(arr, 1, 0, None) == 1                  # x not 16-byte aligned
+    arr[0] = fq._QuantTensor(None, 0, 128, 1, None, None)
+    assert L.fp8_quantize_many(arr, 1, 0, None) == 0                  # empty
