@@ -452,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
                                                              const __grid_constant__ CUtensorMap tX, Params p) {
   constexpr uint32_t kIdescD = (1u << 4) | ((uint32_t)(MP >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  __shared__ float sc_a[kScaleSlots][MP];
+  __shared__ __align__(16) float sc_a[kScaleSlots][MP];
   __shared__ float sc_b[kScaleSlots];
   __shared__ uint64_t bars[2 * kMaxStages + 2 * kTBuf + 2 * kScaleSlots + 2];
   __shared__ uint32_t tmem_slot;
@@ -637,14 +637,28 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
       ld_partial(buf0, v0);
       if (pair) ld_partial(buf1, v1);
       tmem_ld_wait();
-      const float sb0 = sc_b[r0];
+      // acc[m] += RN(sA[m] * sB) * P[m] on packed pairs (two independent roundings each: the
+      // same values as one element at a time)
+      auto promote = [&](uint32_t rs, const uint32_t (&v)[MP]) {
+        const float sb = sc_b[rs];
+        const float2 sb2 = make_float2(sb, sb);
 #pragma unroll
-      for (int m = 0; m < MP; ++m) acc[m] = __fmaf_rn(sc_a[r0][m] * sb0, __uint_as_float(v0[m]), acc[m]);
-      if (pair) {
-        const float sb1 = sc_b[r1];
-#pragma unroll
-        for (int m = 0; m < MP; ++m) acc[m] = __fmaf_rn(sc_a[r1][m] * sb1, __uint_as_float(v1[m]), acc[m]);
-      }
+        for (int m = 0; m < MP; m += 4) {
+          const float4 a4 = *reinterpret_cast<const float4*>(&sc_a[rs][m]);
+          const float2 c01 = __fmul2_rn(make_float2(a4.x, a4.y), sb2);
+          const float2 c23 = __fmul2_rn(make_float2(a4.z, a4.w), sb2);
+          const float2 s01 = __ffma2_rn(c01, make_float2(__uint_as_float(v[m]), __uint_as_float(v[m + 1])),
+                                        make_float2(acc[m], acc[m + 1]));
+          const float2 s23 = __ffma2_rn(c23, make_float2(__uint_as_float(v[m + 2]), __uint_as_float(v[m + 3])),
+                                        make_float2(acc[m + 2], acc[m + 3]));
+          acc[m] = s01.x;
+          acc[m + 1] = s01.y;
+          acc[m + 2] = s23.x;
+          acc[m + 3] = s23.y;
+        }
+      };
+      promote(r0, v0);
+      if (pair) promote(r1, v1);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
