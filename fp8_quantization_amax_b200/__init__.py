@@ -25,6 +25,7 @@ __all__ = [
     "linear_act_workspace_bytes", "fp8_linear_dynamic", "fp8_quantize_mx", "fp8_dequantize_mx",
     "mx_blocked_scale_bytes", "fp8_quantize_mx_blocked", "fp8_gemm_mx", "fp8_pack_b_tiles",
     "fp8_gemm_blockscaled_packed", "fp8_scale_histogram", "fp8_count_underflow", "fp8_quantize_many",
+    "selftest_wait_timeout",
 ]
 
 E4M3, E5M2 = 0, 1
@@ -85,6 +86,8 @@ def lib() -> ctypes.CDLL:
             L.fp8_gemm_mx.argtypes = [vp, vp, i32, vp, vp, i32, i64, i64, i64, vp, vp]
             L.fp8_pack_b_tiles.argtypes = [vp, i64, i64, vp, vp]
             L.fp8_scale_histogram.argtypes = [vp, i64, i32, vp, vp]
+            L.fp8q_selftest_wait_timeout.argtypes = [vp]
+            L.fp8q_selftest_wait_timeout.restype = i32
             L.fp8_quantize_many.argtypes = [ctypes.POINTER(_QuantTensor), i32, i32, vp]
             L.fp8_count_underflow.argtypes = [vp, vp, i64, vp, vp]
             L.fp8_gemm_blockscaled_packed.argtypes = [vp, vp, i32, vp, vp, i32, i64, i64, i64, vp, vp, sz, vp]
@@ -453,6 +456,13 @@ def fp8_gemm_blockscaled_packed(a: torch.Tensor, sa: torch.Tensor, bp: torch.Ten
         _gemm_ws.clear()
     _check("fp8_gemm_blockscaled_packed", st)
     return out
+
+
+def selftest_wait_timeout(device=None) -> None:
+    """Launch the failure-detection self-test on the current stream: one bounded wait on a
+    barrier nothing completes gives up after its time limit and sets bit 0 of device_status()."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    _check("fp8q_selftest_wait_timeout", lib().fp8q_selftest_wait_timeout(_stream(dev)))
 
 
 def fp8_quantize_many(jobs, fmt: int = E4M3):

@@ -7,6 +7,10 @@
 #include "fp8q.h"
 #include "internal.h"
 
+namespace fp8q {
+cudaError_t launch_selftest_wait(cudaStream_t st);
+}
+
 namespace {
 
 constexpr int64_t kMaxElems = int64_t(1) << 33;   // 32-bit indexing of 16-byte pieces of two tensors
@@ -48,6 +52,10 @@ const char* fp8q_status_string(fp8q_status status) {
 int fp8q_version(void) { return 100; }
 
 uint32_t fp8q_device_status(void) { return fp8q::read_and_clear_device_error(); }
+
+fp8q_status fp8q_selftest_wait_timeout(fp8q_stream_t stream) {
+  return from_cuda(fp8q::launch_selftest_wait((cudaStream_t)stream));
+}
 
 size_t fp8q_num_scales(int64_t rows, int64_t cols, fp8q_granularity g) {
   if (rows < 0 || cols < 0 || !valid_gran(g)) return 0;

@@ -111,6 +111,15 @@ FP8Q_API int fp8q_version(void);
  */
 FP8Q_API uint32_t fp8q_device_status(void);
 
+/*
+ * Failure-detection self-test: launches one block whose thread waits, through the same bounded
+ * wait every kernel of the library uses, on a pipeline barrier that nothing ever completes.
+ * After the time limit (2 s) the wait gives up, sets bit 0 of the device error bits and the
+ * kernel returns normally (no trap, no fault; the context stays usable).  A following
+ * fp8q_device_status() therefore returns bit 0 set.  Asynchronous on `stream`.
+ */
+FP8Q_API fp8q_status fp8q_selftest_wait_timeout(fp8q_stream_t stream);
+
 /* ---------------------------------------------------------------- sizes */
 
 /* Number of fp32 scales fp8_quantize writes for a [rows][cols] tensor; 0 on a bad argument. */
