@@ -382,6 +382,20 @@ def supplementary(device, stream, peaks, flush):
             fq.fp8_gemm_blockscaled(a, sa, wc, ws, out=cbuf)
             ms = timed(lambda: fq.fp8_gemm_blockscaled(a, sa, wc, ws, out=cbuf), 10, stream, flush)
             out["gemm_8b_up_m8192"] = gemm_entry(m, W_SHAPE[0], W_SHAPE[1], ms, a, sa, ws, cbuf)
+            # the same GEMM with C quantized to E4M3 1x128 groups in the epilogue, against the two
+            # steps it replaces (bf16 C, then the 1x128 quantizer)
+            qc = torch.empty((m, W_SHAPE[0]), dtype=torch.uint8, device=device)
+            qs = torch.empty(fq.scale_shape(m, W_SHAPE[0], fq.GROUP_1x128), dtype=torch.float32, device=device)
+            fq.fp8_gemm_blockscaled_to_fp8(a, sa, wc, ws, codes=qc, scales=qs)
+            ms_f = timed(lambda: fq.fp8_gemm_blockscaled_to_fp8(a, sa, wc, ws, codes=qc, scales=qs), 10, stream, flush)
+            ms_2 = timed(lambda: (fq.fp8_gemm_blockscaled(a, sa, wc, ws, out=cbuf),
+                                  fq.fp8_quantize(cbuf, fq.E4M3, fq.GROUP_1x128, codes=qc, scales=qs)), 10, stream,
+                         flush)
+            flops = 2.0 * m * W_SHAPE[0] * W_SHAPE[1]
+            out["gemm_8b_up_m8192_to_fp8"] = {"us": round(ms_f * 1e3, 2), "TFLOP/s": round(flops / ms_f / 1e9, 1),
+                                              "frac_fp8_peak": round(flops / ms_f / 1e9 / fp8_peak, 3),
+                                              "two_steps_us": round(ms_2 * 1e3, 2)}
+            del qc, qs
             # MXFP8 on the native block-scaled MMA, same shape: both operands quantized in 1x32
             # groups with power-of-two scales (blocked layout)
             am, sam = fq.fp8_quantize_mx_blocked(dev_bf16(synth.activations(seed=1), device))

@@ -25,7 +25,7 @@ __all__ = [
     "linear_act_workspace_bytes", "fp8_linear_dynamic", "fp8_quantize_mx", "fp8_dequantize_mx",
     "mx_blocked_scale_bytes", "fp8_quantize_mx_blocked", "fp8_gemm_mx", "fp8_pack_b_tiles",
     "fp8_gemm_blockscaled_packed", "fp8_scale_histogram", "fp8_count_underflow", "fp8_quantize_many",
-    "selftest_wait_timeout",
+    "selftest_wait_timeout", "fp8_gemm_blockscaled_to_fp8",
 ]
 
 E4M3, E5M2 = 0, 1
@@ -87,6 +87,8 @@ def lib() -> ctypes.CDLL:
             L.fp8_pack_b_tiles.argtypes = [vp, i64, i64, vp, vp]
             L.fp8_scale_histogram.argtypes = [vp, i64, i32, vp, vp]
             L.fp8q_selftest_wait_timeout.argtypes = [vp]
+            L.fp8_gemm_blockscaled_to_fp8.argtypes = [vp, vp, i32, vp, vp, i32, i64, i64, i64, vp, vp, vp]
+            L.fp8_gemm_blockscaled_to_fp8.restype = i32
             L.fp8q_selftest_wait_timeout.restype = i32
             L.fp8_quantize_many.argtypes = [ctypes.POINTER(_QuantTensor), i32, i32, vp]
             L.fp8_count_underflow.argtypes = [vp, vp, i64, vp, vp]
@@ -418,6 +420,29 @@ def fp8_gemm_blockscaled(a: torch.Tensor, sa: torch.Tensor, b: torch.Tensor, sb:
         _gemm_ws.clear()
     _check("fp8_gemm_blockscaled", st)
     return out
+
+
+def fp8_gemm_blockscaled_to_fp8(a: torch.Tensor, sa: torch.Tensor, b: torch.Tensor, sb: torch.Tensor,
+                                ga: int = GROUP_1x128, gb: int = BLOCK_128x128, codes: torch.Tensor | None = None,
+                                scales: torch.Tensor | None = None):
+    """The block-scaled GEMM (prefill shapes, M > 64) with C quantized in the epilogue:
+    -> (codes uint8 [M][N], scales float32 [N/128][M]), identical to fp8_gemm_blockscaled followed
+    by fp8_quantize(C, E4M3, GROUP_1x128)."""
+    _dev(a, "a", torch.uint8)
+    _dev(b, "b", torch.uint8)
+    _dev(sa, "sa", torch.float32)
+    _dev(sb, "sb", torch.float32)
+    M, K = a.shape
+    N, K2 = b.shape
+    if K != K2:
+        raise ValueError("a and b disagree on K")
+    codes = torch.empty((M, N), dtype=torch.uint8, device=a.device) if codes is None else _dev(codes, "codes", torch.uint8)
+    scales = torch.empty(scale_shape(M, N, GROUP_1x128), dtype=torch.float32, device=a.device) if scales is None else \
+        _dev(scales, "scales", torch.float32)
+    _check("fp8_gemm_blockscaled_to_fp8", lib().fp8_gemm_blockscaled_to_fp8(_ptr(a), _ptr(sa), ga, _ptr(b), _ptr(sb), gb,
+                                                                           M, N, K, _ptr(codes), _ptr(scales),
+                                                                           _stream(a.device)))
+    return codes, scales
 
 
 def fp8_pack_b_tiles(b: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:

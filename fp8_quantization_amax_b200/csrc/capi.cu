@@ -324,6 +324,26 @@ fp8q_status fp8_count_underflow(const void* x, const uint8_t* codes, int64_t n, 
                                                 (cudaStream_t)stream));
 }
 
+fp8q_status fp8_gemm_blockscaled_to_fp8(const uint8_t* A, const float* sA, fp8q_granularity gA, const uint8_t* B,
+                                        const float* sB, fp8q_granularity gB, int64_t M, int64_t N, int64_t K,
+                                        uint8_t* codes, float* scales, fp8q_stream_t stream) {
+  if (M < 0 || N < 0 || K < 0) return FP8Q_ERR_INVALID_ARGUMENT;
+  if (!(gA == FP8Q_GROUP_1x128 || gA == FP8Q_PER_TENSOR)) return FP8Q_ERR_INVALID_ARGUMENT;
+  if (!(gB == FP8Q_BLOCK_128x128 || gB == FP8Q_PER_TENSOR)) return FP8Q_ERR_INVALID_ARGUMENT;
+  if (M == 0 || N == 0) return FP8Q_OK;
+  if (N % 128 != 0 || K % 128 != 0 || K == 0) return FP8Q_ERR_UNSUPPORTED;
+  if (checked_elems(M, K) < 0 || checked_elems(N, K) < 0 || checked_elems(M, N) < 0) return FP8Q_ERR_UNSUPPORTED;
+  if (M > (int64_t(1) << 31) - 1 || N > (int64_t(1) << 31) - 1) return FP8Q_ERR_UNSUPPORTED;
+  if (fp8q::gemm_workspace_bytes(M, N, K) > 0) return FP8Q_ERR_UNSUPPORTED;   // decode shapes
+  if (!A || !B || !codes || !sA || !sB || !scales || !aligned(A, 16) || !aligned(B, 16) || !aligned(codes, 16) ||
+      !aligned(sA, 4) || !aligned(sB, 4) || !aligned(scales, 4))
+    return FP8Q_ERR_INVALID_ARGUMENT;
+  const cudaError_t e = fp8q::launch_gemm_to_fp8(A, sA, gA, B, false, sB, gB, M, N, K, codes, scales,
+                                                 (cudaStream_t)stream);
+  if (e == cudaErrorNotSupported) return FP8Q_ERR_UNSUPPORTED;
+  return from_cuda(e);
+}
+
 fp8q_status fp8_pack_b_tiles(const uint8_t* B, int64_t N, int64_t K, uint8_t* packed, fp8q_stream_t stream) {
   if (N < 0 || K < 0) return FP8Q_ERR_INVALID_ARGUMENT;
   if (N % 128 != 0 || K % 128 != 0) return FP8Q_ERR_UNSUPPORTED;

@@ -77,8 +77,33 @@ struct Params {
   int gB_block;       // 1: sB is [N/128][K/128]; 0: one scale
   const uint8_t* Bp;  // packed B tiles (16 KB each, tile (nb, kb) at nb * num_kb + kb), or null: B via TMA
   uint16_t* C;
+  uint8_t* q_codes;   // non-null: the output is quantized (E4M3, 1x128 groups) instead of stored as bf16
+  float* q_scales;    // [N/128][M]
   uint32_t* err;
 };
+
+// The 1x128 E4M3 quantizer on one 128-column row segment of C held by one thread as 64 packed
+// bf16 pairs (the values a bf16 C would store): the group's amax, its scale, the codes and the
+// scale, with the arithmetic of the stand-alone quantizer, so the result equals quantizing the
+// bf16 C in a second pass.
+__device__ __forceinline__ void store_row_e4m3(const uint32_t (&w)[64], uint8_t* codes_row, float* scale) {
+  uint32_t m = 0u;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) m = absmax_v4(m, make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]));
+  const GroupScale gs = make_group_scale<kE4M3>(packed_amax_to_f32(m));
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint4 a = make_uint4(w[8 * c], w[8 * c + 1], w[8 * c + 2], w[8 * c + 3]);
+    const uint4 b = make_uint4(w[8 * c + 4], w[8 * c + 5], w[8 * c + 6], w[8 * c + 7]);
+    if (gs.fast) {
+      st_stream_v4(codes_row + 16 * c, quant16_fast<kE4M3>(a, b, gs.d, gs.r));
+    } else {
+      st_stream_v2(codes_row + 16 * c, quant8<kE4M3>(a, gs));
+      st_stream_v2(codes_row + 16 * c + 8, quant8<kE4M3>(b, gs));
+    }
+  }
+  *scale = gs.s;
+}
 
 __device__ __forceinline__ void tile_coords(int t, const Params& p, int* m0, int* n0) {
   const int mt = t % p.m_tiles, nt = t / p.m_tiles;
@@ -330,15 +355,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ CU
           const int m = m0 + row_in_tile;
           const int ncol0 = n0 + half * 128;
           if (m < p.M && ncol0 < p.N) {
-            uint16_t* dst = p.C + (size_t)m * p.N + ncol0;
+            if (p.q_codes) {
+              uint32_t w[64];
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              uint4 wv;
-              wv.x = f32x2_to_bf16x2(acc[c * 4 + 0].x, acc[c * 4 + 0].y);
-              wv.y = f32x2_to_bf16x2(acc[c * 4 + 1].x, acc[c * 4 + 1].y);
-              wv.z = f32x2_to_bf16x2(acc[c * 4 + 2].x, acc[c * 4 + 2].y);
-              wv.w = f32x2_to_bf16x2(acc[c * 4 + 3].x, acc[c * 4 + 3].y);
-              st_stream_v4(dst + c * 8, wv);
+              for (int i = 0; i < 64; ++i) w[i] = f32x2_to_bf16x2(acc[i].x, acc[i].y);
+              store_row_e4m3(w, p.q_codes + (size_t)m * p.N + ncol0, p.q_scales + (size_t)(ncol0 >> 7) * p.M + m);
+            } else {
+              uint16_t* dst = p.C + (size_t)m * p.N + ncol0;
+#pragma unroll
+              for (int c = 0; c < 16; ++c) {
+                uint4 wv;
+                wv.x = f32x2_to_bf16x2(acc[c * 4 + 0].x, acc[c * 4 + 0].y);
+                wv.y = f32x2_to_bf16x2(acc[c * 4 + 1].x, acc[c * 4 + 1].y);
+                wv.z = f32x2_to_bf16x2(acc[c * 4 + 2].x, acc[c * 4 + 2].y);
+                wv.w = f32x2_to_bf16x2(acc[c * 4 + 3].x, acc[c * 4 + 3].y);
+                st_stream_v4(dst + c * 8, wv);
+              }
             }
           }
           kb = 0;
@@ -372,10 +404,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ CU
         if (lane == 0) mbar_arrive(&tempty[buf]);
         ++acc_use;
         if (m < p.M && ncol0 < p.N) {
-          uint16_t* dst = p.C + (size_t)m * p.N + ncol0;
+          if (p.q_codes) {
+            store_row_e4m3(out, p.q_codes + (size_t)m * p.N + ncol0, p.q_scales + (size_t)(ncol0 >> 7) * p.M + m);
+          } else {
+            uint16_t* dst = p.C + (size_t)m * p.N + ncol0;
 #pragma unroll
-          for (int c = 0; c < 16; ++c)
-            st_stream_v4(dst + c * 8, make_uint4(out[c * 4], out[c * 4 + 1], out[c * 4 + 2], out[c * 4 + 3]));
+            for (int c = 0; c < 16; ++c)
+              st_stream_v4(dst + c * 8, make_uint4(out[c * 4], out[c * 4 + 1], out[c * 4 + 2], out[c * 4 + 3]));
+          }
         }
       }
     }
@@ -859,13 +895,11 @@ cudaError_t launch_decode_gemm(const DecodePlan& plan, const uint8_t* A, const f
 
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) { return decode_plan(M, N, K).ws_bytes; }
 
-cudaError_t launch_gemm(const uint8_t* A, const float* sA, int gA, const uint8_t* B, bool b_packed, const float* sB,
-                        int gB, int64_t M, int64_t N, int64_t K, uint16_t* C, void* ws, size_t ws_bytes,
-                        cudaStream_t st) {
+// the prefill kernel (M > 64): C in bf16, or (q_codes non-null) quantized to E4M3 1x128 groups
+static cudaError_t launch_prefill(const uint8_t* A, const float* sA, int gA, const uint8_t* B, bool b_packed,
+                                  const float* sB, int gB, int64_t M, int64_t N, int64_t K, uint16_t* C,
+                                  uint8_t* q_codes, float* q_scales, cudaStream_t st) {
   using namespace gemm;
-  if (M == 0 || N == 0) return cudaSuccess;
-  const DecodePlan plan = decode_plan(M, N, K);
-  if (plan.mp > 0) return launch_decode_gemm(plan, A, sA, gA, B, b_packed, sB, gB, M, N, K, C, ws, ws_bytes, st);
   CUtensorMap mA, mB;
   std::memset(&mA, 0, sizeof(mA));
   std::memset(&mB, 0, sizeof(mB));
@@ -886,6 +920,8 @@ cudaError_t launch_gemm(const uint8_t* A, const float* sA, int gA, const uint8_t
   p.gB_block = gB == 2;
   p.Bp = b_packed ? B : nullptr;
   p.C = C;
+  p.q_codes = q_codes;
+  p.q_scales = q_scales;
   p.err = device_error_word();
   const bool promote = p.gA_group || p.gB_block;
   const int grid = std::max(1, std::min(p.tiles, device_sm_count()));
@@ -904,6 +940,23 @@ cudaError_t launch_gemm(const uint8_t* A, const float* sA, int gA, const uint8_t
     }
     return launch_pdl(k_gemm<false>, dim3(grid), dim3(kThreads), kSmemBytes, st, mA, mB, p);
   }
+}
+
+cudaError_t launch_gemm(const uint8_t* A, const float* sA, int gA, const uint8_t* B, bool b_packed, const float* sB,
+                        int gB, int64_t M, int64_t N, int64_t K, uint16_t* C, void* ws, size_t ws_bytes,
+                        cudaStream_t st) {
+  if (M == 0 || N == 0) return cudaSuccess;
+  const DecodePlan plan = decode_plan(M, N, K);
+  if (plan.mp > 0) return launch_decode_gemm(plan, A, sA, gA, B, b_packed, sB, gB, M, N, K, C, ws, ws_bytes, st);
+  return launch_prefill(A, sA, gA, B, b_packed, sB, gB, M, N, K, C, nullptr, nullptr, st);
+}
+
+cudaError_t launch_gemm_to_fp8(const uint8_t* A, const float* sA, int gA, const uint8_t* B, bool b_packed,
+                               const float* sB, int gB, int64_t M, int64_t N, int64_t K, uint8_t* codes,
+                               float* scales, cudaStream_t st) {
+  if (M == 0 || N == 0) return cudaSuccess;
+  if (decode_plan(M, N, K).mp > 0) return cudaErrorNotSupported;   // the decode kernel has no such epilogue
+  return launch_prefill(A, sA, gA, B, b_packed, sB, gB, M, N, K, nullptr, codes, scales, st);
 }
 
 // Linear layer with dynamic activation quantization: C = GEMM(quantize_1x128_E4M3(X), B), as the

@@ -119,6 +119,12 @@ cudaError_t launch_count_underflow(const uint16_t* x, const uint8_t* codes, int6
 cudaError_t launch_pack_b_tiles(const uint8_t* B, int64_t N, int64_t K, uint8_t* packed, cudaStream_t st);
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
+// the same GEMM (prefill shapes, M > 64) with C quantized in the epilogue to E4M3 1x128 groups:
+// codes [M][N], scales [N/128][M]; cudaErrorNotSupported for decode shapes
+cudaError_t launch_gemm_to_fp8(const uint8_t* A, const float* sA, int gA, const uint8_t* B, bool b_packed,
+                               const float* sB, int gB, int64_t M, int64_t N, int64_t K, uint8_t* codes,
+                               float* scales, cudaStream_t st);
+
 // MXFP8 GEMM on the block-scaled MMA: A [M][K], B [N][K] codes (formats fa, fb), scales in the
 // blocked layout; N % 128 == 0, K % 128 == 0
 cudaError_t launch_gemm_mx(const uint8_t* A, const uint8_t* sfa, int fa, const uint8_t* B, const uint8_t* sfb, int fb,

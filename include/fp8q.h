@@ -365,6 +365,24 @@ FP8Q_API fp8q_status fp8_count_underflow(const void *x, const uint8_t *codes, in
                                          unsigned long long *count, fp8q_stream_t stream);
 
 /*
+ * The block-scaled GEMM with its output quantized for the next layer ([W] "激活动态量化": the
+ * next GEMM's activations in 1x128 groups): the epilogue rounds each output to bf16, as
+ * fp8_gemm_blockscaled stores it, and quantizes every 1x128 group of C to E4M3 in place of the
+ * bf16 store, so C never round-trips through memory.  codes and scales are bit-identical to
+ * fp8_gemm_blockscaled followed by fp8_quantize(C, FP8Q_E4M3, FP8Q_GROUP_1x128).
+ *   A, sA, gA, B, sB, gB, M, N, K  as fp8_gemm_blockscaled
+ *   codes   uint8 [M][N] (device, 16-byte aligned, written)
+ *   scales  fp32 [N/128][M] (device, written): the 1x128 layout of fp8_quantize
+ * Prefill shapes only: M must exceed 64 (decode shapes, which fp8q_gemm_workspace_bytes gives a
+ * workspace, return FP8Q_ERR_UNSUPPORTED: quantize their bf16 output with fp8_quantize).  No
+ * workspace.
+ */
+FP8Q_API fp8q_status fp8_gemm_blockscaled_to_fp8(const uint8_t *A, const float *sA, fp8q_granularity gA,
+                                                 const uint8_t *B, const float *sB, fp8q_granularity gB,
+                                                 int64_t M, int64_t N, int64_t K, uint8_t *codes, float *scales,
+                                                 fp8q_stream_t stream);
+
+/*
  * Packed weight tiles for the GEMMs.  Repacks B codes [N][K] (row-major, K-major rows) so
  * that each 128 x 128 tile is one contiguous 16384-byte block: tile (nb, kb) = rows
  * [128 nb, +128) x columns [128 kb, +128) starts at byte 16384 * (nb * K/128 + kb); inside it

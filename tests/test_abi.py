@@ -207,3 +207,14 @@ def test_quantize_many_rejects(L):
     assert L.fp8_quantize_many(arr, 1, 0, None) == 1                  # x not 16-byte aligned
     arr[0] = fq._QuantTensor(None, 0, 128, 1, None, None)
     assert L.fp8_quantize_many(arr, 1, 0, None) == 0                  # empty
+
+
+@host_only
+def test_gemm_to_fp8_rejects(L):
+    a, m = ALIGNED, MISALIGNED
+    # (A, sA, gA, B, sB, gB, M, N, K, codes, scales, stream)
+    assert L.fp8_gemm_blockscaled_to_fp8(a, a, 1, a, a, 2, 16, 256, 256, a, a, None) == 2     # decode shape
+    assert L.fp8_gemm_blockscaled_to_fp8(a, a, 1, a, a, 2, 256, 200, 256, a, a, None) == 2    # N % 128
+    assert L.fp8_gemm_blockscaled_to_fp8(a, a, 1, a, a, 2, 256, 256, 256, m, a, None) == 1    # codes alignment
+    assert L.fp8_gemm_blockscaled_to_fp8(a, a, 3, a, a, 2, 256, 256, 256, a, a, None) == 1    # gA
+    assert L.fp8_gemm_blockscaled_to_fp8(a, a, 1, a, a, 2, 256, 256, 256, a, None, None) == 1  # scales

@@ -246,3 +246,35 @@ def test_packed_gemm_against_oracle(orc):
     got = fq.fp8_gemm_blockscaled_packed(dev(a), dev(sa), dev(orc.pack_b_tiles(b)), dev(sb), N)
     torch.cuda.synchronize()
     check_tolerance(host(got), orc.gemm_rows(a, sa, 1, b, sb, 2, np.arange(M)), "packed")
+
+
+# ---------------------------------------------------------------- C quantized in the epilogue
+
+@pytest.mark.parametrize("ga,gb", [(1, 2), (0, 0)])
+@pytest.mark.parametrize("shape", [(65, 128, 128), (130, 384, 512), (300, 512, 384), (8192, 14336, 4096)])
+def test_gemm_to_fp8_matches_two_steps(orc, ga, gb, shape):
+    """Codes and scales equal fp8_gemm_blockscaled followed by fp8_quantize(C, E4M3, 1x128)."""
+    M, N, K = shape
+    a, sa, b, sb = operands(orc, M, N, K, ga, gb, seed=M + N + K + 3)
+    A, SA, B, SB = dev(a), dev(sa), dev(b), dev(sb)
+    codes, scales = fq.fp8_gemm_blockscaled_to_fp8(A, SA, B, SB, ga, gb)
+    c = fq.fp8_gemm_blockscaled(A, SA, B, SB, ga, gb)
+    c2, s2 = fq.fp8_quantize(c, fq.E4M3, fq.GROUP_1x128)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(codes), host(c2))
+    assert np.array_equal(host(scales).view(np.uint32), host(s2).view(np.uint32))
+
+
+def test_gemm_to_fp8_against_oracle_product(orc):
+    """Dequantized output within FP8 rounding (half a step, relative 2^-4) of the fp64 product."""
+    M, N, K = 200, 384, 640
+    a, sa, b, sb = operands(orc, M, N, K, 1, 2, seed=51)
+    codes, scales = fq.fp8_gemm_blockscaled_to_fp8(dev(a), dev(sa), dev(b), dev(sb))
+    torch.cuda.synchronize()
+    # decoded with torch's float8 type (not the oracle: no CUDA output becomes an oracle input)
+    dec = torch.from_numpy(host(codes)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    s_full = np.repeat(host(scales).T, 128, axis=1)[:, :N].astype(np.float64)
+    got = dec * s_full
+    ref = orc.gemm_rows(a, sa, 1, b, sb, 2, np.arange(M))
+    bound = np.abs(ref) * (2.0 ** -4 + 2.0 ** -8 + ELEM) + s_full * 2.0 ** -9 + 1e-2 * 1e-2
+    assert np.all(np.abs(got - ref) <= bound)
