@@ -307,8 +307,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_mx(const __grid_constant__
       if (m < p.M && ncol0 < p.N) {
         uint16_t* dst = p.C + (size_t)m * p.N + ncol0;
 #pragma unroll
-        for (int c = 0; c < 16; ++c)
-          st_stream_v4(dst + c * 8, make_uint4(out[c * 4], out[c * 4 + 1], out[c * 4 + 2], out[c * 4 + 3]));
+        for (int c = 0; c < 8; ++c)   // 32-byte stores: every store fills whole sectors
+          st_stream_v8(dst + c * 16, make_uint4(out[c * 8], out[c * 8 + 1], out[c * 8 + 2], out[c * 8 + 3]),
+                       make_uint4(out[c * 8 + 4], out[c * 8 + 5], out[c * 8 + 6], out[c * 8 + 7]));
       }
     }
   }

@@ -363,13 +363,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ CU
             } else {
               uint16_t* dst = p.C + (size_t)m * p.N + ncol0;
 #pragma unroll
-              for (int c = 0; c < 16; ++c) {
-                uint4 wv;
-                wv.x = f32x2_to_bf16x2(acc[c * 4 + 0].x, acc[c * 4 + 0].y);
-                wv.y = f32x2_to_bf16x2(acc[c * 4 + 1].x, acc[c * 4 + 1].y);
-                wv.z = f32x2_to_bf16x2(acc[c * 4 + 2].x, acc[c * 4 + 2].y);
-                wv.w = f32x2_to_bf16x2(acc[c * 4 + 3].x, acc[c * 4 + 3].y);
-                st_stream_v4(dst + c * 8, wv);
+              for (int c = 0; c < 8; ++c) {   // 32-byte stores: every store fills whole sectors
+                uint4 lo, hi;
+                lo.x = f32x2_to_bf16x2(acc[c * 8 + 0].x, acc[c * 8 + 0].y);
+                lo.y = f32x2_to_bf16x2(acc[c * 8 + 1].x, acc[c * 8 + 1].y);
+                lo.z = f32x2_to_bf16x2(acc[c * 8 + 2].x, acc[c * 8 + 2].y);
+                lo.w = f32x2_to_bf16x2(acc[c * 8 + 3].x, acc[c * 8 + 3].y);
+                hi.x = f32x2_to_bf16x2(acc[c * 8 + 4].x, acc[c * 8 + 4].y);
+                hi.y = f32x2_to_bf16x2(acc[c * 8 + 5].x, acc[c * 8 + 5].y);
+                hi.z = f32x2_to_bf16x2(acc[c * 8 + 6].x, acc[c * 8 + 6].y);
+                hi.w = f32x2_to_bf16x2(acc[c * 8 + 7].x, acc[c * 8 + 7].y);
+                st_stream_v8(dst + c * 16, lo, hi);
               }
             }
           }
@@ -409,8 +413,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ CU
           } else {
             uint16_t* dst = p.C + (size_t)m * p.N + ncol0;
 #pragma unroll
-            for (int c = 0; c < 16; ++c)
-              st_stream_v4(dst + c * 8, make_uint4(out[c * 4], out[c * 4 + 1], out[c * 4 + 2], out[c * 4 + 3]));
+            for (int c = 0; c < 8; ++c)   // 32-byte stores: every store fills whole sectors
+              st_stream_v8(dst + c * 16, make_uint4(out[c * 8], out[c * 8 + 1], out[c * 8 + 2], out[c * 8 + 3]),
+                           make_uint4(out[c * 8 + 4], out[c * 8 + 5], out[c * 8 + 6], out[c * 8 + 7]));
           }
         }
       }
