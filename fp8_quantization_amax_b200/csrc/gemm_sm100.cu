@@ -82,25 +82,32 @@ struct Params {
   uint32_t* err;
 };
 
-// The 1x128 E4M3 quantizer on one 128-column row segment of C held by one thread as 64 packed
-// bf16 pairs (the values a bf16 C would store): the group's amax, its scale, the codes and the
-// scale, with the arithmetic of the stand-alone quantizer, so the result equals quantizing the
-// bf16 C in a second pass.
-__device__ __forceinline__ void store_row_e4m3(const uint32_t (&w)[64], uint8_t* codes_row, float* scale) {
+// The 1x128 E4M3 quantizer on one 128-column row segment of C held by one thread; pair(i) gives
+// the segment's bf16 pair i (0..63), the values a bf16 C would store: the group's amax, its
+// scale, the codes and the scale, with the arithmetic of the stand-alone quantizer, so the
+// result equals quantizing the bf16 C in a second pass.
+template <class PairFn>
+__device__ __forceinline__ void store_row_e4m3(PairFn pair, uint8_t* codes_row, float* scale) {
   uint32_t m = 0u;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) m = absmax_v4(m, make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]));
+  for (int i = 0; i < 16; ++i) m = absmax_v4(m, make_uint4(pair(4 * i), pair(4 * i + 1), pair(4 * i + 2), pair(4 * i + 3)));
   const GroupScale gs = make_group_scale<kE4M3>(packed_amax_to_f32(m));
+  if (gs.fast) {
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const uint4 a = make_uint4(w[8 * c], w[8 * c + 1], w[8 * c + 2], w[8 * c + 3]);
-    const uint4 b = make_uint4(w[8 * c + 4], w[8 * c + 5], w[8 * c + 6], w[8 * c + 7]);
-    if (gs.fast) {
-      st_stream_v4(codes_row + 16 * c, quant16_fast<kE4M3>(a, b, gs.d, gs.r));
-    } else {
-      st_stream_v2(codes_row + 16 * c, quant8<kE4M3>(a, gs));
-      st_stream_v2(codes_row + 16 * c + 8, quant8<kE4M3>(b, gs));
+    for (int c = 0; c < 4; ++c) {   // 32 codes per 32-byte store
+      const uint4 q0 = quant16_fast<kE4M3>(make_uint4(pair(16 * c), pair(16 * c + 1), pair(16 * c + 2), pair(16 * c + 3)),
+                                           make_uint4(pair(16 * c + 4), pair(16 * c + 5), pair(16 * c + 6), pair(16 * c + 7)),
+                                           gs.d, gs.r);
+      const uint4 q1 =
+          quant16_fast<kE4M3>(make_uint4(pair(16 * c + 8), pair(16 * c + 9), pair(16 * c + 10), pair(16 * c + 11)),
+                              make_uint4(pair(16 * c + 12), pair(16 * c + 13), pair(16 * c + 14), pair(16 * c + 15)),
+                              gs.d, gs.r);
+      st_stream_v8(codes_row + 32 * c, q0, q1);
     }
+  } else {
+#pragma unroll
+    for (int c = 0; c < 16; ++c)
+      st_stream_v2(codes_row + 8 * c, quant8<kE4M3>(make_uint4(pair(4 * c), pair(4 * c + 1), pair(4 * c + 2), pair(4 * c + 3)), gs));
   }
   *scale = gs.s;
 }
@@ -356,10 +363,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ CU
           const int ncol0 = n0 + half * 128;
           if (m < p.M && ncol0 < p.N) {
             if (p.q_codes) {
-              uint32_t w[64];
-#pragma unroll
-              for (int i = 0; i < 64; ++i) w[i] = f32x2_to_bf16x2(acc[i].x, acc[i].y);
-              store_row_e4m3(w, p.q_codes + (size_t)m * p.N + ncol0, p.q_scales + (size_t)(ncol0 >> 7) * p.M + m);
+              store_row_e4m3([&](int i) { return f32x2_to_bf16x2(acc[i].x, acc[i].y); },
+                             p.q_codes + (size_t)m * p.N + ncol0, p.q_scales + (size_t)(ncol0 >> 7) * p.M + m);
             } else {
               uint16_t* dst = p.C + (size_t)m * p.N + ncol0;
 #pragma unroll
@@ -409,7 +414,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ CU
         ++acc_use;
         if (m < p.M && ncol0 < p.N) {
           if (p.q_codes) {
-            store_row_e4m3(out, p.q_codes + (size_t)m * p.N + ncol0, p.q_scales + (size_t)(ncol0 >> 7) * p.M + m);
+            store_row_e4m3([&](int i) { return out[i]; }, p.q_codes + (size_t)m * p.N + ncol0,
+                           p.q_scales + (size_t)(ncol0 >> 7) * p.M + m);
           } else {
             uint16_t* dst = p.C + (size_t)m * p.N + ncol0;
 #pragma unroll
