@@ -449,16 +449,19 @@ constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + (2 * kStages + 4) *
 // contiguously over all CTAs (a CTA's range may cross tile boundaries); each CTA promotes its
 // units per K block (acc[m] += sB[tile][kb] * sA[kb][m] * P^T[n][m], thread = weight row n).
 // A tile that lies wholly in one CTA's range is rounded to bf16 and stored directly.  A tile
-// shared by several CTAs: each writes its fp32 partial to the workspace and counts itself in on
-// the tile's counter; the CTA that completes the count adds the partials in ascending CTA order
-// (deterministic: the same sum whichever CTA finishes last), stores the tile, and clears the
-// partials and the counter, so every completed call leaves the whole workspace zero.
+// shared by several CTAs is finished by the CTA that started it (the lowest contributor, for
+// which it is the last segment of its range): every later contributor writes its fp32 partial
+// to the workspace and counts itself in on the tile's counter without waiting (for them it is
+// the first segment, done early in their run); the first contributor's reducer warp polls the
+// counter while its units stream, then its promotion warps add the other partials to their own
+// in ascending CTA order (deterministic), store the tile, and clear the partials and the
+// counter, so every completed call leaves the whole workspace zero.
 //   warp 0 TMA producer, warp 1 MMA issuer (four TMEM buffers), warp 2 scale producer,
-//   warps 3-6 promotion.
+//   warps 3-6 promotion, warp 7 split-tile bookkeeping.
 namespace dec {
 
 constexpr int BM = 128;                 // weight rows per tile (the MMA's M)
-constexpr int kThreads = 32 * 7;
+constexpr int kThreads = 32 * 8;
 constexpr int kTBuf = 4;                // TMEM buffers of kMaxMp columns
 constexpr int kMaxMp = 64;
 constexpr uint32_t kTmemCols = kTBuf * kMaxMp;
@@ -503,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
   __shared__ float sc_b[kScaleSlots];
   __shared__ uint64_t bars[2 * kMaxStages + 2 * kTBuf + 2 * kScaleSlots + 2];
   __shared__ uint32_t tmem_slot;
-  __shared__ uint32_t s_last;
+  __shared__ uint32_t s_fin_ok;
   uint8_t* smem = smem_raw + (((smem_u32(smem_raw) + 1023u) & ~1023u) - smem_u32(smem_raw));
   const int S = p.stages;
   uint64_t* full = bars;
@@ -513,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
   uint64_t* sfull = tempty + kTBuf;
   uint64_t* sempty = sfull + kScaleSlots;
   uint64_t* seg_written = sempty + kScaleSlots;   // the four promotion warps' partials are out
-  uint64_t* seg_decided = seg_written + 1;        // the tile's counter has been bumped
+  uint64_t* fin_ready = seg_written + 1;          // every later contributor of the last tile is in
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t lo = range_lo(blockIdx.x, p.W, p.G), hi = range_lo(blockIdx.x + 1, p.W, p.G);
   const uint32_t n_units = hi - lo;
@@ -533,7 +536,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
   }
   if (threadIdx.x == 0) {
     mbar_init(seg_written, 4);
-    mbar_init(seg_decided, 1);
+    mbar_init(fin_ready, 1);
     for (int i = 0; i < S; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
@@ -642,6 +645,47 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
       }
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
+  } else if (warp == 7) {
+    // reducer: the split-tile bookkeeping, off the promotion warps' path.  A CTA's range holds at
+    // most one segment of a tile a lower CTA started (its first: the partial is counted in here)
+    // and at most one segment of a tile it starts but a higher CTA ends (its last: this CTA adds
+    // the others' partials to its own, once all of them are counted in).
+    if (lane == 0 && n_units > 0) {
+      const uint32_t t0 = lo / nkb, t1 = (hi - 1) / nkb;
+      if (lo % nkb != 0) {
+        const uint32_t c_first = cta_of(t0 * nkb, p.W, p.G), c_last = cta_of(t0 * nkb + nkb - 1, p.W, p.G);
+        // the promotion warps hand their partial writes over through the mbarrier (release /
+        // acquire at CTA scope); this gpu-scope fence then orders all of them (cumulatively)
+        // before the count
+        if (mbar_wait(seg_written, 0, p.err)) {
+          __threadfence();
+          const uint32_t old = atomicAdd(p.counters + t0, 1u);
+          if (old >= c_last - c_first) raise_device_error(p.err, kErrWorkspaceDirty);
+        }
+      }
+      if ((t1 > t0 || lo % nkb == 0) && hi % nkb != 0) {
+        // polled from the start, so the wait is normally over before the last unit is promoted
+        const uint32_t need = cta_of(t1 * nkb + nkb - 1, p.W, p.G) - blockIdx.x;
+        const uint64_t t_start = globaltimer_ns();
+        uint32_t v = 0;
+        bool timed_out = false;
+        for (;;) {
+          asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p.counters + t1) : "memory");
+          if (v >= need) break;
+          if (globaltimer_ns() - t_start > kWaitLimitNs) {
+            raise_device_error(p.err, kErrWaitTimeout);
+            timed_out = true;
+            break;
+          }
+          __nanosleep(128);
+        }
+        const bool ok = !timed_out && v == need;
+        if (!timed_out && v > need) raise_device_error(p.err, kErrWorkspaceDirty);
+        if (ok) p.counters[t1] = 0;   // every later contributor has counted in: leave it zero
+        s_fin_ok = ok ? 1u : 0u;
+        mbar_arrive(fin_ready);
+      }
+    }
   } else {
     // promotion: thread = weight row (TMEM lane) of the tile, MP accumulators (one per token)
     const int quarter = warp & 3;
@@ -650,7 +694,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
     float acc[MP];
 #pragma unroll
     for (int m = 0; m < MP; ++m) acc[m] = 0.0f;
-    uint32_t r = 0, sph = 0, seg_k = 0;
+    uint32_t r = 0, sph = 0;
     const uint32_t first_tile = lo / nkb;
     // Units are taken in pairs when the next unit belongs to the same tile: one round of waits,
     // both partials loaded before one tcgen05.wait, applied in unit order (the same fp32 sums as
@@ -728,47 +772,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
         // this CTA's segment of tile t ends
         const uint32_t c_first = cta_of(t * nkb, p.W, p.G), c_last = cta_of(t * nkb + nkb - 1, p.W, p.G);
         bool finish = c_first == c_last;   // the whole tile is this CTA's
-        if (!finish) {
-          // publish this row's partial ([m][row] layout, coalesced over rows), then count the
-          // segment in; the CTA that brings the count to the number of contributors adds them up
+        if (!finish && blockIdx.x != c_first) {
+          // a lower CTA started the tile: publish this row's partial ([m][row] layout, coalesced
+          // over rows) and hand it to the reducer warp, which counts it in; nothing to wait for
           float* dst = p.partials + ((size_t)(blockIdx.x * p.maxseg + (t - first_tile)) * MP) * BM + row;
 #pragma unroll
           for (int m = 0; m < MP; ++m) dst[(size_t)m * BM] = acc[m];
-          // the four warps hand their writes to one thread through the mbarrier (release /
-          // acquire at CTA scope); its gpu-scope fence then orders all of them (cumulatively)
-          // before its atomic, so no per-thread fence is needed
           __syncwarp();
           if (lane == 0) mbar_arrive(seg_written);
-          if (warp == 3 && lane == 0) {
-            const bool ok = mbar_wait(seg_written, seg_k & 1u, p.err);
-            uint32_t last = 0;
-            if (ok) {
-              __threadfence();
-              const uint32_t n_contrib = c_last - c_first + 1;
-              const uint32_t old = atomicAdd(p.counters + t, 1u);
-              if (old >= n_contrib) raise_device_error(p.err, kErrWorkspaceDirty);
-              last = old + 1 == n_contrib;
-              if (last) {
-                __threadfence();           // acquire: the other contributors' partials
-                p.counters[t] = 0;         // every contributor has counted in: leave it zero
-              }
-            }
-            s_last = last;
-            mbar_arrive(seg_decided);
-          }
-          if (!mbar_wait(seg_decided, seg_k & 1u, p.err)) break;
-          ++seg_k;
-          finish = s_last != 0;
+        } else if (!finish) {
+          // this CTA started the tile and a higher one ends it (always this CTA's last segment):
+          // once the reducer has seen every later contributor counted in, add their partials to
+          // this row in ascending CTA order (the same order whichever CTA is slower, so reruns
+          // are bit-identical), and clear them, so that a completed call leaves the workspace zero
+          if (!mbar_wait(fin_ready, 0, p.err)) break;
+          finish = s_fin_ok != 0;
           if (finish) {
-            // sum the tile's partials in ascending CTA order (this CTA's own included: each
-            // thread re-reads the row it wrote), so the result does not depend on which CTA
-            // finishes last; then clear them, so that a completed call leaves the whole
-            // workspace zero whatever the shape of the next call that reuses it
             __threadfence();
-#pragma unroll
-            for (int m = 0; m < MP; ++m) acc[m] = 0.0f;
 #pragma unroll 1
-            for (uint32_t c = c_first; c <= c_last; ++c) {
+            for (uint32_t c = c_first + 1; c <= c_last; ++c) {
               const uint32_t clo = range_lo(c, p.W, p.G);
               float* src = p.partials + ((size_t)(c * (uint32_t)p.maxseg + (t - clo / nkb)) * MP) * BM + row;
 #pragma unroll
