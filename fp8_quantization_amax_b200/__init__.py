@@ -10,6 +10,7 @@ allocated with torch.empty.  There is no CPU path: CPU tensors and a missing lib
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 import threading
 
@@ -57,6 +58,8 @@ def library_path() -> str:
 def lib() -> ctypes.CDLL:
     """The loaded libfp8q.so with argument types set.  Raises if it has not been built."""
     global _lib
+    if _lib is not None:
+        return _lib
     with _lock:
         if _lib is None:
             if not os.path.exists(_LIB_PATH):
@@ -163,6 +166,7 @@ def kv_workspace_bytes(tokens: int, heads: int, head_dim: int, gran: int) -> int
     return int(lib().fp8q_kv_workspace_bytes(tokens, heads, head_dim, gran))
 
 
+@functools.lru_cache(maxsize=256)
 def gemm_workspace_bytes(M: int, N: int, K: int) -> int:
     return int(lib().fp8q_gemm_workspace_bytes(M, N, K))
 
@@ -201,8 +205,19 @@ def _ptr(t: torch.Tensor | None):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
+def _stream_handle(device) -> int:
+    """The raw cudaStream_t of the current stream on `device` (the per-call host cost matters
+    for decode-sized launches, so the direct lookup is used when torch provides it)."""
+    if _raw_stream is not None:
+        return _raw_stream(device.index if device.index is not None else torch.cuda.current_device())
+    return torch.cuda.current_stream(device).cuda_stream
+
+
 def _stream(device) -> ctypes.c_void_p:
-    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    return ctypes.c_void_p(_stream_handle(device))
 
 
 def _workspace(nbytes: int, device, ws: torch.Tensor | None) -> torch.Tensor | None:
@@ -218,10 +233,10 @@ def _workspace(nbytes: int, device, ws: torch.Tensor | None) -> torch.Tensor | N
 _gemm_ws: dict = {}
 
 
-def _gemm_workspace(nbytes: int, device) -> torch.Tensor | None:
+def _gemm_workspace(nbytes: int, device, stream: int) -> torch.Tensor | None:
     if nbytes == 0:
         return None
-    key = (device.index, torch.cuda.current_stream(device).cuda_stream)
+    key = (device.index, stream)
     buf = _gemm_ws.get(key)
     if buf is None or buf.numel() < nbytes:
         buf = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
@@ -411,11 +426,12 @@ def fp8_gemm_blockscaled(a: torch.Tensor, sa: torch.Tensor, b: torch.Tensor, sb:
         raise ValueError("a and b disagree on K")
     out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device) if out is None else _dev(out, "out", torch.bfloat16)
     need = gemm_workspace_bytes(M, N, K)
+    stream = _stream_handle(a.device)
     cached = ws is None
     if cached:
-        ws = _gemm_workspace(need, a.device)
+        ws = _gemm_workspace(need, a.device, stream)
     st = lib().fp8_gemm_blockscaled(_ptr(a), _ptr(sa), ga, _ptr(b), _ptr(sb), gb, M, N, K, _ptr(out), _ptr(ws),
-                                    0 if ws is None else ws.numel() * ws.element_size(), _stream(a.device))
+                                    0 if ws is None else ws.numel() * ws.element_size(), ctypes.c_void_p(stream))
     if st != 0 and cached:
         _gemm_ws.clear()
     _check("fp8_gemm_blockscaled", st)
@@ -471,12 +487,13 @@ def fp8_gemm_blockscaled_packed(a: torch.Tensor, sa: torch.Tensor, bp: torch.Ten
         raise ValueError("bp holds fewer than N * K bytes")
     out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device) if out is None else _dev(out, "out", torch.bfloat16)
     need = gemm_workspace_bytes(M, N, K)
+    stream = _stream_handle(a.device)
     cached = ws is None
     if cached:
-        ws = _gemm_workspace(need, a.device)
+        ws = _gemm_workspace(need, a.device, stream)
     st = lib().fp8_gemm_blockscaled_packed(_ptr(a), _ptr(sa), ga, _ptr(bp), _ptr(sb), gb, M, N, K, _ptr(out),
                                            _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
-                                           _stream(a.device))
+                                           ctypes.c_void_p(stream))
     if st != 0 and cached:
         _gemm_ws.clear()
     _check("fp8_gemm_blockscaled_packed", st)
@@ -562,12 +579,13 @@ def fp8_linear_dynamic(x: torch.Tensor, b: torch.Tensor, sb: torch.Tensor, gb: i
         raise ValueError("x and b disagree on K")
     out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if out is None else _dev(out, "out", torch.bfloat16)
     act_ws = _workspace(linear_act_workspace_bytes(M, K), x.device, act_ws)
+    stream = _stream_handle(x.device)
     cached = ws is None
     if cached:
-        ws = _gemm_workspace(gemm_workspace_bytes(M, N, K), x.device)
+        ws = _gemm_workspace(gemm_workspace_bytes(M, N, K), x.device, stream)
     st = lib().fp8_linear_dynamic(_ptr(x), M, N, K, _ptr(b), _ptr(sb), gb, _ptr(out), _ptr(act_ws),
                                   0 if act_ws is None else act_ws.numel() * act_ws.element_size(), _ptr(ws),
-                                  0 if ws is None else ws.numel() * ws.element_size(), _stream(x.device))
+                                  0 if ws is None else ws.numel() * ws.element_size(), ctypes.c_void_p(stream))
     if st != 0 and cached:
         _gemm_ws.clear()
     _check("fp8_linear_dynamic", st)

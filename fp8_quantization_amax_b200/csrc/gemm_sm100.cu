@@ -842,7 +842,7 @@ struct DecodePlan {
   size_t ws_bytes = 0, counter_bytes = 0;
 };
 
-DecodePlan decode_plan(int64_t M, int64_t N, int64_t K) {
+DecodePlan decode_plan_uncached(int64_t M, int64_t N, int64_t K) {
   DecodePlan d;
   if (M <= 0 || M > gemm::dec::kMaxMp || N % 128 != 0 || K % 128 != 0 || N == 0 || K == 0) return d;
   d.mp = (int)((M + 15) / 16 * 16);
@@ -857,6 +857,26 @@ DecodePlan decode_plan(int64_t M, int64_t N, int64_t K) {
   d.counter_bytes = ((size_t)tiles * sizeof(uint32_t) + 255) / 256 * 256;
   d.ws_bytes = d.counter_bytes + (size_t)d.G * d.maxseg * d.mp * gemm::dec::BM * sizeof(float);
   return d;
+}
+
+// The plan walks every CTA's range; a decode step asks for the same few shapes on every call
+// (once for the workspace size, once to launch), so the last plan is kept per host thread.
+DecodePlan decode_plan(int64_t M, int64_t N, int64_t K) {
+  struct Entry {
+    int64_t M = -1, N = -1, K = -1;
+    int sms = -1;
+    DecodePlan plan;
+  };
+  thread_local Entry last;
+  const int sms = device_sm_count();
+  if (last.M != M || last.N != N || last.K != K || last.sms != sms) {
+    last.plan = decode_plan_uncached(M, N, K);
+    last.M = M;
+    last.N = N;
+    last.K = K;
+    last.sms = sms;
+  }
+  return last.plan;
 }
 
 template <int MP>
