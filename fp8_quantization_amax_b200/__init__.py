@@ -90,6 +90,8 @@ def lib() -> ctypes.CDLL:
             L.fp8_pack_b_tiles.argtypes = [vp, i64, i64, vp, vp]
             L.fp8_scale_histogram.argtypes = [vp, i64, i32, vp, vp]
             L.fp8q_selftest_wait_timeout.argtypes = [vp]
+            L.fp8q_check_decode_split.argtypes = [i64, i64, i64, i32]
+            L.fp8q_check_decode_split.restype = i32
             L.fp8_gemm_blockscaled_to_fp8.argtypes = [vp, vp, i32, vp, vp, i32, i64, i64, i64, vp, vp, vp]
             L.fp8_gemm_blockscaled_to_fp8.restype = i32
             L.fp8q_selftest_wait_timeout.restype = i32
@@ -505,6 +507,13 @@ def selftest_wait_timeout(device=None) -> None:
     barrier nothing completes gives up after its time limit and sets bit 0 of device_status()."""
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     _check("fp8q_selftest_wait_timeout", lib().fp8q_selftest_wait_timeout(_stream(dev)))
+
+
+def check_decode_split(M: int, N: int, K: int, sms: int) -> int:
+    """Host-only self-check of the decode GEMM's work split for a device with `sms` SMs (no GPU
+    needed): 0 when its split-tile hand-off invariants hold, else the code of the first violation
+    (-1: not a decode shape).  See fp8q_check_decode_split in include/fp8q.h."""
+    return int(lib().fp8q_check_decode_split(M, N, K, sms))
 
 
 def fp8_quantize_many(jobs, fmt: int = E4M3):

@@ -57,6 +57,10 @@ fp8q_status fp8q_selftest_wait_timeout(fp8q_stream_t stream) {
   return from_cuda(fp8q::launch_selftest_wait((cudaStream_t)stream));
 }
 
+int fp8q_check_decode_split(int64_t M, int64_t N, int64_t K, int sms) {
+  return fp8q::check_decode_split(M, N, K, sms);
+}
+
 size_t fp8q_num_scales(int64_t rows, int64_t cols, fp8q_granularity g) {
   if (rows < 0 || cols < 0 || !valid_gran(g)) return 0;
   if (g == FP8Q_PER_TENSOR) return 1;

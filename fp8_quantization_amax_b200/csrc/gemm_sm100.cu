@@ -30,6 +30,7 @@
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
+#include <vector>
 
 #include "fp8q_device.cuh"
 #include "internal.h"
@@ -489,6 +490,15 @@ struct Params {
 // first unit of CTA c when W units are split over G CTAs (W * G < 2^32, checked by the planner)
 __host__ __device__ __forceinline__ uint32_t range_lo(uint32_t c, uint32_t W, uint32_t G) { return (c * W) / G; }
 
+// A range's first segment adds to a tile that a lower CTA started when the range does not begin
+// on a tile boundary; its last segment starts a tile that a higher CTA ends when the range holds
+// that tile's first unit but not its last.  (The split-tile hand-off relies on these being the
+// only shared segments of a range; fp8q_check_decode_split verifies it.)
+__host__ __device__ __forceinline__ bool first_seg_adds_to_lower(uint32_t lo, uint32_t nkb) { return lo % nkb != 0; }
+__host__ __device__ __forceinline__ bool last_seg_finishes_shared(uint32_t lo, uint32_t hi, uint32_t nkb) {
+  return (lo <= ((hi - 1) / nkb) * nkb) && hi % nkb != 0;
+}
+
 // the CTA whose range holds unit u
 __host__ __device__ __forceinline__ uint32_t cta_of(uint32_t u, uint32_t W, uint32_t G) {
   uint32_t c = (u * G) / W;
@@ -652,7 +662,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
     // the others' partials to its own, once all of them are counted in).
     if (lane == 0 && n_units > 0) {
       const uint32_t t0 = lo / nkb, t1 = (hi - 1) / nkb;
-      if (lo % nkb != 0) {
+      if (first_seg_adds_to_lower(lo, nkb)) {
         const uint32_t c_first = cta_of(t0 * nkb, p.W, p.G), c_last = cta_of(t0 * nkb + nkb - 1, p.W, p.G);
         // the promotion warps hand their partial writes over through the mbarrier (release /
         // acquire at CTA scope); this gpu-scope fence then orders all of them (cumulatively)
@@ -663,7 +673,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
           if (old >= c_last - c_first) raise_device_error(p.err, kErrWorkspaceDirty);
         }
       }
-      if ((t1 > t0 || lo % nkb == 0) && hi % nkb != 0) {
+      if (last_seg_finishes_shared(lo, hi, nkb)) {
         // polled from the start, so the wait is normally over before the last unit is promoted
         const uint32_t need = cta_of(t1 * nkb + nkb - 1, p.W, p.G) - blockIdx.x;
         const uint64_t t_start = globaltimer_ns();
@@ -947,6 +957,59 @@ cudaError_t launch_decode_gemm(const DecodePlan& plan, const uint8_t* A, const f
 }  // namespace
 
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) { return decode_plan(M, N, K).ws_bytes; }
+
+// The invariants of the decode kernel's split-tile hand-off, checked on the host with the
+// kernel's own range functions (see fp8q_check_decode_split in fp8q.h for the list).
+int check_decode_split(int64_t M, int64_t N, int64_t K, int sms) {
+  using gemm::dec::cta_of;
+  using gemm::dec::range_lo;
+  if (M <= 0 || M > gemm::dec::kMaxMp || N <= 0 || K <= 0 || N % 128 != 0 || K % 128 != 0 || sms <= 0) return -1;
+  const uint32_t nkb = (uint32_t)(K / 128), tiles = (uint32_t)(N / 128);
+  if ((uint64_t)tiles * nkb * (uint64_t)sms >= (1ull << 32)) return -1;
+  const uint32_t W = tiles * nkb, G = std::min<uint32_t>((uint32_t)sms, W);
+  int maxseg = 0;
+  for (uint32_t c = 0; c < G; ++c) {
+    const uint32_t lo = range_lo(c, W, G), hi = range_lo(c + 1, W, G);
+    if (hi <= lo) return 1;                                   // every CTA has work
+    maxseg = std::max<int>(maxseg, (int)((hi - 1) / nkb - lo / nkb + 1));
+  }
+  std::vector<uint32_t> later(tiles, 0), finishers(tiles, 0);
+  for (uint32_t c = 0; c < G; ++c) {
+    const uint32_t lo = range_lo(c, W, G), hi = range_lo(c + 1, W, G);
+    const uint32_t t0 = lo / nkb, t1 = (hi - 1) / nkb;
+    // the bookkeeping warp's view
+    const bool red_later = gemm::dec::first_seg_adds_to_lower(lo, nkb);
+    const bool red_fin = gemm::dec::last_seg_finishes_shared(lo, hi, nkb);
+    // the promotion warps' view, segment by segment
+    int n_later = 0, n_fin = 0;
+    for (uint32_t t = t0; t <= t1; ++t) {
+      const uint32_t c_first = cta_of(t * nkb, W, G), c_last = cta_of(t * nkb + nkb - 1, W, G);
+      if (c_first > c || c_last < c) return 2;                // the range functions disagree
+      if (c_first == c_last) continue;                        // whole tile: stored directly
+      if (c != c_first) {
+        ++n_later;
+        if (t != t0 || !red_later) return 3;                  // only the first segment, seen by both
+        if ((int)(t - t0) >= maxseg) return 4;                // its partial slot is in the workspace
+        ++later[t];
+      } else {
+        ++n_fin;
+        if (t != t1 || !red_fin) return 5;                    // only the last segment, seen by both
+        ++finishers[t];
+      }
+    }
+    if (n_later > 1 || n_fin > 1) return 6;
+    if ((n_later == 1) != red_later || (n_fin == 1) != red_fin) return 7;
+  }
+  for (uint32_t t = 0; t < tiles; ++t) {
+    const uint32_t c_first = cta_of(t * nkb, W, G), c_last = cta_of(t * nkb + nkb - 1, W, G);
+    if (c_first == c_last) {
+      if (later[t] != 0 || finishers[t] != 0) return 8;
+    } else if (finishers[t] != 1 || later[t] != c_last - c_first) {
+      return 9;                                               // one finisher, every other contributor counted once
+    }
+  }
+  return 0;
+}
 
 // the prefill kernel (M > 64): C in bf16, or (q_codes non-null) quantized to E4M3 1x128 groups
 static cudaError_t launch_prefill(const uint8_t* A, const float* sA, int gA, const uint8_t* B, bool b_packed,

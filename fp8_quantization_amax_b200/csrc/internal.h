@@ -118,6 +118,8 @@ cudaError_t launch_count_underflow(const uint16_t* x, const uint8_t* codes, int6
 // a TMA load, tile (nb, kb) at 16384 (nb K/128 + kb)
 cudaError_t launch_pack_b_tiles(const uint8_t* B, int64_t N, int64_t K, uint8_t* packed, cudaStream_t st);
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+// host-only consistency check of the decode split (fp8q_check_decode_split)
+int check_decode_split(int64_t M, int64_t N, int64_t K, int sms);
 
 // the same GEMM (prefill shapes, M > 64) with C quantized in the epilogue to E4M3 1x128 groups:
 // codes [M][N], scales [N/128][M]; cudaErrorNotSupported for decode shapes

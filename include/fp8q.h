@@ -120,6 +120,19 @@ FP8Q_API uint32_t fp8q_device_status(void);
  */
 FP8Q_API fp8q_status fp8q_selftest_wait_timeout(fp8q_stream_t stream);
 
+/*
+ * Host-only self-check of the decode GEMM's work split (no device work, no GPU needed): for the
+ * plan fp8_gemm_blockscaled uses for a decode shape (M <= 64) on a device with `sms` SMs, walks
+ * every CTA's contiguous range of (weight tile, K block) units with the kernel's own range
+ * functions and checks what its split-tile hand-off relies on: each CTA holds at most one
+ * segment of a tile a lower CTA started (its first segment) and at most one of a tile it starts
+ * but a higher CTA ends (its last); the promotion warps and the bookkeeping warp pick out the same
+ * segments; every shared tile has exactly one finishing CTA (its lowest) and c_last - c_first
+ * later contributors; every partial slot lies inside the workspace.  Returns 0 when all hold,
+ * a positive code naming the first violation, or -1 for a shape that is not a decode shape.
+ */
+FP8Q_API int fp8q_check_decode_split(int64_t M, int64_t N, int64_t K, int sms);
+
 /* ---------------------------------------------------------------- sizes */
 
 /* Number of fp32 scales fp8_quantize writes for a [rows][cols] tensor; 0 on a bad argument. */
