@@ -670,7 +670,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
         if (mbar_wait(seg_written, 0, p.err)) {
           __threadfence();
           const uint32_t old = atomicAdd(p.counters + t0, 1u);
-          if (old >= c_last - c_first) raise_device_error(p.err, kErrWorkspaceDirty);
+          if (old >= c_last - c_first) {
+            // a workspace that was not zero: report it and mark the counter (its top bit stays
+            // set however the other adds interleave), so the finishing CTA sees a count above its
+            // target rather than a wrapped-around one it would wait on
+            raise_device_error(p.err, kErrWorkspaceDirty);
+            atomicOr(p.counters + t0, 0x80000000u);
+          }
         }
       }
       if (last_seg_finishes_shared(lo, hi, nkb)) {

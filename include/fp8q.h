@@ -343,8 +343,10 @@ FP8Q_API fp8q_status fp8_kv_quantize_delayed(const void *k, const void *v, int64
  * to completion leaves all of it zero-filled again (counters and partial sums), so it can be
  * reused as is, by calls of any shape.  After a device error
  * (fp8q_device_status() != 0) zero it again.  Calls that may run concurrently (e.g. on
- * unordered streams) need separate workspaces.  A counter found non-zero raises device error
- * bit 1 and leaves the affected output tiles unwritten.
+ * unordered streams) need separate workspaces.  Detection of a workspace that was not zero is
+ * best effort: a tile counter at or above the tile's number of contributors raises device error
+ * bit 1 and leaves that tile unwritten; a smaller stale count may go unseen and leave the tile
+ * summed from incomplete partials.  The call completes either way.
  * Requirements: M >= 1; N % 128 == 0; K % 128 == 0 (else FP8Q_ERR_UNSUPPORTED);
  * A, B, C 16-byte aligned.  ws may be NULL when fp8q_gemm_workspace_bytes() is 0.
  */

@@ -162,12 +162,23 @@ def test_gemm_decode_workspace_reused_across_shapes(orc):
 
 
 def test_gemm_decode_dirty_workspace_is_reported(orc):
-    """Counters that are not zero on entry raise device error bit 1 (no wait depends on them)."""
+    """Counters at or above a shared tile's number of contributors on entry (here all 0xFF bytes)
+    raise device error bit 1: the tile's finishing CTA and its later contributors see the excess at
+    once, so the call ends without its bounded wait running out (bit 0 clear); once the workspace
+    is zero-filled again the results are right."""
     M, N, K = 16, 2048, 4096
     a, sa, b, sb = operands(orc, M, N, K, 1, 2, seed=13)
-    ws = torch.full((fq.gemm_workspace_bytes(M, N, K),), 0xFF, dtype=torch.uint8, device="cuda")
-    fq.fp8_gemm_blockscaled(dev(a), dev(sa), dev(b), dev(sb), 1, 2, ws=ws)
-    assert fq.device_status() & 2
+    args = (dev(a), dev(sa), dev(b), dev(sb), 1, 2)
+    nbytes = fq.gemm_workspace_bytes(M, N, K)
+    ws = torch.full((nbytes,), 0xFF, dtype=torch.uint8, device="cuda")
+    fq.fp8_gemm_blockscaled(*args, ws=ws)
+    torch.cuda.synchronize()
+    assert fq.device_status() == 2
+    ws.zero_()
+    got = fq.fp8_gemm_blockscaled(*args, ws=ws)
+    torch.cuda.synchronize()
+    assert fq.device_status() == 0
+    check_tolerance(host(got), orc.gemm_rows(a, sa, 1, b, sb, 2, np.arange(M)), "after re-zeroing")
 
 
 def test_gemm_config2_prefill_8b(orc):
