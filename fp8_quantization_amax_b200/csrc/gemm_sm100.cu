@@ -467,6 +467,13 @@ constexpr int kTBuf = 4;                // TMEM buffers of kMaxMp columns
 constexpr int kMaxMp = 64;
 constexpr uint32_t kTmemCols = kTBuf * kMaxMp;
 constexpr int kScaleSlots = 8;
+// At 64 tokens the scale warp forms each unit's products RN(sA[m] * sB) once for the CTA (from
+// raw scales staged by cp.async kRawLag units ahead) and the promotion only loads them: there the
+// promotion's instructions are the bound (70B shapes: 56.6 -> 53.7 us).  With fewer tokens the
+// per-thread products are cheaper than the staging, whose per-unit wait then paces the kernel
+// (measured slower at 16, 32 and 48 tokens).
+constexpr int kProdMinMp = 64;
+constexpr int kRawLag = 8;
 constexpr uint32_t kStageW = BM * BK;   // 16 KB of weight codes
 constexpr int kMaxStages = 10;
 
@@ -512,8 +519,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
                                                              const __grid_constant__ CUtensorMap tX, Params p) {
   constexpr uint32_t kIdescD = (1u << 4) | ((uint32_t)(MP >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  __shared__ __align__(16) float sc_a[kScaleSlots][MP];
+  constexpr bool kProd = MP >= kProdMinMp;
+  __shared__ __align__(16) float sc_a[kScaleSlots][MP];   // sA[m], or RN(sA[m] * sB) when kProd
   __shared__ float sc_b[kScaleSlots];
+  __shared__ __align__(16) float raw_a[kProd ? kRawLag + 1 : 1][MP];
+  __shared__ float raw_b[kProd ? kRawLag + 1 : 1][32];
   __shared__ uint64_t bars[2 * kMaxStages + 2 * kTBuf + 2 * kScaleSlots + 2];
   __shared__ uint32_t tmem_slot;
   __shared__ uint32_t s_fin_ok;
@@ -627,34 +637,79 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
       if (i > 0) mbar_wait(&tfull[(i - 1) % kTBuf], ((i - 1) / kTBuf) & 1u, p.err);
     }
   } else if (warp == 2) {
-    // scale producer: the K block's activation scales (one per token, zero beyond M) and the
-    // tile's weight scale, copied with cp.async into a ring slot
-    uint32_t r = 0, ph = 0;
-    for (uint32_t i = 0; i < n_units; ++i) {
-      const uint32_t u = lo + i, t = u / nkb, kb = u - t * nkb;
-      if (i >= (uint32_t)kScaleSlots && !mbar_wait(&sempty[r], ph ^ 1u, p.err)) break;
+    if constexpr (kProd) {
+      // scale producer, product form: each unit's activation scales (zero beyond M) and weight
+      // scale are copied with cp.async into a staging ring; kRawLag units later, when they have
+      // landed, each lane forms the products RN(sA[m] * sB) of its two tokens once for the CTA
+      // (the roundings the promotion would make) and publishes them in the ring
+      uint32_t r = 0, ph = 0;
+      const int m0 = lane * 2;
+      for (uint32_t i = 0; i < n_units + kRawLag; ++i) {
+        if (i < n_units) {
+          const uint32_t u = lo + i, t = u / nkb, kb = u - t * nkb, rs = i % (kRawLag + 1);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int m = lane * 2 + h;
-        if (m < MP) {
-          const float* src = p.gA_group ? p.sA + (size_t)kb * p.M + (m < p.M ? m : 0) : p.sA;
-          const uint32_t nbytes = (p.gA_group && m >= p.M) ? 0u : 4u;
-          asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(&sc_a[r][m])), "l"(src),
-                       "r"(nbytes)
+          for (int h = 0; h < 2; ++h) {
+            const int m = m0 + h;
+            if (m < MP) {
+              const float* src = p.gA_group ? p.sA + (size_t)kb * p.M + (m < p.M ? m : 0) : p.sA;
+              const uint32_t nbytes = (p.gA_group && m >= p.M) ? 0u : 4u;
+              asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(&raw_a[rs][m])), "l"(src),
+                           "r"(nbytes)
+                           : "memory");
+            }
+          }
+          const float* srcb = p.gB_block ? p.sB + (size_t)t * nkb + kb : p.sB;
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(&raw_b[rs][lane])), "l"(srcb)
                        : "memory");
         }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        if (i < (uint32_t)kRawLag) continue;
+        // this lane's copies for unit j have landed once at most kRawLag later groups are pending
+        const uint32_t j = i - kRawLag, rs = j % (kRawLag + 1);
+        asm volatile("cp.async.wait_group %0;" ::"n"(kRawLag) : "memory");
+        if (j >= (uint32_t)kScaleSlots && !mbar_wait(&sempty[r], ph ^ 1u, p.err)) break;
+        if (m0 < MP) {
+          const float sb = raw_b[rs][lane];
+          const float2 c = __fmul2_rn(make_float2(raw_a[rs][m0], raw_a[rs][m0 + 1]), make_float2(sb, sb));
+          *reinterpret_cast<float2*>(&sc_a[r][m0]) = c;
+        }
+        mbar_arrive(&sfull[r]);   // release: this lane's products
+        if (++r == kScaleSlots) {
+          r = 0;
+          ph ^= 1u;
+        }
       }
-      if (lane == 0) {
-        const float* src = p.gB_block ? p.sB + (size_t)t * nkb + kb : p.sB;
-        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(&sc_b[r])), "l"(src) : "memory");
+      asm volatile("cp.async.wait_all;" ::: "memory");
+    } else {
+      // scale producer: the K block's activation scales (one per token, zero beyond M) and the
+      // tile's weight scale, copied with cp.async into a ring slot
+      uint32_t r = 0, ph = 0;
+      for (uint32_t i = 0; i < n_units; ++i) {
+        const uint32_t u = lo + i, t = u / nkb, kb = u - t * nkb;
+        if (i >= (uint32_t)kScaleSlots && !mbar_wait(&sempty[r], ph ^ 1u, p.err)) break;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int m = lane * 2 + h;
+          if (m < MP) {
+            const float* src = p.gA_group ? p.sA + (size_t)kb * p.M + (m < p.M ? m : 0) : p.sA;
+            const uint32_t nbytes = (p.gA_group && m >= p.M) ? 0u : 4u;
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(&sc_a[r][m])), "l"(src),
+                         "r"(nbytes)
+                         : "memory");
+          }
+        }
+        if (lane == 0) {
+          const float* src = p.gB_block ? p.sB + (size_t)t * nkb + kb : p.sB;
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(&sc_b[r])), "l"(src) : "memory");
+        }
+        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&sfull[r])) : "memory");
+        if (++r == kScaleSlots) {
+          r = 0;
+          ph ^= 1u;
+        }
       }
-      asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&sfull[r])) : "memory");
-      if (++r == kScaleSlots) {
-        r = 0;
-        ph ^= 1u;
-      }
+      asm volatile("cp.async.wait_all;" ::: "memory");
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == 7) {
     // reducer: the split-tile bookkeeping, off the promotion warps' path.  A CTA's range holds at
     // most one segment of a tile a lower CTA started (its first: the partial is counted in here)
@@ -747,13 +802,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
       // acc[m] += RN(sA[m] * sB) * P[m] on packed pairs (two independent roundings each: the
       // same values as one element at a time)
       auto promote = [&](uint32_t rs, const uint32_t (&v)[MP]) {
-        const float sb = sc_b[rs];
+        const float sb = kProd ? 1.0f : sc_b[rs];
         const float2 sb2 = make_float2(sb, sb);
 #pragma unroll
         for (int m = 0; m < MP; m += 4) {
           const float4 a4 = *reinterpret_cast<const float4*>(&sc_a[rs][m]);
-          const float2 c01 = __fmul2_rn(make_float2(a4.x, a4.y), sb2);
-          const float2 c23 = __fmul2_rn(make_float2(a4.z, a4.w), sb2);
+          const float2 c01 = kProd ? make_float2(a4.x, a4.y) : __fmul2_rn(make_float2(a4.x, a4.y), sb2);
+          const float2 c23 = kProd ? make_float2(a4.z, a4.w) : __fmul2_rn(make_float2(a4.z, a4.w), sb2);
           const float2 s01 = __ffma2_rn(c01, make_float2(__uint_as_float(v[m]), __uint_as_float(v[m + 1])),
                                         make_float2(acc[m], acc[m + 1]));
           const float2 s23 = __ffma2_rn(c23, make_float2(__uint_as_float(v[m + 2]), __uint_as_float(v[m + 3])),
