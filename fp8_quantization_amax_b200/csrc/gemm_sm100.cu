@@ -541,9 +541,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
   const uint32_t lo = range_lo(blockIdx.x, p.W, p.G), hi = range_lo(blockIdx.x + 1, p.W, p.G);
   const uint32_t n_units = hi - lo;
   const int nkb = p.nkb;
-  if (warp == 0 && lane == 0 && n_units > 0) {
+  if (warp == 2 && lane == 0 && n_units > 0) {
     // the weights are read once: start their first tiles towards L2 before waiting on the
-    // previous grid (a prefetch only warms L2, which stays coherent with any later write)
+    // previous grid (a prefetch only warms L2, which stays coherent with any later write); the
+    // scale warp is idle until then, so thread 0's barrier set-up does not wait behind it
     if (!p.Bp) tma_prefetch_desc(&tW);
     tma_prefetch_desc(&tX);
     for (uint32_t i = 0; i < n_units && i < (uint32_t)S; ++i) {
