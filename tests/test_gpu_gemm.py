@@ -108,12 +108,14 @@ def test_gemm_block_scale_selection(orc):
 
 
 @pytest.mark.parametrize("ga,gb", [(1, 2), (0, 0)])
-@pytest.mark.parametrize("M", [1, 7, 16, 33, 48, 64, 65])
+@pytest.mark.parametrize("M", [1, 7, 16, 33, 48, 57, 64, 65])
 @pytest.mark.parametrize("NK", [(128, 128), (384, 640), (1024, 4096), (2048, 1280)])
 def test_gemm_decode_split(orc, ga, gb, M, NK):
     """Decode shapes (M <= 64) split the (weight tile, K block) units over all SMs; these N, K
     give ranges that start and end inside tiles, a tile spread over several CTAs and a single
-    unit.  M = 65 is the first shape past the split path."""
+    unit.  M rounds up to 16, 48 or 64 tokens on the MMA's N side (57: zero-filled rows on the
+    64-token path, whose scale products come from the scale warp); M = 65 is the first shape past
+    the split path."""
     N, K = NK
     a, sa, b, sb = operands(orc, M, N, K, ga, gb, seed=7 * M + N + K)
     got = run_gpu(a, sa, b, sb, ga, gb)
