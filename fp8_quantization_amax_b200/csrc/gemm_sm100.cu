@@ -736,7 +736,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
         }
       }
       if (last_seg_finishes_shared(lo, hi, nkb)) {
-        // polled from the start, so the wait is normally over before the last unit is promoted
+        // polled while this CTA's units stream (the later contributors count in early in their
+        // runs), so the wait is normally over before the last unit is promoted
         const uint32_t need = cta_of(t1 * nkb + nkb - 1, p.W, p.G) - blockIdx.x;
         const uint64_t t_start = globaltimer_ns();
         uint32_t v = 0;
