@@ -744,9 +744,10 @@ def profile_target(name, reps):
     stream = torch.cuda.Stream(device)
     with torch.cuda.stream(stream):
         if name.startswith("gemm") and not name.startswith("gemm_mx"):
-            if name == "gemm_70b_up_m16384":
+            if name in ("gemm_70b_up_m16384", "gemm_70b_up_m64"):
                 w = dev_bf16(synth.weight_70b(seed=4, which="up"), device)
-                x = dev_bf16(synth.activations_70b(seed=4, m=16384, which="up"), device)
+                m70 = 64 if name == "gemm_70b_up_m64" else 16384
+                x = dev_bf16(synth.activations_70b(seed=4, m=m70, which="up"), device)
             else:
                 w = dev_bf16(synth.weight_8b(seed=1), device)
                 x = dev_bf16(synth.activations(seed=1), device)
@@ -804,7 +805,7 @@ def main():
     ap.add_argument("--skip-extras", action="store_true",
                     help="time the steps only: no e2e, CPU baseline or supplementary kernels (for profiling)")
     ap.add_argument("--profile-target", default=None,
-                    choices=["gemm_8b_m8192", "gemm_8b_m16", "gemm_mx_8b_m8192", "gemm_70b_up_m16384", "kv_tok128", "kv_head",
+                    choices=["gemm_8b_m8192", "gemm_8b_m16", "gemm_mx_8b_m8192", "gemm_70b_up_m16384", "gemm_70b_up_m64", "kv_tok128", "kv_head",
                              "kv_delayed", "mx_8b", "dequant_8b"],
                     help="run one workload a few times and exit (a small target for ncu)")
     args = ap.parse_args()
