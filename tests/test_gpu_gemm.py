@@ -207,25 +207,31 @@ def test_gemm_config2_decode_8b(orc):
 @pytest.mark.parametrize("which", ["up", "down"])
 @pytest.mark.parametrize("M", [16384, 64])
 def test_gemm_config4_70b(orc, which, M):
+    """Prefill: one sampled row in every one of the 128 M tiles (plus the first and last row), so
+    every output tile, and every tile of every persistent CTA's walk, is compared."""
     w = synth.weight_70b(seed=4, which=which)
     x = synth.activations_70b(seed=4, m=M, which=which)
     N, K = w.shape
     a, sa, b, sb = operands(orc, M, N, K, 1, 2, 4, x=x, w=w)
     got = run_gpu(a, sa, b, sb, 1, 2)
-    rows = sample_rows(M)[:40] if M > 64 else np.arange(M)
+    rows = sample_rows(M) if M > 64 else np.arange(M)
+    assert M <= 64 or np.array_equal(np.unique(rows // 128), np.arange(M // 128))
     ref = orc.gemm_rows(a, sa, 1, b, sb, 2, rows)
     check_tolerance(got[rows], ref, f"config 4 {which} M={M}")
 
 
-def test_gemm_config4_per_tensor_variant(orc):
+@pytest.mark.parametrize("M", [1024, 16384])
+def test_gemm_config4_per_tensor_variant(orc, M):
+    """The per-tensor-scale variant at the configuration's prefill size, every M tile sampled."""
     w = synth.weight_70b(seed=4, which="up")
-    x = synth.activations_70b(seed=4, m=1024, which="up")
+    x = synth.activations_70b(seed=4, m=M, which="up")
     N, K = w.shape
-    a, sa, b, sb = operands(orc, 1024, N, K, 0, 0, 4, x=x, w=w)
+    a, sa, b, sb = operands(orc, M, N, K, 0, 0, 4, x=x, w=w)
     got = run_gpu(a, sa, b, sb, 0, 0)
-    rows = sample_rows(1024)
+    rows = sample_rows(M)
+    assert np.array_equal(np.unique(rows // 128), np.arange(M // 128))
     ref = orc.gemm_rows(a, sa, 0, b, sb, 0, rows)
-    check_tolerance(got[rows], ref, "config 4 per-tensor")
+    check_tolerance(got[rows], ref, f"config 4 per-tensor M={M}")
 
 
 # ---------------------------------------------------------------- packed weight tiles

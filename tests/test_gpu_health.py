@@ -4,6 +4,11 @@ The scale histogram runs on real scale arrays (1x128 and 128x128 quantization, t
 per-head x 128-token scales, MXFP8 bytes) and on hand-made arrays with zero, subnormal, NaN and
 Inf scales; the underflow count on the codes of a quantization whose small values flush to
 zero, including lengths that are not a multiple of the kernel's eight-element vectors.
+
+No CUDA output becomes an oracle input: the expected histogram and count come from the
+oracle's own quantization of the same input.  Each case checks the counting kernel on the
+oracle's scales or codes, and then the whole GPU chain (the GPU's quantizer followed by its
+counting kernel) against the same expected value.
 """
 import numpy as np
 import pytest
@@ -34,21 +39,29 @@ def gpu_hist(scales_t):
 @pytest.mark.parametrize("gran", [fq.GROUP_1x128, fq.BLOCK_128x128])
 def test_histogram_of_quantizer_scales(orc, gran):
     x = synth.activations(seed=3, m=1000, k=2048)
+    _, want_s = orc.quantize(x, orc.E4M3, gran)
+    want = orc.scale_histogram(want_s)
+    assert np.array_equal(gpu_hist(dev(want_s)), want)
     _, s = fq.fp8_quantize(dev_bf16(x), fq.E4M3, gran)
-    assert np.array_equal(gpu_hist(s), orc.scale_histogram(host(s)))
+    assert np.array_equal(gpu_hist(s), want)
 
 
 def test_histogram_of_kv_scales(orc):
     k, v = synth.kv_70b(seed=3, tokens=4096)
-    r = fq.fp8_kv_quantize(dev_bf16(k), dev_bf16(v), fq.E4M3, fq.KV_PER_HEAD_TOK128)
-    ks = r[2]
-    assert np.array_equal(gpu_hist(ks), orc.scale_histogram(host(ks)))
+    want_ks = orc.kv_quantize(k, v, orc.E4M3, fq.KV_PER_HEAD_TOK128)[2]
+    want = orc.scale_histogram(want_ks)
+    assert np.array_equal(gpu_hist(dev(want_ks)), want)
+    ks = fq.fp8_kv_quantize(dev_bf16(k), dev_bf16(v), fq.E4M3, fq.KV_PER_HEAD_TOK128)[2]
+    assert np.array_equal(gpu_hist(ks), want)
 
 
 def test_histogram_of_mx_bytes(orc):
     x = synth.activations(seed=1)
+    _, want_s = orc.quantize_mx(x, orc.E4M3)
+    want = orc.scale_histogram(want_s)
+    assert np.array_equal(gpu_hist(dev(want_s)), want)
     _, s = fq.fp8_quantize_mx(dev_bf16(x))
-    assert np.array_equal(gpu_hist(s), orc.scale_histogram(host(s)))
+    assert np.array_equal(gpu_hist(s), want)
 
 
 def test_histogram_special_values_and_accumulation(orc):
@@ -76,8 +89,13 @@ def test_underflow_count_of_a_quantization(orc):
     x = synth.activations(seed=1)
     x = x.copy()
     x[0, :4] = 0x7F00                                # outliers ~1.7e38: every other value underflows
-    codes, _ = fq.fp8_quantize(dev_bf16(x), fq.E4M3, fq.PER_TENSOR)
-    got = fq.fp8_count_underflow(dev_bf16(x), codes)
+    want_codes, _ = orc.quantize(x, orc.E4M3, orc.PER_TENSOR)
+    want = orc.count_underflow(x, want_codes)
+    assert want > 1000
+    xd = dev_bf16(x)
+    from_oracle_codes = fq.fp8_count_underflow(xd, dev(want_codes))
+    codes, _ = fq.fp8_quantize(xd, fq.E4M3, fq.PER_TENSOR)
+    from_gpu_codes = fq.fp8_count_underflow(xd, codes)
     torch.cuda.synchronize()
-    want = orc.count_underflow(x, host(codes))
-    assert want > 1000 and int(host(got)[0]) == want
+    assert int(host(from_oracle_codes)[0]) == want
+    assert int(host(from_gpu_codes)[0]) == want
