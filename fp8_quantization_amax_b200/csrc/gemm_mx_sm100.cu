@@ -352,11 +352,8 @@ cudaError_t launch_gemm_mx(const uint8_t* A, const uint8_t* sfa, int fa, const u
   p.C = C;
   p.err = device_error_word();
   const int grid = std::max(1, std::min(p.tiles, device_sm_count()));
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(k_gemm_mx, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-    attr = true;
-  }
+  const cudaError_t ea = ensure_dynamic_smem((const void*)k_gemm_mx, kSmemBytes);
+  if (ea != cudaSuccess) return ea;
   return launch_pdl(k_gemm_mx, dim3(grid), dim3(kThreads), kSmemBytes, st, mA, mB, p);
 }
 

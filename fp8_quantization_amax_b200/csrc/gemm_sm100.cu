@@ -450,13 +450,19 @@ constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + (2 * kStages + 4) *
 // contiguously over all CTAs (a CTA's range may cross tile boundaries); each CTA promotes its
 // units per K block (acc[m] += sB[tile][kb] * sA[kb][m] * P^T[n][m], thread = weight row n).
 // A tile that lies wholly in one CTA's range is rounded to bf16 and stored directly.  A tile
-// shared by several CTAs is finished by the CTA that started it (the lowest contributor, for
-// which it is the last segment of its range): every later contributor writes its fp32 partial
-// to the workspace and counts itself in on the tile's counter without waiting (for them it is
-// the first segment, done early in their run); the first contributor's reducer warp polls the
-// counter while its units stream, then its promotion warps add the other partials to their own
-// in ascending CTA order (deterministic), store the tile, and clear the partials and the
-// counter, so every completed call leaves the whole workspace zero.
+// shared by several CTAs is finished without any CTA waiting for another, so the result does
+// not depend on which CTAs are resident at the same time.  Every later contributor (for which
+// the tile is the first segment of its range, done early in its run) writes its fp32 partial to
+// the workspace and counts itself in on the tile's counter.  The CTA that started the tile (for
+// which it is the last segment) polls that counter while its units stream:
+//   - when every later contributor is in by the time its own promotion of the tile ends, its
+//     promotion warps add the other partials to their own and store the tile;
+//   - otherwise it publishes its partial too and counts itself in, and whichever contributor
+//     counts in last (the atomic add that completes the count) sums every partial and stores
+//     the tile with its bookkeeping warp.
+// Both ways add the partials in ascending CTA order starting from the first contributor's, so
+// the output is the same bits whichever CTA finishes.  The finisher clears the partials it read
+// and the counter, so every completed call leaves the whole workspace zero.
 //   warp 0 TMA producer, warp 1 MMA issuer (four TMEM buffers), warp 2 scale producer,
 //   warps 3-6 promotion, warp 7 split-tile bookkeeping.
 namespace dec {
@@ -514,6 +520,68 @@ __host__ __device__ __forceinline__ uint32_t cta_of(uint32_t u, uint32_t W, uint
   return c;
 }
 
+// The bookkeeping warp's decision (s_fin) for the tile a CTA started and a higher CTA ends.
+constexpr uint32_t kFinSkip = 0;      // nothing more here: a workspace error, or another CTA finishes
+constexpr uint32_t kFinHere = 1;      // every later contributor is in: the promotion warps finish it
+constexpr uint32_t kFinPublish = 2;   // publish this CTA's partial and count it in
+// how long the starting CTA keeps polling once its own part of the tile is done, before it
+// publishes its partial instead (a bounded optimisation, not a dependency)
+constexpr uint64_t kFinGraceNs = 3000;
+
+// CTA c's partial of tile t: [MP][128] fp32, rows contiguous (slot t - c's first tile of c's maxseg)
+__device__ __forceinline__ float* partial_slot(const Params& p, int mp, uint32_t c, uint32_t t) {
+  const uint32_t t_first = range_lo(c, p.W, p.G) / (uint32_t)p.nkb;
+  return p.partials + ((size_t)(c * (uint32_t)p.maxseg + (t - t_first)) * mp) * BM;
+}
+
+// One warp finishes tile t once every contributor c_first..c_last has published its partial:
+// lane l owns rows 4l..4l+3; the partials are added in ascending CTA order starting from
+// c_first's (the order the promotion warps use when c_first finishes the tile itself), rounded
+// to bf16 and stored; then the partials are cleared and the tile's counter reset.
+template <int MP>
+__device__ __forceinline__ void finish_tile_warp(const Params& p, uint32_t t, uint32_t c_first, uint32_t c_last,
+                                              int lane) {
+  constexpr int kChunk = 16;
+  const int r0 = lane * 4;
+  for (int m0 = 0; m0 < MP; m0 += kChunk) {
+    float4 sum[kChunk];
+    const float* first = partial_slot(p, MP, c_first, t) + (size_t)m0 * BM + r0;
+#pragma unroll
+    for (int j = 0; j < kChunk; ++j) sum[j] = __ldcg(reinterpret_cast<const float4*>(first + (size_t)j * BM));
+#pragma unroll 1
+    for (uint32_t c = c_first + 1; c <= c_last; ++c) {
+      const float* src = partial_slot(p, MP, c, t) + (size_t)m0 * BM + r0;
+      float4 part[kChunk];
+#pragma unroll
+      for (int j = 0; j < kChunk; ++j) part[j] = __ldcg(reinterpret_cast<const float4*>(src + (size_t)j * BM));
+#pragma unroll
+      for (int j = 0; j < kChunk; ++j) {
+        sum[j].x += part[j].x;
+        sum[j].y += part[j].y;
+        sum[j].z += part[j].z;
+        sum[j].w += part[j].w;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kChunk; ++j) {
+      const int m = m0 + j;
+      if (m < p.M) {
+        const uint2 v = make_uint2(f32x2_to_bf16x2(sum[j].x, sum[j].y), f32x2_to_bf16x2(sum[j].z, sum[j].w));
+        *reinterpret_cast<uint2*>(p.C + (size_t)m * p.N + (size_t)t * BM + r0) = v;
+      }
+    }
+  }
+  const float4 zero = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll 1
+  for (uint32_t c = c_first; c <= c_last; ++c) {
+    float* dst = partial_slot(p, MP, c, t) + r0;
+#pragma unroll 4
+    for (int m = 0; m < MP; ++m) *reinterpret_cast<float4*>(dst + (size_t)m * BM) = zero;
+  }
+  __syncwarp();
+  if (lane == 0) p.counters[t] = 0;
+}
+
 template <int MP>
 __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constant__ CUtensorMap tW,
                                                              const __grid_constant__ CUtensorMap tX, Params p) {
@@ -524,9 +592,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
   __shared__ float sc_b[kScaleSlots];
   __shared__ __align__(16) float raw_a[kProd ? kRawLag + 1 : 1][MP];
   __shared__ float raw_b[kProd ? kRawLag + 1 : 1][32];
-  __shared__ uint64_t bars[2 * kMaxStages + 2 * kTBuf + 2 * kScaleSlots + 2];
+  __shared__ uint64_t bars[2 * kMaxStages + 2 * kTBuf + 2 * kScaleSlots + 4];
   __shared__ uint32_t tmem_slot;
-  __shared__ uint32_t s_fin_ok;
+  __shared__ uint32_t s_fin;   // the bookkeeping warp's decision for the tile this CTA started
   uint8_t* smem = smem_raw + (((smem_u32(smem_raw) + 1023u) & ~1023u) - smem_u32(smem_raw));
   const int S = p.stages;
   uint64_t* full = bars;
@@ -535,8 +603,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
   uint64_t* tempty = tfull + kTBuf;
   uint64_t* sfull = tempty + kTBuf;
   uint64_t* sempty = sfull + kScaleSlots;
-  uint64_t* seg_written = sempty + kScaleSlots;   // the four promotion warps' partials are out
-  uint64_t* fin_ready = seg_written + 1;          // every later contributor of the last tile is in
+  uint64_t* seg_written = sempty + kScaleSlots;   // first segment: the promotion warps' partials are out
+  uint64_t* at_end = seg_written + 1;             // last segment: the promotion warps have its partial
+  uint64_t* fin_ready = at_end + 1;               // last segment: s_fin is set
+  uint64_t* seg_pub = fin_ready + 1;              // last segment: its partial is published
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t lo = range_lo(blockIdx.x, p.W, p.G), hi = range_lo(blockIdx.x + 1, p.W, p.G);
   const uint32_t n_units = hi - lo;
@@ -557,7 +627,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
   }
   if (threadIdx.x == 0) {
     mbar_init(seg_written, 4);
+    mbar_init(at_end, 4);
     mbar_init(fin_ready, 1);
+    mbar_init(seg_pub, 4);
     for (int i = 0; i < S; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
@@ -712,51 +784,89 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
       asm volatile("cp.async.wait_all;" ::: "memory");
     }
   } else if (warp == 7) {
-    // reducer: the split-tile bookkeeping, off the promotion warps' path.  A CTA's range holds at
-    // most one segment of a tile a lower CTA started (its first: the partial is counted in here)
-    // and at most one segment of a tile it starts but a higher CTA ends (its last: this CTA adds
-    // the others' partials to its own, once all of them are counted in).
-    if (lane == 0 && n_units > 0) {
+    // split-tile bookkeeping.  A CTA's range holds at most one segment of a tile a lower CTA
+    // started (its first: the partial is counted in here) and at most one segment of a tile it
+    // starts but a higher CTA ends (its last: the decision below).  No step waits for another CTA.
+    if (n_units > 0) {
       const uint32_t t0 = lo / nkb, t1 = (hi - 1) / nkb;
       if (first_seg_adds_to_lower(lo, nkb)) {
         const uint32_t c_first = cta_of(t0 * nkb, p.W, p.G), c_last = cta_of(t0 * nkb + nkb - 1, p.W, p.G);
+        uint32_t last = 0;
         // the promotion warps hand their partial writes over through the mbarrier (release /
         // acquire at CTA scope); this gpu-scope fence then orders all of them (cumulatively)
         // before the count
-        if (mbar_wait(seg_written, 0, p.err)) {
+        if (lane == 0 && mbar_wait(seg_written, 0, p.err)) {
           __threadfence();
           const uint32_t old = atomicAdd(p.counters + t0, 1u);
-          if (old >= c_last - c_first) {
+          if (old > c_last - c_first) {
             // a workspace that was not zero: report it and mark the counter (its top bit stays
-            // set however the other adds interleave), so the finishing CTA sees a count above its
-            // target rather than a wrapped-around one it would wait on
+            // set however the other adds interleave), so no contributor takes it for complete
             raise_device_error(p.err, kErrWorkspaceDirty);
             atomicOr(p.counters + t0, 0x80000000u);
+          } else {
+            last = old == c_last - c_first;   // every other contributor, the starter included, is in
           }
+        }
+        if (__shfl_sync(0xffffffffu, last, 0)) {
+          __threadfence();
+          finish_tile_warp<MP>(p, t0, c_first, c_last, lane);
         }
       }
       if (last_seg_finishes_shared(lo, hi, nkb)) {
-        // polled while this CTA's units stream (the later contributors count in early in their
-        // runs), so the wait is normally over before the last unit is promoted
-        const uint32_t need = cta_of(t1 * nkb + nkb - 1, p.W, p.G) - blockIdx.x;
-        const uint64_t t_start = globaltimer_ns();
-        uint32_t v = 0;
-        bool timed_out = false;
-        for (;;) {
-          asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p.counters + t1) : "memory");
-          if (v >= need) break;
-          if (globaltimer_ns() - t_start > kWaitLimitNs) {
-            raise_device_error(p.err, kErrWaitTimeout);
-            timed_out = true;
-            break;
+        const uint32_t c_last = cta_of(t1 * nkb + nkb - 1, p.W, p.G);
+        const uint32_t need = c_last - blockIdx.x;   // later contributors
+        uint32_t dec = kFinSkip;
+        if (lane == 0) {
+          // polled while this CTA's units stream (the later contributors count in early in their
+          // runs); the poll ends when they are all in, or kFinGraceNs after this CTA's own
+          // promotion of the tile is done, whichever comes first.  The grace only saves the
+          // publish-and-reduce round trips when a contributor is about to count in (a middle CTA
+          // ends its run when this one does); nothing depends on another CTA being resident.
+          const uint64_t t_start = globaltimer_ns();
+          uint64_t t_end = 0;
+          for (;;) {
+            uint32_t v;
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p.counters + t1) : "memory");
+            if (v == need) {
+              p.counters[t1] = 0;   // nobody else touches it in this call: leave it zero
+              dec = kFinHere;
+              break;
+            }
+            if (v > need) {
+              raise_device_error(p.err, kErrWorkspaceDirty);
+              break;
+            }
+            if (t_end == 0 && mbar_test(at_end, 0)) t_end = globaltimer_ns();
+            if (t_end != 0 && globaltimer_ns() - t_end > kFinGraceNs) {
+              dec = kFinPublish;
+              break;
+            }
+            if (globaltimer_ns() - t_start > kWaitLimitNs) {
+              raise_device_error(p.err, kErrWaitTimeout);
+              break;
+            }
+            __nanosleep(128);
           }
-          __nanosleep(128);
+          s_fin = dec;
+          mbar_arrive(fin_ready);
         }
-        const bool ok = !timed_out && v == need;
-        if (!timed_out && v > need) raise_device_error(p.err, kErrWorkspaceDirty);
-        if (ok) p.counters[t1] = 0;   // every later contributor has counted in: leave it zero
-        s_fin_ok = ok ? 1u : 0u;
-        mbar_arrive(fin_ready);
+        if (__shfl_sync(0xffffffffu, dec, 0) == kFinPublish) {
+          uint32_t last = 0;
+          if (lane == 0 && mbar_wait(seg_pub, 0, p.err)) {
+            __threadfence();
+            const uint32_t old = atomicAdd(p.counters + t1, 1u);
+            if (old > need) {
+              raise_device_error(p.err, kErrWorkspaceDirty);
+              atomicOr(p.counters + t1, 0x80000000u);
+            } else {
+              last = old == need;   // the later contributors came in meanwhile
+            }
+          }
+          if (__shfl_sync(0xffffffffu, last, 0)) {
+            __threadfence();
+            finish_tile_warp<MP>(p, t1, blockIdx.x, c_last, lane);
+          }
+        }
       }
     }
   } else {
@@ -855,11 +965,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_mma(const __grid_constan
           if (lane == 0) mbar_arrive(seg_written);
         } else if (!finish) {
           // this CTA started the tile and a higher one ends it (always this CTA's last segment):
-          // once the reducer has seen every later contributor counted in, add their partials to
-          // this row in ascending CTA order (the same order whichever CTA is slower, so reruns
-          // are bit-identical), and clear them, so that a completed call leaves the workspace zero
+          // the bookkeeping warp decides, without waiting for the other CTAs, whether they are
+          // all in.  If so, add their partials to this row in ascending CTA order (the order the
+          // bookkeeping warp of whichever CTA finishes uses too) and clear them; if not, publish
+          // this row's partial for the CTA that counts in last.
+          __syncwarp();
+          if (lane == 0) mbar_arrive(at_end);
           if (!mbar_wait(fin_ready, 0, p.err)) break;
-          finish = s_fin_ok != 0;
+          const uint32_t dec = s_fin;
+          finish = dec == kFinHere;
+          if (dec == kFinPublish) {
+            float* dst = p.partials + ((size_t)(blockIdx.x * p.maxseg + (t - first_tile)) * MP) * BM + row;
+#pragma unroll
+            for (int m = 0; m < MP; ++m) dst[(size_t)m * BM] = acc[m];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(seg_pub);
+          }
           if (finish) {
             __threadfence();
 #pragma unroll 1
@@ -956,11 +1077,8 @@ template <int MP>
 cudaError_t launch_decode(const CUtensorMap& mW, const CUtensorMap& mX, gemm::dec::Params& p, cudaStream_t st) {
   using namespace gemm::dec;
   const size_t smem = 1024 + (size_t)p.stages * p.stage_bytes;
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(k_decode_mma<MP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    attr = true;
-  }
+  const cudaError_t ea = ensure_dynamic_smem((const void*)k_decode_mma<MP>, smem);
+  if (ea != cudaSuccess) return ea;
   // a programmatic dependent of what precedes it on the stream: its set-up (and the L2 prefetch
   // of the first weight tiles) overlaps that grid's tail; griddepcontrol.wait orders every
   // load and store of operands, scales, workspace and output after it
@@ -1057,6 +1175,7 @@ int check_decode_split(int64_t M, int64_t N, int64_t K, int sms) {
       } else {
         ++n_fin;
         if (t != t1 || !red_fin) return 5;                    // only the last segment, seen by both
+        if ((int)(t - t0) >= maxseg) return 4;                // the slot it may publish into exists
         ++finishers[t];
       }
     }
@@ -1105,18 +1224,12 @@ static cudaError_t launch_prefill(const uint8_t* A, const float* sA, int gA, con
   const bool promote = p.gA_group || p.gB_block;
   const int grid = std::max(1, std::min(p.tiles, device_sm_count()));
   if (promote) {
-    static bool attr = false;
-    if (!attr) {
-      cudaFuncSetAttribute(k_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-      attr = true;
-    }
+    const cudaError_t ea = ensure_dynamic_smem((const void*)k_gemm<true>, kSmemBytes);
+    if (ea != cudaSuccess) return ea;
     return launch_pdl(k_gemm<true>, dim3(grid), dim3(kThreads), kSmemBytes, st, mA, mB, p);
   } else {
-    static bool attr = false;
-    if (!attr) {
-      cudaFuncSetAttribute(k_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-      attr = true;
-    }
+    const cudaError_t ea = ensure_dynamic_smem((const void*)k_gemm<false>, kSmemBytes);
+    if (ea != cudaSuccess) return ea;
     return launch_pdl(k_gemm<false>, dim3(grid), dim3(kThreads), kSmemBytes, st, mA, mB, p);
   }
 }

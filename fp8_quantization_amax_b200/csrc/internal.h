@@ -30,6 +30,11 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // number of SMs of the current device (queried once per device)
 int device_sm_count();
 
+// Raise `kernel`'s dynamic shared-memory limit on the current device to at least `bytes`, once
+// per (kernel, device) and size (thread-safe); returns the error of cudaFuncSetAttribute, or
+// cudaSuccess when an earlier call on this device already set a limit this large.
+cudaError_t ensure_dynamic_smem(const void* kernel, size_t bytes);
+
 // device address of the library's error word on the current device (kernels set bits in it
 // when a bounded wait gives up); read_and_clear_device_error() synchronizes the device first
 uint32_t* device_error_word();

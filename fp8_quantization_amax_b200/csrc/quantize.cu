@@ -319,11 +319,8 @@ static cudaError_t launch_group128_fmt(const uint16_t* x, int64_t rows, int64_t 
   p.wide_stores = cols % 16 == 0;
   p.err = device_error_word();
   const size_t smem = ring_smem(p.stages, kGroupStage);
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(k_group128<FMT, MX>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    attr = true;
-  }
+  const cudaError_t ea = ensure_dynamic_smem((const void*)k_group128<FMT, MX>, smem);
+  if (ea != cudaSuccess) return ea;
   const int grid = grid_for(k_group128<FMT, MX>, smem, p.nitems);
   return launch_pdl(k_group128<FMT, MX>, dim3(grid), dim3(kThreads), smem, st, map, p);
 }
@@ -632,11 +629,8 @@ template <int FMT, int MODE, int CPR, int MAXC>
 static cudaError_t launch_tile_impl(const CUtensorMap& m0, const CUtensorMap& m1, TileParams& p, int max_grid,
                                     cudaStream_t st, int* grid_used) {
   const size_t smem = ring_smem(p.stages, p.stage_bytes);
-  static size_t attr = 0;
-  if (attr < smem) {
-    cudaFuncSetAttribute(k_tile128<FMT, MODE, CPR, MAXC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    attr = smem;
-  }
+  const cudaError_t ea = ensure_dynamic_smem((const void*)k_tile128<FMT, MODE, CPR, MAXC>, smem);
+  if (ea != cudaSuccess) return ea;
   int grid = grid_for(k_tile128<FMT, MODE, CPR, MAXC>, smem, std::max<uint32_t>(p.nitems, 1));
   if (max_grid > 0) grid = std::min(grid, max_grid);
   if (grid_used) *grid_used = grid;
@@ -1000,11 +994,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_quant_many(const __grid_constan
 template <int FMT>
 static cudaError_t launch_many_fmt(const ManyMaps& maps, const ManyParams& p, cudaStream_t st) {
   const size_t smem = ring_smem(p.stages, kGroupStage);
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(k_quant_many<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    attr = true;
-  }
+  const cudaError_t ea = ensure_dynamic_smem((const void*)k_quant_many<FMT>, smem);
+  if (ea != cudaSuccess) return ea;
   const int grid = grid_for(k_quant_many<FMT>, smem, p.nitems);
   return launch_pdl(k_quant_many<FMT>, dim3(grid), dim3(kThreads), smem, st, maps, p);
 }

@@ -7,6 +7,7 @@
 
 #include <cstdint>
 #include <mutex>
+#include <vector>
 
 #include "internal.h"
 #include "sm100.cuh"
@@ -52,6 +53,31 @@ bool make_tmap_2d(CUtensorMap* map, int elem_bytes, const void* base, uint64_t i
                         swizzle_128b ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+cudaError_t ensure_dynamic_smem(const void* kernel, size_t bytes) {
+  struct Entry {
+    const void* kernel;
+    int dev;
+    size_t bytes;
+  };
+  static std::vector<Entry> done;
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (Entry& d : done) {
+    if (d.kernel == kernel && d.dev == dev) {
+      if (d.bytes >= bytes) return cudaSuccess;
+      e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+      if (e == cudaSuccess) d.bytes = bytes;
+      return e;
+    }
+  }
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) done.push_back({kernel, dev, bytes});
+  return e;
 }
 
 uint32_t* device_error_word() {

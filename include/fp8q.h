@@ -127,8 +127,9 @@ FP8Q_API fp8q_status fp8q_selftest_wait_timeout(fp8q_stream_t stream);
  * functions and checks what its split-tile hand-off relies on: each CTA holds at most one
  * segment of a tile a lower CTA started (its first segment) and at most one of a tile it starts
  * but a higher CTA ends (its last); the promotion warps and the bookkeeping warp pick out the same
- * segments; every shared tile has exactly one finishing CTA (its lowest) and c_last - c_first
- * later contributors; every partial slot lies inside the workspace.  Returns 0 when all hold,
+ * segments; every shared tile has exactly one starting CTA (its lowest, which finishes it or
+ * publishes its own partial) and c_last - c_first later contributors; every partial slot, the
+ * starting CTA's included, lies inside the workspace.  Returns 0 when all hold,
  * a positive code naming the first violation, or -1 for a shape that is not a decode shape.
  */
 FP8Q_API int fp8q_check_decode_split(int64_t M, int64_t N, int64_t K, int sms);
@@ -337,7 +338,10 @@ FP8Q_API fp8q_status fp8_kv_quantize_delayed(const void *k, const void *v, int64
  * scaled once at the end: C = bf16(sA * sB * sum_k a*b).
  * Decode shapes (M <= 64) split the (128-row weight tile, K block) pairs evenly over the SMs;
  * per-tensor scales are then applied per K block.  A tile shared by several SMs has its fp32
- * partial sums added in a fixed order, so results are deterministic.  ws: caller-owned device
+ * partial sums added in a fixed order, so results are deterministic.  No block waits for
+ * another (the last contributor to count in finishes a shared tile), so the call completes and
+ * is correct however many of its blocks the device runs at once (other streams' kernels, MPS
+ * or a partitioned device taking SMs make it slower, not wrong).  ws: caller-owned device
  * memory of at least fp8q_gemm_workspace_bytes(M, N, K) bytes, 16-byte aligned (else
  * FP8Q_ERR_WORKSPACE), which must be ZERO-FILLED before its first use; every call that runs
  * to completion leaves all of it zero-filled again (counters and partial sums), so it can be
