@@ -79,6 +79,7 @@ struct Params {
   int M, N, K;
   int num_kb;
   int m_tiles, n_tiles, tiles;
+  int group_m;          // tile walk band height (tile_walk)
   uint32_t idesc;
   const uint8_t* sfa;   // blocked, ceil(M / 128) x K / 128 chunks
   const uint8_t* sfb;   // blocked, N / 128 x K / 128 chunks
@@ -177,7 +178,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_mx(const __grid_constant__
         bool ok = true;
         for (int k = 0; k < my_tiles && ok; ++k) {
           const int t = (int)blockIdx.x + k * (int)gridDim.x;
-          const int mt = t % p.m_tiles, nt = t / p.m_tiles;
+          int mt, nt;
+          tile_walk(t, p.m_tiles, p.n_tiles, p.group_m, &mt, &nt);
           const int m0 = mt * BM, n0 = nt * BN;
           const int nhalves = min(2, (p.N - n0) / 128);    // N % 128 == 0: 1 or 2 valid B halves
           const uint8_t* sfa = p.sfa + (size_t)mt * p.num_kb * kSfChunk;
@@ -271,8 +273,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_mx(const __grid_constant__
     const uint32_t lane_base = tmem_base + ((uint32_t)(quarter * 32) << 16) + half * 128;
     for (int k = 0; k < my_tiles; ++k) {
       const int t = (int)blockIdx.x + k * (int)gridDim.x;
-      const int m = (t % p.m_tiles) * BM + row_in_tile;
-      const int ncol0 = (t / p.m_tiles) * BN + half * 128;
+      int mt, nt;
+      tile_walk(t, p.m_tiles, p.n_tiles, p.group_m, &mt, &nt);
+      const int m = mt * BM + row_in_tile;
+      const int ncol0 = nt * BN + half * 128;
       const uint32_t buf = (uint32_t)k & 1u;
       if (!mbar_wait(&tfull[buf], (uint32_t)(k >> 1) & 1u, p.err)) break;
       tc_fence_after();
@@ -346,6 +350,7 @@ cudaError_t launch_gemm_mx(const uint8_t* A, const uint8_t* sfa, int fa, const u
   p.m_tiles = (int)((M + BM - 1) / BM);
   p.n_tiles = (int)((N + BN - 1) / BN);
   p.tiles = p.m_tiles * p.n_tiles;
+  p.group_m = gemm::tile_group_m(M, K, p.m_tiles);
   p.idesc = idesc_mx(fa, fb);
   p.sfa = sfa;
   p.sfb = sfb;

@@ -72,6 +72,7 @@ struct Params {
   int M, N, K;
   int num_kb;
   int m_tiles, n_tiles, tiles;
+  int group_m;        // tile walk band height (tile_walk)
   const float* sA;
   const float* sB;
   int gA_group;       // 1: sA is [K/128][M]; 0: one scale
@@ -114,7 +115,8 @@ __device__ __forceinline__ void store_row_e4m3(PairFn pair, uint8_t* codes_row, 
 }
 
 __device__ __forceinline__ void tile_coords(int t, const Params& p, int* m0, int* n0) {
-  const int mt = t % p.m_tiles, nt = t / p.m_tiles;
+  int mt, nt;
+  tile_walk(t, p.m_tiles, p.n_tiles, p.group_m, &mt, &nt);
   *m0 = mt * BM;
   *n0 = nt * BN;
 }
@@ -1212,6 +1214,7 @@ static cudaError_t launch_prefill(const uint8_t* A, const float* sA, int gA, con
   p.m_tiles = (int)((M + BM - 1) / BM);
   p.n_tiles = (int)((N + BN - 1) / BN);
   p.tiles = p.m_tiles * p.n_tiles;
+  p.group_m = tile_group_m(M, K, p.m_tiles);
   p.sA = sA;
   p.sB = sB;
   p.gA_group = gA == 1;

@@ -36,6 +36,29 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                : "memory");
 }
 
+// Persistent tile walk of the prefill GEMMs: tile index t -> (M tile, N tile).  Tiles go in
+// bands of group_m M tiles; inside a band M varies fastest, then N.  The CTAs running at the same
+// time (consecutive t) then share group_m A panels and about gridDim / group_m B panels, and both
+// are read from HBM about once per band instead of the whole A once per N column.  With
+// group_m = m_tiles this is the plain M-fastest walk (kept when all of A fits in L2).
+__host__ __device__ __forceinline__ void tile_walk(int t, int m_tiles, int n_tiles, int group_m, int* mt, int* nt) {
+  const int per_band = group_m * n_tiles;
+  const int band = t / per_band;
+  const int r = t - band * per_band;
+  const int rows = min(group_m, m_tiles - band * group_m);   // the last band may be shorter
+  *nt = r / rows;
+  *mt = band * group_m + (r - *nt * rows);
+}
+
+// The band height for an M x K A operand of E4M3 codes: the M-fastest walk while A fits in L2
+// next to the B panels in flight, else 16 M tiles (for G concurrent CTAs the panels per band
+// are about 16 of A and G / 16 of B, the minimum of A + B bytes per wave near G = 148).
+inline int tile_group_m(int64_t M, int64_t K, int m_tiles) {
+  constexpr int64_t kAInL2 = 48ll << 20;
+  if (M * K <= kAInL2) return m_tiles;
+  return m_tiles < 16 ? m_tiles : 16;
+}
+
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 

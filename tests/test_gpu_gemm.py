@@ -7,6 +7,8 @@ Small shapes cover partial M tiles, N not a multiple of the 256-column tile and 
 combination; the configuration shapes are checked on sampled rows (one per 128-row M tile at
 varying offsets, plus the first and last row), which touch every output tile.
 """
+import time
+
 import numpy as np
 import pytest
 import torch
@@ -161,6 +163,47 @@ def test_gemm_decode_workspace_reused_across_shapes(orc):
         assert int(ws.count_nonzero()) == 0, (M, N, K)
         check_tolerance(host(got), orc.gemm_rows(a, sa, 1, b, sb, 2, np.arange(M)), f"{M}x{N}x{K}")
     assert fq.device_status() == 0
+
+
+@pytest.mark.parametrize("M", [16, 64])
+def test_gemm_decode_with_sms_taken(orc, M):
+    """Forward progress without co-residency: a prefill GEMM with 64 persistent CTAs (each using
+    most of an SM's shared memory) holds 64 SMs on one stream while the decode GEMM runs on
+    another, so the decode's higher-numbered CTAs can only start once the prefill ends, long after
+    the lower ones finished.  Tiles those CTAs share are then completed by whichever CTA counts in
+    last.  The output must equal the idle-GPU result bit for bit, with no device error and the
+    workspace left zero."""
+    N, K = 14336, 4096
+    a, sa, b, sb = operands(orc, M, N, K, 1, 2, seed=17 + M)
+    A, SA, B, SB = dev(a), dev(sa), dev(b), dev(sb)
+    ws = torch.zeros(fq.gemm_workspace_bytes(M, N, K), dtype=torch.uint8, device="cuda")
+    want = fq.fp8_gemm_blockscaled(A, SA, B, SB, 1, 2, ws=ws)
+    torch.cuda.synchronize()
+    # the hog: 64 M tiles x 1 N tile, K = 131072 (about half a millisecond on 64 SMs)
+    ha = torch.zeros((8192, 131072), dtype=torch.uint8, device="cuda")
+    hb = torch.zeros((256, 131072), dtype=torch.uint8, device="cuda")
+    one = torch.ones(1, dtype=torch.float32, device="cuda")
+    hc = torch.empty((8192, 256), dtype=torch.bfloat16, device="cuda")
+    s_hog, s_dec = torch.cuda.Stream(), torch.cuda.Stream()
+    got = torch.empty_like(want)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    for _ in range(3):
+        torch.cuda.synchronize()
+        with torch.cuda.stream(s_hog):
+            ev[0].record(s_hog)
+            fq.fp8_gemm_blockscaled(ha, one, hb, one, fq.PER_TENSOR, fq.PER_TENSOR, out=hc)
+            ev[1].record(s_hog)
+        time.sleep(0.002)                            # the hog's CTAs are resident before the decode starts
+        with torch.cuda.stream(s_dec):
+            ev[2].record(s_dec)
+            fq.fp8_gemm_blockscaled(A, SA, B, SB, 1, 2, out=got, ws=ws)
+            ev[3].record(s_dec)
+        torch.cuda.synchronize()
+        assert torch.equal(got.view(torch.int16), want.view(torch.int16))
+        assert int(ws.count_nonzero()) == 0
+        print(f"M={M}: hog {ev[0].elapsed_time(ev[1]) * 1e3:.0f} us, decode {ev[2].elapsed_time(ev[3]) * 1e3:.0f} us")
+    assert fq.device_status() == 0
+    check_tolerance(host(got), orc.gemm_rows(a, sa, 1, b, sb, 2, np.arange(M)), f"M={M} with SMs taken")
 
 
 def test_gemm_decode_dirty_workspace_is_reported(orc):
