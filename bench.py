@@ -16,9 +16,18 @@ e2e    = the same metric through the Python binding of the C ABI with pinned hos
          Steps are pipelined over upload / compute / download streams and two device buffer
          sets, as a streaming user would run them: one step's upload overlaps the previous
          step's download (PCIe is full duplex), so a step costs about its upload time.
-roofline: the step's kernel (k_quant_many), per-launch CUDA events on one step in ten.
-cpu_baseline: the CPU oracle on a bounded row sample of the same workload (rank 0, N = 1).
-supplementary: the other measured kernels (per-tensor, KV cache, dequantize, GEMM).
+The timed region holds exactly K launches of the step's kernel, queued behind a short GPU
+sleep (outside the region) so that it measures the kernels rather than the host's launch rate.
+roofline: the step's kernel (k_quant_many): algorithmic bytes per launch over the mean launch
+         duration in the timed region (region time / K, one launch per step).
+clocks: nvidia-smi sampled every 50 ms for the whole run, summarised over the timed region
+         (the nearest samples when the region is shorter than the interval) and over a 300 ms
+         run of the same steps right after it; every GEMM line carries its own.
+cpu_baseline: the CPU oracle on bounded samples (rank 0, N = 1): the step's two quantizers
+         (all threads and one thread), the KV quantizers, the dequantizer, and the GEMM (8B
+         decode shape in full, 70B prefill on sampled rows with the full time extrapolated).
+supplementary: the other measured kernels (per-tensor, KV cache, dequantize, GEMM), each the
+         median of at least 20 CUDA-event timings.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 """
@@ -97,7 +106,8 @@ def ncu_traffic(kernel_key):
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    """nvidia-smi in loop mode during the timed region (reads settings only)."""
+    """nvidia-smi in loop mode for the whole run (reads settings only); summaries are taken over
+    the wall-clock window of each timed region."""
 
     FIELDS = ["timestamp", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
               "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
@@ -109,7 +119,7 @@ class ClockSampler:
         self.proc = None
 
     def start(self):
-        cmd = ["nvidia-smi", "--query-gpu=" + ",".join(self.FIELDS), "--format=csv,noheader,nounits", "-lms", "100"]
+        cmd = ["nvidia-smi", "--query-gpu=" + ",".join(self.FIELDS), "--format=csv,noheader,nounits", "-lms", "50"]
         if self.gpu_id:
             cmd += ["-i", self.gpu_id]
         try:
@@ -140,11 +150,16 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self, t0, t1):
-        inside = [s for s in self.samples if t0 - 0.05 <= s[0] <= t1 + 0.05]
-        window = "timed"
-        if len(inside) < 3:
-            inside = self.samples
-            window = "whole run (timed region shorter than the sampling interval)"
+        """Median SM clock, max clock and throttle reasons of the samples inside [t0, t1]; a
+        window shorter than the sampling interval takes the three samples nearest its middle."""
+        samples = list(self.samples)
+        inside = [s for s in samples if t0 - 0.01 <= s[0] <= t1 + 0.01]
+        window = "timed region"
+        if len(inside) < 3 and samples:
+            mid = 0.5 * (t0 + t1)
+            inside = sorted(samples, key=lambda s: abs(s[0] - mid))[:3]
+            window = (f"the 3 samples nearest a {1e3 * (t1 - t0):.1f} ms timed region "
+                      f"(max {1e3 * max(abs(s[0] - mid) for s in inside):.0f} ms from its middle)")
         if not inside:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
@@ -182,11 +197,12 @@ def dev_bf16(a, device):
     return torch.from_numpy(np.ascontiguousarray(a, np.uint16).view(np.int16)).view(torch.bfloat16).to(device)
 
 
-def timed(fn, reps, stream, flush=None):
-    """Mean device time (ms) of fn over reps, CUDA events on `stream`, optional L2 flush between."""
+def timed(fn, reps, stream, flush=None, min_reps=20):
+    """Median device time (ms) of fn over reps (at least min_reps), CUDA events on `stream`,
+    optional L2 flush between reps (outside the events)."""
     import torch
-    total = 0.0
-    for _ in range(reps):
+    times = []
+    for _ in range(max(reps, min_reps)):
         if flush is not None:
             flush()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -194,15 +210,15 @@ def timed(fn, reps, stream, flush=None):
         fn()
         b.record(stream)
         b.synchronize()
-        total += a.elapsed_time(b)
-    return total / reps
+        times.append(a.elapsed_time(b))
+    return statistics.median(times)
 
 
 def timed_graph(fn, reps, stream, flush=None):
-    """Mean device time (ms) of one replay of fn captured as a CUDA graph (how a decode step's
+    """Median device time (ms) of one replay of fn captured as a CUDA graph (how a decode step's
     launches run: no host work between them), CUDA events on `stream`, optional L2 flush
-    between replays (outside the timed region).  fn runs once before capture so any lazily
-    created buffers exist outside the graph."""
+    between replays (outside the timed region), at least 20 replays.  fn runs once before
+    capture so any lazily created buffers exist outside the graph."""
     import torch
     with torch.cuda.stream(stream):
         fn()
@@ -212,8 +228,8 @@ def timed_graph(fn, reps, stream, flush=None):
             fn()
         g.replay()
         stream.synchronize()
-        total = 0.0
-        for _ in range(reps):
+        times = []
+        for _ in range(max(reps, 20)):
             if flush is not None:
                 flush()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -221,9 +237,9 @@ def timed_graph(fn, reps, stream, flush=None):
             g.replay()
             b.record(stream)
             b.synchronize()
-            total += a.elapsed_time(b)
+            times.append(a.elapsed_time(b))
     del g
-    return total / reps
+    return statistics.median(times)
 
 
 def gpu_identity(device):
@@ -277,29 +293,104 @@ def reference_arm(args):
 
 # ------------------------------------------------------------------ our arm
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def _cpu_loop(fn, min_s, max_reps=200):
+    """Mean wall time (s) of fn, repeated until min_s has passed (at least once)."""
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        fn()
+        reps += 1
+        if time.perf_counter() - t0 > min_s or reps >= max_reps:
+            break
+    return (time.perf_counter() - t0) / reps, reps
+
+
 def cpu_baseline_leg():
+    """The oracle as it stands, timed on this host's cores on bounded samples of each workload:
+    the benchmarked step (all threads and one thread), the KV quantizers, the dequantizer and
+    the block-scaled GEMM (the 8B decode shape in full, the 70B prefill on sampled rows)."""
     import oracle as orc
     import synth
     rows = 512
-    w = synth.weight_8b(seed=1)[:rows]
-    x = synth.activations(seed=1)[:rows]
+    w = synth.weight_8b(seed=1)
+    x = synth.activations(seed=1)
+    ws_, xs_ = w[:rows], x[:rows]
     nbytes = bytes_w(rows, W_SHAPE[1]) + bytes_x(rows, X_SHAPE[1])
     threads = orc._threads(None)
-    reps, t0 = 0, time.perf_counter()
-    while True:
-        orc.quantize(w, orc.E4M3, orc.BLOCK_128x128, threads=threads)
-        orc.quantize(x, orc.E4M3, orc.GROUP_1x128, threads=threads)
-        reps += 1
-        if time.perf_counter() - t0 > 10.0 or reps >= 200:
-            break
-    dt = (time.perf_counter() - t0) / reps
-    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
-            "sample": f"rows 0..{rows - 1} of the weight (128x128 blocks) and of the activations (1x128 groups), "
-                      f"{reps} repetitions, {threads} threads"}
+
+    def step(th):
+        orc.quantize(ws_, orc.E4M3, orc.BLOCK_128x128, threads=th)
+        orc.quantize(xs_, orc.E4M3, orc.GROUP_1x128, threads=th)
+
+    dt, reps = _cpu_loop(lambda: step(threads), 5.0)
+    dt1, reps1 = _cpu_loop(lambda: step(1), 2.0)
+    out = {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+           "sample": f"rows 0..{rows - 1} of the weight (128x128 blocks) and of the activations (1x128 groups), "
+                     f"{reps} repetitions, {threads} threads",
+           "cpu_model": cpu_model(), "host_cpus": os.cpu_count(),
+           "single_thread": {"value": round(nbytes / dt1 / 1e9, 4), "unit": "GB/s", "reps": reps1}}
+    # KV cache (config 3): the first 8192 tokens of the [131072][8][128] K and V caches; the
+    # oracle's KV quantizer is one thread
+    k, v = synth.kv_70b(seed=3, tokens=8192)
+    e2 = 2 * k.size
+    kv = {}
+    for gran, name, fmt, per_elem in ((orc.KV_PER_HEAD_TOK128, "kv_head_tok128_e4m3", orc.E4M3, 3),
+                                      (orc.KV_PER_HEAD, "kv_head_e4m3", orc.E4M3, 5),
+                                      (orc.KV_PER_TENSOR, "kv_tensor_e5m2", orc.E5M2, 5)):
+        dtk, _ = _cpu_loop(lambda: orc.kv_quantize(k, v, fmt, gran), 1.0, 20)
+        kv[name] = {"GB/s": round(e2 * per_elem / dtk / 1e9, 4), "ms": round(dtk * 1e3, 2)}
+    out["kv"] = {"threads": 1, "sample": "tokens 0..8191 of the config-3 K and V caches (8 heads x 128)", **kv}
+    # dequantize: the 8B weight's first 512 rows from their 128x128 codes (one thread)
+    wc, wsc = orc.quantize(ws_, orc.E4M3, orc.BLOCK_128x128)
+    dtd, _ = _cpu_loop(lambda: orc.dequantize(wc, wsc, orc.E4M3, orc.BLOCK_128x128), 1.0, 50)
+    out["dequant"] = {"GB/s": round(wc.size * 3 / dtd / 1e9, 4), "threads": 1,
+                      "sample": "rows 0..511 of the 14336x4096 weight, 128x128 scales"}
+    # GEMM (fp64 over dequantized operands): the 8B decode shape (M = 16) in full
+    b8, sb8 = orc.quantize(w, orc.E4M3, orc.BLOCK_128x128, threads=threads)
+    a16, sa16 = orc.quantize(x[:16], orc.E4M3, orc.GROUP_1x128)
+    t0 = time.perf_counter()
+    orc.gemm_rows(a16, sa16, 1, b8, sb8, 2, np.arange(16), threads=threads)
+    dtg = time.perf_counter() - t0
+    gemm = {"gemm_8b_up_m16": {"ms": round(dtg * 1e3, 1), "GFLOP/s": round(2.0 * 16 * W_SHAPE[0] * W_SHAPE[1] / dtg / 1e9, 3),
+                               "threads": threads, "sample": "all 16 rows (full)"}}
+    del b8, sb8, w
+    # the 70B up-projection prefill (M = 16384) on sampled rows: one row per 128-row M tile in
+    # tile order, a batch of `threads` rows at a time, until about 5 s have passed
+    b70, sb70 = orc.quantize(synth.weight_70b(seed=4, which="up"), orc.E4M3, orc.BLOCK_128x128, threads=threads)
+    x70 = synth.activations_70b(seed=4, m=16384, which="up")
+    rng = np.random.default_rng(0)
+    sample = np.array([t * 128 + int(rng.integers(0, 128)) for t in range(128)], np.int64)
+    done, t0 = 0, time.perf_counter()
+    while done < sample.size and time.perf_counter() - t0 < 5.0:
+        rws = sample[done:done + threads]
+        a, sa = orc.quantize(x70[rws], orc.E4M3, orc.GROUP_1x128)     # 1x128 groups are row-local
+        orc.gemm_rows(a, sa, 1, b70, sb70, 2, np.arange(rws.size), threads=threads)
+        done += rws.size
+    dtr = time.perf_counter() - t0
+    rows_s = done / dtr
+    n70, k70 = b70.shape
+    gemm["gemm_70b_up_m16384"] = {"rows_per_s": round(rows_s, 3),
+                                  "GFLOP/s": round(2.0 * n70 * k70 * rows_s / 1e9, 3),
+                                  "extrapolated_full_s": round(16384 / rows_s, 1), "threads": threads,
+                                  "sample": f"{done} rows (one per 128-row M tile, tiles 0..{done - 1}), all 28672 "
+                                            f"columns; the full time is extrapolated"}
+    out["gemm"] = gemm
+    return out
 
 
-def supplementary(device, stream, peaks, flush):
-    """Other kernels of the path, each on its own workload (short, device-timed)."""
+def supplementary(device, stream, peaks, flush, sampler):
+    """Other kernels of the path, each on its own workload (short, device-timed); each GEMM line
+    carries the SM clock sampled while it ran."""
     import torch
 
     import fp8_quantization_amax_b200 as fq
@@ -308,6 +399,21 @@ def supplementary(device, stream, peaks, flush):
     hbm = peaks["hbm_gbs"]
     fp8_peak = 2.0 * peaks["bf16_tflops"]                                   # burst
     fp8_peak_sustained = 2.0 * peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])   # under the power cap
+
+    window = [(0.0, 0.0)]
+
+    def ctimed(fn, reps, fl, graph=False):
+        """timed / timed_graph, remembering the wall-clock window for the clock record."""
+        t0 = time.time()
+        ms = (timed_graph if graph else timed)(fn, reps, stream, fl)
+        window[0] = (t0, time.time())
+        return ms
+
+    def add_clocks(key):
+        c = sampler.summary(*window[0])
+        mhz = c["sm_mhz"]
+        out[key]["clocks"] = {"sm_mhz": mhz, "reasons": c["reasons"], "samples": c["samples"],
+                              "sm_cycles_M": round(out[key]["us"] * mhz / 1e6, 3) if mhz else None}
 
     def gbs(nbytes, ms):
         return {"us": round(ms * 1e3, 2), "GB/s": round(nbytes / ms / 1e6, 1), "frac_hbm": round(nbytes / ms / 1e6 / hbm, 3)}
@@ -408,29 +514,32 @@ def supplementary(device, stream, peaks, flush):
             a, sa = xc[:m].contiguous(), xs[:, :m].contiguous()
             cbuf = torch.empty((m, W_SHAPE[0]), dtype=torch.bfloat16, device=device)
             fq.fp8_gemm_blockscaled(a, sa, wc, ws, out=cbuf)
-            ms = timed(lambda: fq.fp8_gemm_blockscaled(a, sa, wc, ws, out=cbuf), 10, stream, flush)
+            ms = ctimed(lambda: fq.fp8_gemm_blockscaled(a, sa, wc, ws, out=cbuf), 20, flush)
             out["gemm_8b_up_m8192"] = gemm_entry(m, W_SHAPE[0], W_SHAPE[1], ms, a, sa, ws, cbuf)
+            add_clocks("gemm_8b_up_m8192")
             # the same GEMM with C quantized to E4M3 1x128 groups in the epilogue, against the two
             # steps it replaces (bf16 C, then the 1x128 quantizer)
             qc = torch.empty((m, W_SHAPE[0]), dtype=torch.uint8, device=device)
             qs = torch.empty(fq.scale_shape(m, W_SHAPE[0], fq.GROUP_1x128), dtype=torch.float32, device=device)
             fq.fp8_gemm_blockscaled_to_fp8(a, sa, wc, ws, codes=qc, scales=qs)
-            ms_f = timed(lambda: fq.fp8_gemm_blockscaled_to_fp8(a, sa, wc, ws, codes=qc, scales=qs), 10, stream, flush)
+            ms_f = ctimed(lambda: fq.fp8_gemm_blockscaled_to_fp8(a, sa, wc, ws, codes=qc, scales=qs), 20, flush)
             ms_2 = timed(lambda: (fq.fp8_gemm_blockscaled(a, sa, wc, ws, out=cbuf),
-                                  fq.fp8_quantize(cbuf, fq.E4M3, fq.GROUP_1x128, codes=qc, scales=qs)), 10, stream,
+                                  fq.fp8_quantize(cbuf, fq.E4M3, fq.GROUP_1x128, codes=qc, scales=qs)), 20, stream,
                          flush)
             flops = 2.0 * m * W_SHAPE[0] * W_SHAPE[1]
             out["gemm_8b_up_m8192_to_fp8"] = {"us": round(ms_f * 1e3, 2), "TFLOP/s": round(flops / ms_f / 1e9, 1),
                                               "frac_fp8_peak": round(flops / ms_f / 1e9 / fp8_peak, 3),
                                               "two_steps_us": round(ms_2 * 1e3, 2)}
+            add_clocks("gemm_8b_up_m8192_to_fp8")
             del qc, qs
             # MXFP8 on the native block-scaled MMA, same shape: both operands quantized in 1x32
             # groups with power-of-two scales (blocked layout)
             am, sam = fq.fp8_quantize_mx_blocked(dev_bf16(synth.activations(seed=1), device))
             bm, sbm = fq.fp8_quantize_mx_blocked(dev_bf16(synth.weight_8b(seed=1), device))
             fq.fp8_gemm_mx(am, sam, bm, sbm, out=cbuf)
-            ms = timed(lambda: fq.fp8_gemm_mx(am, sam, bm, sbm, out=cbuf), 10, stream, flush)
+            ms = ctimed(lambda: fq.fp8_gemm_mx(am, sam, bm, sbm, out=cbuf), 20, flush)
             out["gemm_mx_8b_up_m8192"] = gemm_entry(m, W_SHAPE[0], W_SHAPE[1], ms, am, sam, sbm, cbuf)
+            add_clocks("gemm_mx_8b_up_m8192")
             del cbuf, am, sam, bm, sbm
             # decode: back-to-back calls as in a decode step, each on one of four copies of the
             # weight codes (4 x 58.7 MB > L2), so every call streams its weights from HBM
@@ -445,12 +554,13 @@ def supplementary(device, stream, peaks, flush):
                 for i in range(calls):
                     fq.fp8_gemm_blockscaled(a, sa, copies[i % 4], ws, out=cbuf)
 
-            ms = timed_graph(batch, 5, stream, flush) / calls
-            ms_py = timed(batch, 5, stream, flush) / calls
+            ms = ctimed(batch, 20, flush, graph=True) / calls
+            ms_py = timed(batch, 20, stream, flush) / calls
             out["gemm_8b_up_m16"] = gemm_entry(m, W_SHAPE[0], W_SHAPE[1], ms, a, sa, ws, cbuf)
             out["gemm_8b_up_m16"]["timing"] = (f"{calls} back-to-back calls over 4 weight copies replayed from a "
-                                               f"CUDA graph, mean per call")
+                                               f"CUDA graph, median per call")
             out["gemm_8b_up_m16"]["python_loop_us"] = round(ms_py * 1e3, 2)
+            add_clocks("gemm_8b_up_m16")
             # the same decode GEMM from bf16 activations: the caller's two calls, and the linear
             # entry point (the same two kernels as one call)
             xb = dev_bf16(synth.activations(seed=1)[:m], device)
@@ -466,11 +576,12 @@ def supplementary(device, stream, peaks, flush):
                 for i in range(calls):
                     fq.fp8_linear_dynamic(xb, copies[i % 4], ws, out=cbuf, act_ws=act_ws)
 
-            ms2 = timed_graph(two_step, 5, stream, flush) / calls
-            ms3 = timed_graph(fused, 5, stream, flush) / calls
+            ms2 = ctimed(two_step, 20, flush, graph=True) / calls
+            ms3 = ctimed(fused, 20, flush, graph=True) / calls
             out["linear_8b_m16_quantize_then_gemm"] = gemm_entry(m, W_SHAPE[0], W_SHAPE[1], ms2, a, sa, ws, cbuf)
             out["linear_8b_m16_dynamic"] = gemm_entry(m, W_SHAPE[0], W_SHAPE[1], ms3, a, sa, ws, cbuf)
             out["linear_8b_m16_dynamic"]["timing"] = "bf16 activations in; same batching and graph replay as gemm_8b_up_m16"
+            add_clocks("linear_8b_m16_dynamic")
             del copies, cbuf
             # decode on the 70B up-projection (one weight, 235 MB > L2)
             w70 = dev_bf16(synth.weight_70b(seed=4, which="up"), device)
@@ -487,10 +598,11 @@ def supplementary(device, stream, peaks, flush):
                 for _ in range(calls):
                     fq.fp8_gemm_blockscaled(a70, sa70, b70, s70, out=c70)
 
-            ms = timed_graph(batch70, 5, stream, flush) / calls
+            ms = ctimed(batch70, 20, flush, graph=True) / calls
             out["gemm_70b_up_m64"] = gemm_entry(64, b70.shape[0], b70.shape[1], ms, a70, sa70, s70, c70)
             out["gemm_70b_up_m64"]["timing"] = (f"{calls} back-to-back calls (weight 235 MB > L2) replayed from a CUDA "
-                                                f"graph, mean per call")
+                                                f"graph, median per call")
+            add_clocks("gemm_70b_up_m64")
             del a70, sa70, c70
             # prefill on the 70B up and down projections (M = 16384), block-scaled and per-tensor
             for which in ("up", "down"):
@@ -506,19 +618,22 @@ def supplementary(device, stream, peaks, flush):
                 del x70
                 c70 = torch.empty((16384, b70.shape[0]), dtype=torch.bfloat16, device=device)
                 fq.fp8_gemm_blockscaled(a70, sa70, b70, s70, out=c70)
-                ms = timed(lambda: fq.fp8_gemm_blockscaled(a70, sa70, b70, s70, out=c70), 3, stream, flush)
+                ms = ctimed(lambda: fq.fp8_gemm_blockscaled(a70, sa70, b70, s70, out=c70), 20, flush)
                 out[f"gemm_70b_{which}_m16384"] = gemm_entry(16384, b70.shape[0], b70.shape[1], ms, a70, sa70, s70, c70)
+                add_clocks(f"gemm_70b_{which}_m16384")
                 if which == "up":
                     one = torch.ones(1, dtype=torch.float32, device=device)
                     fq.fp8_gemm_blockscaled(a70, one, b70, one, fq.PER_TENSOR, fq.PER_TENSOR, out=c70)
-                    ms = timed(lambda: fq.fp8_gemm_blockscaled(a70, one, b70, one, fq.PER_TENSOR, fq.PER_TENSOR,
-                                                               out=c70), 3, stream, flush)
+                    ms = ctimed(lambda: fq.fp8_gemm_blockscaled(a70, one, b70, one, fq.PER_TENSOR, fq.PER_TENSOR,
+                                                                out=c70), 20, flush)
                     out["gemm_70b_up_m16384_per_tensor"] = gemm_entry(16384, b70.shape[0], b70.shape[1], ms, a70, one,
                                                                       one, c70)
+                    add_clocks("gemm_70b_up_m16384_per_tensor")
                     fq.fp8_gemm_mx(a70m, sa70m, b70m, s70m, out=c70)
-                    ms = timed(lambda: fq.fp8_gemm_mx(a70m, sa70m, b70m, s70m, out=c70), 3, stream, flush)
+                    ms = ctimed(lambda: fq.fp8_gemm_mx(a70m, sa70m, b70m, s70m, out=c70), 20, flush)
                     out["gemm_mx_70b_up_m16384"] = gemm_entry(16384, b70.shape[0], b70.shape[1], ms, a70m, sa70m,
                                                               s70m, c70)
+                    add_clocks("gemm_mx_70b_up_m16384")
                     del a70m, sa70m, b70m, s70m
                 del a70, sa70, c70
             del b70, s70
@@ -549,6 +664,8 @@ def our_arm(args):
     fq.lib()
     peaks = load_peaks()
     stream = torch.cuda.Stream(device)
+    sampler = ClockSampler(gpu_identity(device))
+    sampler.start()
 
     # inputs: N_SETS rotating copies of the weight and activations
     w_np = synth.weight_8b(seed=1)
@@ -572,21 +689,12 @@ def our_arm(args):
         flush_buf.zero_()
         flush_rd.sum()
 
-    n_ev = min(args.steps, 2000)
-    every = max(1, args.steps // n_ev)
-    ev_s = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_ev)]
     jobs = [[(W[j], fq.BLOCK_128x128, WC[j], WS[j]), (X[j], fq.GROUP_1x128, XC[j], XS[j])] for j in range(N_SETS)]
 
-    def step(i, rec=None):
+    def step(i):
         # both tensors in one launch (fp8_quantize_many)
-        if rec is not None:
-            rec[0].record(stream)
         fq.fp8_quantize_many(jobs[i % N_SETS], fq.E4M3)
-        if rec is not None:
-            rec[1].record(stream)
 
-    sampler = ClockSampler(gpu_identity(device))
-    sampler.start()
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
             step(i)
@@ -595,27 +703,37 @@ def our_arm(args):
         torch.cuda.synchronize(device)
         t_start = torch.cuda.Event(enable_timing=True)
         t_end = torch.cuda.Event(enable_timing=True)
-        wall0 = time.time()
+        # the GPU sleeps (outside the timed region) while the host queues the start event and
+        # the steps behind it, so the region measures the kernels, not the host's launch rate
+        torch.cuda._sleep(int(min(2e9, 2e6 + 40e3 * args.steps)))
         t_start.record(stream)
-        used = 0
         for i in range(args.steps):
-            rec = None
-            if i % every == 0 and used < n_ev:
-                rec = ev_s[used]
-                used += 1
-            step(i, rec)
+            step(i)
         t_end.record(stream)
+        t_start.synchronize()
+        wall0 = time.time()
         torch.cuda.synchronize(device)
         wall1 = time.time()
         barrier()
-    sampler.stop()
     ms_total = reduce_max(t_start.elapsed_time(t_end), device)
     ms_step = ms_total / max(args.steps, 1)
     value = job_throughput_gbs(step_bytes, args.steps, world, ms_total)
-    s_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_s[:used])
+    s_ms = ms_step
+    # the timed region is shorter than nvidia-smi's sampling interval at small step counts:
+    # also sample a longer run of the same steps right after it (reported beside it)
+    with torch.cuda.stream(stream):
+        n_long = max(args.steps, int(300.0 / max(ms_step, 1e-3)))
+        torch.cuda._sleep(int(2e6))
+        wl0 = time.time()
+        for i in range(n_long):
+            step(i)
+        torch.cuda.synchronize(device)
+        wl1 = time.time()
     clocks = sampler.summary(wall0, wall1)
+    clocks["same_steps_300ms"] = sampler.summary(wl0, wl1)
 
     if args.skip_extras:
+        sampler.stop()
         if rank == 0:
             print(json.dumps({"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
                               "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
@@ -699,8 +817,11 @@ def our_arm(args):
                          "frac": round(achieved / peak, 4), "traffic": traffic,
                          "kernel": "k_quant_many (the step: 128x128 weight blocks + 1x128 activation groups, "
                                    "one launch)", "bytes_per_launch": step_bytes,
+                         "launch_us": round(s_ms * 1e3, 2),
+                         "timing": "CUDA events around the timed region on the launching stream, which holds "
+                                   "exactly one launch of this kernel per step: mean launch duration = "
+                                   "region time / steps",
                          "peak_source": f"{peaks['source']} hbm_gbs"},
-            "kernels": {"quant_step_one_launch": {"us": round(s_ms * 1e3, 2), "GB/s": round(achieved, 1)}},
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": args.steps,
             "clocks": clocks,
@@ -724,8 +845,9 @@ def our_arm(args):
     del W, X, WC, XC, WS, XS, jobs
     if rank == 0 and world == 1:
         if not args.no_supplementary:
-            result["supplementary"] = supplementary(device, stream, peaks, flush)
+            result["supplementary"] = supplementary(device, stream, peaks, flush, sampler)
         result["cpu_baseline"] = cpu_baseline_leg()
+    sampler.stop()
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
@@ -790,7 +912,7 @@ def profile_target(name, reps):
             fn = lambda: fq.fp8_dequantize(wc, ws, fq.E4M3, fq.BLOCK_128x128, out=y)  # noqa: E731
         for _ in range(2):
             fn()
-        ms = timed(fn, max(reps, 1), stream)
+        ms = timed(fn, max(reps, 1), stream, min_reps=1)
     print(json.dumps({"profile_target": name, "reps": reps, "ms": round(ms, 4)}), flush=True)
     return 0 if fq.device_status() == 0 else 1
 
