@@ -2,9 +2,13 @@
 
 Loads fp8_oracle.c (plain C, built with gcc here) through ctypes.  Only the
 test suite, the smoke check and the benchmark's CPU-baseline leg may import
-this package; the GPU library never does.  The wrappers only marshal numpy
-arrays and split independent scale groups across threads (ctypes releases the
-GIL during a foreign call); all arithmetic happens in the C file.
+this package; the GPU library never does.  The wrappers marshal numpy arrays
+and split independent scale groups across threads (ctypes releases the GIL
+during a foreign call); every value the method computes (codes, scales, decoded
+values, products, counts) is computed in the C file.  Two wrappers are layout
+permutations written here in numpy index arithmetic and nothing else:
+mx_blocked_scales (the blocked MX scale layout) and pack_b_tiles (the packed
+weight-tile layout), each pinned by hand-worked byte positions.
 
 Every function cites the page passage it follows in fp8_oracle.c; the pins
 that check it against the pages live in tests/test_oracle_*.py.

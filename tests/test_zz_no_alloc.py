@@ -42,7 +42,8 @@ def test_noalloc_matches_workspace_entry_point_twice():
     L = fq.lib()
     assert fq.device_status() == 0
     cases = [((4096, 8, 128), 3, fq.KV_PER_HEAD, fq.E4M3),      # first call: per-head E4M3
-             ((3000, 8, 128), 5, fq.KV_PER_TENSOR, fq.E5M2)]     # second call: other data, per-tensor E5M2
+             ((3000, 8, 128), 5, fq.KV_PER_TENSOR, fq.E5M2),     # second call: other data, per-tensor E5M2
+             ((1000, 8, 128), 7, fq.KV_PER_HEAD_TOK128, fq.E4M3)]  # one-pass granularity: no scratch used
     for shape, seed, gran, fmt in cases:
         T, H, D = shape
         k_np, v_np = synth.kv_70b(seed=seed, tokens=T, heads=H, head_dim=D)
