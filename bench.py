@@ -495,9 +495,8 @@ def supplementary(device, stream, peaks, flush, sampler):
                      xa.numel() * 3 + ms_.numel())
         del xa, mc, ms_, ymx, mcs, ymxs
         # GEMM (8B up-proj shape) on the quantized config-1 operands
-        x = dev_bf16(synth.activations(seed=1), device)
-        xc, xs = fq.fp8_quantize(x, fq.E4M3, fq.GROUP_1x128)
-        del x
+        x8 = dev_bf16(synth.activations(seed=1), device)
+        xc, xs = fq.fp8_quantize(x8, fq.E4M3, fq.GROUP_1x128)
 
         def gemm_entry(m, n, k, ms, a, sa, wscale, c):
             flops = 2.0 * m * n * k
@@ -517,6 +516,16 @@ def supplementary(device, stream, peaks, flush, sampler):
             ms = ctimed(lambda: fq.fp8_gemm_blockscaled(a, sa, wc, ws, out=cbuf), 20, flush)
             out["gemm_8b_up_m8192"] = gemm_entry(m, W_SHAPE[0], W_SHAPE[1], ms, a, sa, ws, cbuf)
             add_clocks("gemm_8b_up_m8192")
+            # the prefill linear layer from bf16 activations (1x128 quantizer, then the GEMM: two
+            # dependent launches), beside the quantizer alone: the most any fusion of the two saves
+            act8 = torch.empty(fq.linear_act_workspace_bytes(m, W_SHAPE[1]), dtype=torch.uint8, device=device)
+            ms_lin = ctimed(lambda: fq.fp8_linear_dynamic(x8, wc, ws, out=cbuf, act_ws=act8), 20, flush)
+            ms_q1 = timed(lambda: fq.fp8_quantize(x8, fq.E4M3, fq.GROUP_1x128, codes=a, scales=sa), 20, stream, flush)
+            out["linear_8b_m8192_dynamic"] = gemm_entry(m, W_SHAPE[0], W_SHAPE[1], ms_lin, a, sa, ws, cbuf)
+            out["linear_8b_m8192_dynamic"].update({"gemm_alone_us": round(ms * 1e3, 2),
+                                                   "quantize_alone_us": round(ms_q1 * 1e3, 2)})
+            add_clocks("linear_8b_m8192_dynamic")
+            del act8
             # the same GEMM with C quantized to E4M3 1x128 groups in the epilogue, against the two
             # steps it replaces (bf16 C, then the 1x128 quantizer)
             qc = torch.empty((m, W_SHAPE[0]), dtype=torch.uint8, device=device)
@@ -582,7 +591,7 @@ def supplementary(device, stream, peaks, flush, sampler):
             out["linear_8b_m16_dynamic"] = gemm_entry(m, W_SHAPE[0], W_SHAPE[1], ms3, a, sa, ws, cbuf)
             out["linear_8b_m16_dynamic"]["timing"] = "bf16 activations in; same batching and graph replay as gemm_8b_up_m16"
             add_clocks("linear_8b_m16_dynamic")
-            del copies, cbuf
+            del copies, cbuf, x8
             # decode on the 70B up-projection (one weight, 235 MB > L2)
             w70 = dev_bf16(synth.weight_70b(seed=4, which="up"), device)
             b70, s70 = fq.fp8_quantize(w70, fq.E4M3, fq.BLOCK_128x128)
@@ -615,12 +624,24 @@ def supplementary(device, stream, peaks, flush, sampler):
                 a70, sa70 = fq.fp8_quantize(x70, fq.E4M3, fq.GROUP_1x128)
                 if which == "up":
                     a70m, sa70m = fq.fp8_quantize_mx_blocked(x70)
-                del x70
                 c70 = torch.empty((16384, b70.shape[0]), dtype=torch.bfloat16, device=device)
                 fq.fp8_gemm_blockscaled(a70, sa70, b70, s70, out=c70)
                 ms = ctimed(lambda: fq.fp8_gemm_blockscaled(a70, sa70, b70, s70, out=c70), 20, flush)
                 out[f"gemm_70b_{which}_m16384"] = gemm_entry(16384, b70.shape[0], b70.shape[1], ms, a70, sa70, s70, c70)
                 add_clocks(f"gemm_70b_{which}_m16384")
+                if which == "up":
+                    act70 = torch.empty(fq.linear_act_workspace_bytes(16384, b70.shape[1]), dtype=torch.uint8,
+                                        device=device)
+                    ms_lin = ctimed(lambda: fq.fp8_linear_dynamic(x70, b70, s70, out=c70, act_ws=act70), 20, flush)
+                    ms_q1 = timed(lambda: fq.fp8_quantize(x70, fq.E4M3, fq.GROUP_1x128, codes=a70, scales=sa70), 20,
+                                  stream, flush)
+                    out["linear_70b_up_m16384_dynamic"] = gemm_entry(16384, b70.shape[0], b70.shape[1], ms_lin, a70,
+                                                                     sa70, s70, c70)
+                    out["linear_70b_up_m16384_dynamic"].update({"gemm_alone_us": round(ms * 1e3, 2),
+                                                                "quantize_alone_us": round(ms_q1 * 1e3, 2)})
+                    add_clocks("linear_70b_up_m16384_dynamic")
+                    del act70
+                del x70
                 if which == "up":
                     one = torch.ones(1, dtype=torch.float32, device=device)
                     fq.fp8_gemm_blockscaled(a70, one, b70, one, fq.PER_TENSOR, fq.PER_TENSOR, out=c70)
@@ -721,16 +742,17 @@ def our_arm(args):
     s_ms = ms_step
     # the timed region is shorter than nvidia-smi's sampling interval at small step counts:
     # also sample a longer run of the same steps right after it (reported beside it)
-    with torch.cuda.stream(stream):
-        n_long = max(args.steps, int(300.0 / max(ms_step, 1e-3)))
-        torch.cuda._sleep(int(2e6))
-        wl0 = time.time()
-        for i in range(n_long):
-            step(i)
-        torch.cuda.synchronize(device)
-        wl1 = time.time()
     clocks = sampler.summary(wall0, wall1)
-    clocks["same_steps_300ms"] = sampler.summary(wl0, wl1)
+    if not args.skip_extras:
+        with torch.cuda.stream(stream):
+            n_long = max(args.steps, int(300.0 / max(ms_step, 1e-3)))
+            torch.cuda._sleep(int(2e6))
+            wl0 = time.time()
+            for i in range(n_long):
+                step(i)
+            torch.cuda.synchronize(device)
+            wl1 = time.time()
+        clocks["same_steps_300ms"] = sampler.summary(wl0, wl1)
 
     if args.skip_extras:
         sampler.stop()
