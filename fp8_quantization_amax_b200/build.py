@@ -88,13 +88,25 @@ def build(force: bool = False, verbose: bool = False) -> str:
 
     with ThreadPoolExecutor(max(1, min(len(sources), os.cpu_count() or 1))) as ex:
         objs = list(ex.map(compile_one, sources))
-    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs):
+    # the objects the library was last linked from: a source removed or added relinks it even
+    # when every remaining object is older than the library
+    stamp = os.path.join(BUILD, "linked_objects.txt")
+    listing = "\n".join(os.path.basename(o) for o in objs)
+    try:
+        with open(stamp) as f:
+            same_objects = f.read() == listing
+    except OSError:
+        same_objects = False
+    if (force or not same_objects or not os.path.exists(LIB)
+            or os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs)):
         tmp = LIB + f".tmp{os.getpid()}"
         cmd = [nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
         os.replace(tmp, LIB)
+        with open(stamp, "w") as f:
+            f.write(listing)
     return LIB
 
 
