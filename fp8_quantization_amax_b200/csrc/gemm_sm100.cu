@@ -523,6 +523,16 @@ __host__ __device__ __forceinline__ bool last_seg_finishes_shared(uint32_t lo, u
   return (lo <= ((hi - 1) / nkb) * nkb) && hi % nkb != 0;
 }
 
+// CTAs for `tiles` weight tiles of nkb units on `sms` SMs.  When whole tiles keep at least three
+// quarters of the SMs busy, each CTA takes exactly one tile and no tile is shared (the split-tile
+// hand-off measured 3.8 us of a 16.5 us call at the 8B shape, 112 tiles); otherwise the units are
+// spread evenly over all SMs, ranges crossing tile boundaries.
+__host__ __device__ __forceinline__ uint32_t decode_ctas(uint32_t tiles, uint32_t nkb, uint32_t sms) {
+  if (tiles <= sms && 4u * tiles >= 3u * sms) return tiles;
+  const uint32_t W = tiles * nkb;
+  return W < sms ? W : sms;
+}
+
 // the CTA whose range holds unit u
 __host__ __device__ __forceinline__ uint32_t cta_of(uint32_t u, uint32_t W, uint32_t G) {
   uint32_t c = (u * G) / W;
@@ -1054,7 +1064,7 @@ DecodePlan decode_plan_uncached(int64_t M, int64_t N, int64_t K) {
   const int64_t nkb = K / 128, tiles = N / 128;
   if ((uint64_t)tiles * nkb * (uint64_t)std::max(1, device_sm_count()) >= (1ull << 32)) return d;
   d.W = (uint32_t)(tiles * nkb);
-  d.G = (int)std::min<int64_t>(device_sm_count(), d.W);
+  d.G = (int)gemm::dec::decode_ctas((uint32_t)tiles, (uint32_t)nkb, (uint32_t)std::max(1, device_sm_count()));
   for (int c = 0; c < d.G; ++c) {
     const uint32_t lo = gemm::dec::range_lo(c, d.W, d.G), hi = gemm::dec::range_lo(c + 1, d.W, d.G);
     if (hi > lo) d.maxseg = std::max<int>(d.maxseg, (int)((hi - 1) / nkb - lo / nkb + 1));
@@ -1135,7 +1145,10 @@ cudaError_t launch_decode_gemm(const DecodePlan& plan, const uint8_t* A, const f
   d.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + plan.counter_bytes);
   d.C = C;
   d.stage_bytes = kStageW + (uint32_t)plan.mp * BK;
-  const uint32_t budget = ctas_per_sm(plan.mp) == 2 ? kHalfSmStageBytes : kFullSmStageBytes;
+  // half-SM CTAs only when every SM has one: with one whole tile per CTA on fewer CTAs than SMs
+  // the scheduler could put two on one SM, so those take a full SM's stages
+  const bool whole_tiles = (uint32_t)plan.G * (uint32_t)(K / BK) == plan.W;
+  const uint32_t budget = (ctas_per_sm(plan.mp) == 2 && !whole_tiles) ? kHalfSmStageBytes : kFullSmStageBytes;
   d.stages = (int)std::max<uint32_t>(2, std::min<uint32_t>(kMaxStages, budget / d.stage_bytes));
   d.Bp = b_packed ? B : nullptr;
   d.err = device_error_word();
@@ -1159,7 +1172,7 @@ int check_decode_split(int64_t M, int64_t N, int64_t K, int sms) {
   if (M <= 0 || M > gemm::dec::kMaxMp || N <= 0 || K <= 0 || N % 128 != 0 || K % 128 != 0 || sms <= 0) return -1;
   const uint32_t nkb = (uint32_t)(K / 128), tiles = (uint32_t)(N / 128);
   if ((uint64_t)tiles * nkb * (uint64_t)sms >= (1ull << 32)) return -1;
-  const uint32_t W = tiles * nkb, G = std::min<uint32_t>((uint32_t)sms, W);
+  const uint32_t W = tiles * nkb, G = gemm::dec::decode_ctas(tiles, nkb, (uint32_t)sms);
   int maxseg = 0;
   for (uint32_t c = 0; c < G; ++c) {
     const uint32_t lo = range_lo(c, W, G), hi = range_lo(c + 1, W, G);

@@ -155,8 +155,9 @@ def test_gemm_decode_workspace_left_zero(orc):
 def test_gemm_decode_workspace_reused_across_shapes(orc):
     """One zero-filled workspace serves decode calls of different shapes in turn: after each call
     the whole workspace (counters and partial sums) is zero again."""
-    ws = torch.zeros(fq.gemm_workspace_bytes(64, 14336, 4096), dtype=torch.uint8, device="cuda")
-    for (M, N, K) in [(16, 1024, 4096), (64, 2048, 1280), (16, 14336, 4096), (33, 384, 640)]:
+    shapes = [(16, 1024, 4096), (64, 2048, 1280), (16, 14336, 4096), (33, 384, 640)]
+    ws = torch.zeros(max(fq.gemm_workspace_bytes(*s) for s in shapes), dtype=torch.uint8, device="cuda")
+    for (M, N, K) in shapes:
         a, sa, b, sb = operands(orc, M, N, K, 1, 2, seed=M * 7 + N)
         got = fq.fp8_gemm_blockscaled(dev(a), dev(sa), dev(b), dev(sb), 1, 2, ws=ws)
         torch.cuda.synchronize()
