@@ -230,8 +230,9 @@ def _workspace(nbytes: int, device, ws: torch.Tensor | None) -> torch.Tensor | N
     return ws
 
 
-# GEMM workspaces must be zero-filled before their first use and every successful call leaves
-# them zero again, so one zeroed buffer per (device, stream) is kept and grown on demand.
+# A GEMM workspace's counters (its first 64 KB) must be zero before its first use and every
+# successful call leaves them zero again, so one zeroed buffer per (device, stream) is kept and
+# grown on demand.
 _gemm_ws: dict = {}
 
 
@@ -415,9 +416,10 @@ def fp8_gemm_blockscaled(a: torch.Tensor, sa: torch.Tensor, b: torch.Tensor, sb:
                          ws: torch.Tensor | None = None) -> torch.Tensor:
     """C[M][N] (bf16) = block-scaled FP8 product of A [M][K] and B [N][K] (E4M3 codes, K-major).
 
-    Decode shapes (M <= 64) need a workspace.  Without `ws` a zero-filled buffer kept per
-    (device, stream) is used; a caller-provided `ws` must be zero-filled before its first use
-    (every successful call leaves it zero) and not shared by calls that may overlap."""
+    Decode shapes (M <= 64) whose weight tiles are split over several blocks need a workspace.
+    Without `ws` a zero-filled buffer kept per (device, stream) is used; a caller-provided `ws`
+    must have its first 64 KB (the counters) zero before its first use (every successful call
+    leaves them zero) and must not be shared by calls that may overlap."""
     _dev(a, "a", torch.uint8)
     _dev(b, "b", torch.uint8)
     _dev(sa, "sa", torch.float32)

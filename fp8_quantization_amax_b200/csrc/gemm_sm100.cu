@@ -463,8 +463,8 @@ constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + (2 * kStages + 4) *
 //     counts in last (the atomic add that completes the count) sums every partial and stores
 //     the tile with its bookkeeping warp.
 // Both ways add the partials in ascending CTA order starting from the first contributor's, so
-// the output is the same bits whichever CTA finishes.  The finisher clears the partials it read
-// and the counter, so every completed call leaves the whole workspace zero.
+// the output is the same bits whichever CTA finishes.  The finisher resets the tile's counter,
+// so every completed call leaves the counters zero; the partial slots are scratch.
 //   warp 0 TMA producer, warp 1 MMA issuer (four TMEM buffers), warp 2 scale producer,
 //   warps 3-6 promotion, warp 7 split-tile bookkeeping.
 namespace dec {
@@ -494,6 +494,13 @@ __host__ __device__ constexpr int ctas_per_sm(int mp) { return mp <= 16 ? 2 : 1;
 constexpr uint32_t kHalfSmStageBytes = 96u * 1024u;
 constexpr uint32_t kFullSmStageBytes = 200u * 1024u;
 
+// The workspace: per-tile counters in a fixed region at its start, then the partial slots.  Only
+// the counters carry state between calls (zero on entry, reset by every call that completes);
+// the slots are scratch, written by each contributor before anyone reads them.  The fixed
+// region keeps one call's slots clear of another shape's counters when calls of different
+// shapes share a workspace.
+constexpr size_t kCounterRegionBytes = 65536;   // 16384 tiles: N <= 2,097,152
+
 struct Params {
   int M, N, K, nkb;
   uint32_t W;         // units: N / 128 tiles x nkb K blocks
@@ -502,8 +509,8 @@ struct Params {
   const float* sA;
   const float* sB;
   int gA_group, gB_block;
-  uint32_t* counters; // [N / 128]: segments counted in per tile; zero between calls
-  float* partials;    // [G][maxseg][Mp][128]
+  uint32_t* counters; // [N / 128]: segments counted in per tile; zero between calls (null: none shared)
+  float* partials;    // [G][maxseg][Mp][128], scratch
   uint16_t* C;
   int stages;
   uint32_t stage_bytes;
@@ -558,7 +565,7 @@ __device__ __forceinline__ float* partial_slot(const Params& p, int mp, uint32_t
 // One warp finishes tile t once every contributor c_first..c_last has published its partial:
 // lane l owns rows 4l..4l+3; the partials are added in ascending CTA order starting from
 // c_first's (the order the promotion warps use when c_first finishes the tile itself), rounded
-// to bf16 and stored; then the partials are cleared and the tile's counter reset.
+// to bf16 and stored; then the tile's counter is reset (the partial slots are scratch).
 template <int MP>
 __device__ __forceinline__ void finish_tile_warp(const Params& p, uint32_t t, uint32_t c_first, uint32_t c_last,
                                               int lane) {
@@ -591,13 +598,6 @@ __device__ __forceinline__ void finish_tile_warp(const Params& p, uint32_t t, ui
         *reinterpret_cast<uint2*>(p.C + (size_t)m * p.N + (size_t)t * BM + r0) = v;
       }
     }
-  }
-  const float4 zero = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-#pragma unroll 1
-  for (uint32_t c = c_first; c <= c_last; ++c) {
-    float* dst = partial_slot(p, MP, c, t) + r0;
-#pragma unroll 4
-    for (int m = 0; m < MP; ++m) *reinterpret_cast<float4*>(dst + (size_t)m * BM) = zero;
   }
   __syncwarp();
   if (lane == 0) p.counters[t] = 0;
@@ -988,7 +988,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(MP)) k_decode_mma(const 
           // this CTA started the tile and a higher one ends it (always this CTA's last segment):
           // the bookkeeping warp decides, without waiting for the other CTAs, whether they are
           // all in.  If so, add their partials to this row in ascending CTA order (the order the
-          // bookkeeping warp of whichever CTA finishes uses too) and clear them; if not, publish
+          // bookkeeping warp of whichever CTA finishes uses too); if not, publish
           // this row's partial for the CTA that counts in last.
           __syncwarp();
           if (lane == 0) mbar_arrive(at_end);
@@ -1014,10 +1014,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(MP)) k_decode_mma(const 
 #pragma unroll
                 for (int j = 0; j < 16; ++j) part[j] = __ldcg(src + (size_t)(m0 + j) * BM);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                  acc[m0 + j] += part[j];
-                  src[(size_t)(m0 + j) * BM] = 0.0f;
-                }
+                for (int j = 0; j < 16; ++j) acc[m0 + j] += part[j];
               }
             }
           }
@@ -1062,14 +1059,19 @@ DecodePlan decode_plan_uncached(int64_t M, int64_t N, int64_t K) {
   if (M <= 0 || M > gemm::dec::kMaxMp || N % 128 != 0 || K % 128 != 0 || N == 0 || K == 0) return d;
   d.mp = (int)((M + 15) / 16 * 16);
   const int64_t nkb = K / 128, tiles = N / 128;
-  if ((uint64_t)tiles * nkb * (uint64_t)std::max(1, device_sm_count()) >= (1ull << 32)) return d;
+  if ((uint64_t)tiles * nkb * (uint64_t)std::max(1, device_sm_count()) >= (1ull << 32) ||
+      tiles > (int64_t)(gemm::dec::kCounterRegionBytes / sizeof(uint32_t))) {
+    d.mp = 0;   // not a decode shape: the prefill kernel takes it
+    return d;
+  }
   d.W = (uint32_t)(tiles * nkb);
   d.G = (int)gemm::dec::decode_ctas((uint32_t)tiles, (uint32_t)nkb, (uint32_t)std::max(1, device_sm_count()));
   for (int c = 0; c < d.G; ++c) {
     const uint32_t lo = gemm::dec::range_lo(c, d.W, d.G), hi = gemm::dec::range_lo(c + 1, d.W, d.G);
     if (hi > lo) d.maxseg = std::max<int>(d.maxseg, (int)((hi - 1) / nkb - lo / nkb + 1));
   }
-  d.counter_bytes = ((size_t)tiles * sizeof(uint32_t) + 255) / 256 * 256;
+  if ((uint64_t)d.G * nkb == d.W) return d;   // one whole tile per CTA: nothing shared, no workspace
+  d.counter_bytes = gemm::dec::kCounterRegionBytes;
   d.ws_bytes = d.counter_bytes + (size_t)d.G * d.maxseg * d.mp * gemm::dec::BM * sizeof(float);
   return d;
 }
@@ -1121,7 +1123,7 @@ cudaError_t launch_decode_gemm(const DecodePlan& plan, const uint8_t* A, const f
                                void* ws, size_t ws_bytes, cudaStream_t st) {
   using namespace gemm::dec;
   using gemm::BK;
-  if (!ws || ws_bytes < plan.ws_bytes) return cudaErrorInvalidValue;
+  if (plan.ws_bytes > 0 && (!ws || ws_bytes < plan.ws_bytes)) return cudaErrorInvalidValue;
   CUtensorMap mW, mX;
   std::memset(&mW, 0, sizeof(mW));
   std::memset(&mX, 0, sizeof(mX));
@@ -1141,8 +1143,8 @@ cudaError_t launch_decode_gemm(const DecodePlan& plan, const uint8_t* A, const f
   d.sB = sB;
   d.gA_group = gA == 1;
   d.gB_block = gB == 2;
-  d.counters = static_cast<uint32_t*>(ws);
-  d.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + plan.counter_bytes);
+  d.counters = plan.ws_bytes > 0 ? static_cast<uint32_t*>(ws) : nullptr;
+  d.partials = plan.ws_bytes > 0 ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + plan.counter_bytes) : nullptr;
   d.C = C;
   d.stage_bytes = kStageW + (uint32_t)plan.mp * BK;
   // half-SM CTAs only when every SM has one: with one whole tile per CTA on fewer CTAs than SMs
@@ -1170,6 +1172,7 @@ int check_decode_split(int64_t M, int64_t N, int64_t K, int sms) {
   using gemm::dec::cta_of;
   using gemm::dec::range_lo;
   if (M <= 0 || M > gemm::dec::kMaxMp || N <= 0 || K <= 0 || N % 128 != 0 || K % 128 != 0 || sms <= 0) return -1;
+  if (N / 128 > (int64_t)(gemm::dec::kCounterRegionBytes / sizeof(uint32_t))) return -1;
   const uint32_t nkb = (uint32_t)(K / 128), tiles = (uint32_t)(N / 128);
   if ((uint64_t)tiles * nkb * (uint64_t)sms >= (1ull << 32)) return -1;
   const uint32_t W = tiles * nkb, G = gemm::dec::decode_ctas(tiles, nkb, (uint32_t)sms);

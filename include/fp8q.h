@@ -343,10 +343,13 @@ FP8Q_API fp8q_status fp8_kv_quantize_delayed(const void *k, const void *v, int64
  * is correct however many of its blocks the device runs at once (other streams' kernels, MPS
  * or a partitioned device taking SMs make it slower, not wrong).  ws: caller-owned device
  * memory of at least fp8q_gemm_workspace_bytes(M, N, K) bytes, 16-byte aligned (else
- * FP8Q_ERR_WORKSPACE), which must be ZERO-FILLED before its first use; every call that runs
- * to completion leaves all of it zero-filled again (counters and partial sums), so it can be
- * reused as is, by calls of any shape.  After a device error
- * (fp8q_device_status() != 0) zero it again.  Calls that may run concurrently (e.g. on
+ * FP8Q_ERR_WORKSPACE).  Its first 65536 bytes hold per-tile counters and must be ZERO-FILLED
+ * before its first use; every call that runs to completion leaves them zero again, so the
+ * workspace can be reused as is, by calls of any shape (the rest is scratch that each call
+ * writes before reading).  After a device error (fp8q_device_status() != 0) zero the counters
+ * again.  The size is 0 (ws may be NULL) when each block of the call holds whole weight tiles
+ * (the 8B shapes on a full B200) and for M > 64; decode shapes with more than 16384 weight
+ * tiles (N > 2,097,152) run on the prefill kernel and need none either.  Calls that may run concurrently (e.g. on
  * unordered streams) need separate workspaces.  Detection of a workspace that was not zero is
  * best effort: a tile counter at or above the tile's number of contributors raises device error
  * bit 1 and leaves that tile unwritten; a smaller stale count may go unseen and leave the tile
@@ -392,9 +395,8 @@ FP8Q_API fp8q_status fp8_count_underflow(const void *x, const uint8_t *codes, in
  *   A, sA, gA, B, sB, gB, M, N, K  as fp8_gemm_blockscaled
  *   codes   uint8 [M][N] (device, 16-byte aligned, written)
  *   scales  fp32 [N/128][M] (device, written): the 1x128 layout of fp8_quantize
- * Prefill shapes only: M must exceed 64 (decode shapes, which fp8q_gemm_workspace_bytes gives a
- * workspace, return FP8Q_ERR_UNSUPPORTED: quantize their bf16 output with fp8_quantize).  No
- * workspace.
+ * Prefill shapes only: M must exceed 64 (decode shapes, M <= 64, return FP8Q_ERR_UNSUPPORTED:
+ * quantize their bf16 output with fp8_quantize).  No workspace.
  */
 FP8Q_API fp8q_status fp8_gemm_blockscaled_to_fp8(const uint8_t *A, const float *sA, fp8q_granularity gA,
                                                  const uint8_t *B, const float *sB, fp8q_granularity gB,

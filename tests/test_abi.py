@@ -58,10 +58,15 @@ def test_sizes(L):
     assert fq.kv_num_scales(131072, 8, fq.KV_PER_TENSOR) == 1
     assert fq.kv_workspace_bytes(131072, 8, 128, fq.KV_PER_HEAD_TOK128) == 0
     assert fq.kv_workspace_bytes(131072, 8, 128, fq.KV_PER_HEAD) >= fq.kv_workspace_bytes(131072, 8, 128, fq.KV_PER_TENSOR)
-    # decode shapes (M <= 64) keep fp32 partial sums in the workspace; larger M needs none
-    assert fq.gemm_workspace_bytes(16, 14336, 4096) >= 16 * 14336 * 4
-    assert fq.gemm_workspace_bytes(64, 128, 128) == 256 + 64 * 128 * 4     # tile counters + one partial
+    # decode shapes (M <= 64) whose weight tiles are shared by several CTAs keep per-tile counters
+    # (a fixed 64 KB region) and fp32 partial sums in the workspace (148 SMs when no GPU is
+    # visible); one whole tile per CTA, larger M, or more tiles than the counters hold need none
+    assert fq.gemm_workspace_bytes(16, 2048, 4096) == 65536 + 148 * 2 * 16 * 128 * 4   # two segments a CTA
+    assert fq.gemm_workspace_bytes(64, 2048, 1280) == 65536 + 148 * 1 * 64 * 128 * 4
+    assert fq.gemm_workspace_bytes(16, 14336, 4096) == 0       # 112 tiles: one whole tile per CTA
+    assert fq.gemm_workspace_bytes(64, 128, 128) == 0          # a single unit
     assert fq.gemm_workspace_bytes(65, 14336, 4096) == 0
+    assert fq.gemm_workspace_bytes(16, 128 * 20000, 128) == 0  # 20000 tiles: the prefill kernel
 
 
 P = ctypes.c_void_p
@@ -139,7 +144,7 @@ def test_gemm_rejects(L):
     assert L.fp8_gemm_blockscaled(a, a, 1, a, a, 1, 128, 128, 128, a, None, 0, None) == 1      # gB
     assert L.fp8_gemm_blockscaled(MISALIGNED, a, 1, a, a, 2, 128, 128, 128, a, None, 0, None) == 1
     assert L.fp8_gemm_blockscaled(a, a, 1, a, a, 2, 0, 128, 128, a, None, 0, None) == 0
-    assert L.fp8_gemm_blockscaled(a, a, 1, a, a, 2, 16, 128, 128, a, None, 0, None) == 3        # no workspace
+    assert L.fp8_gemm_blockscaled(a, a, 1, a, a, 2, 16, 2048, 4096, a, None, 0, None) == 3      # no workspace
 
 
 def test_binding_refuses_cpu_tensors():

@@ -154,14 +154,14 @@ def test_gemm_decode_workspace_left_zero(orc):
 
 def test_gemm_decode_workspace_reused_across_shapes(orc):
     """One zero-filled workspace serves decode calls of different shapes in turn: after each call
-    the whole workspace (counters and partial sums) is zero again."""
+    its counter region (the first 64 KB) is zero again; the partial slots behind it are scratch."""
     shapes = [(16, 1024, 4096), (64, 2048, 1280), (16, 14336, 4096), (33, 384, 640)]
     ws = torch.zeros(max(fq.gemm_workspace_bytes(*s) for s in shapes), dtype=torch.uint8, device="cuda")
     for (M, N, K) in shapes:
         a, sa, b, sb = operands(orc, M, N, K, 1, 2, seed=M * 7 + N)
         got = fq.fp8_gemm_blockscaled(dev(a), dev(sa), dev(b), dev(sb), 1, 2, ws=ws)
         torch.cuda.synchronize()
-        assert int(ws.count_nonzero()) == 0, (M, N, K)
+        assert int(ws[:65536].count_nonzero()) == 0, (M, N, K)
         check_tolerance(host(got), orc.gemm_rows(a, sa, 1, b, sb, 2, np.arange(M)), f"{M}x{N}x{K}")
     assert fq.device_status() == 0
 
@@ -172,9 +172,9 @@ def test_gemm_decode_with_sms_taken(orc, M):
     most of an SM's shared memory) holds 64 SMs on one stream while the decode GEMM runs on
     another, so the decode's higher-numbered CTAs can only start once the prefill ends, long after
     the lower ones finished.  Tiles those CTAs share are then completed by whichever CTA counts in
-    last.  The output must equal the idle-GPU result bit for bit, with no device error and the
-    workspace left zero."""
-    N, K = 14336, 4096
+    last.  N = 4096 (32 weight tiles) splits every tile over four to six CTAs.  The output must
+    equal the idle-GPU result bit for bit, with no device error and the counters left zero."""
+    N, K = 4096, 4096
     a, sa, b, sb = operands(orc, M, N, K, 1, 2, seed=17 + M)
     A, SA, B, SB = dev(a), dev(sa), dev(b), dev(sb)
     ws = torch.zeros(fq.gemm_workspace_bytes(M, N, K), dtype=torch.uint8, device="cuda")
@@ -201,7 +201,7 @@ def test_gemm_decode_with_sms_taken(orc, M):
             ev[3].record(s_dec)
         torch.cuda.synchronize()
         assert torch.equal(got.view(torch.int16), want.view(torch.int16))
-        assert int(ws.count_nonzero()) == 0
+        assert int(ws[:65536].count_nonzero()) == 0
         print(f"M={M}: hog {ev[0].elapsed_time(ev[1]) * 1e3:.0f} us, decode {ev[2].elapsed_time(ev[3]) * 1e3:.0f} us")
     assert fq.device_status() == 0
     check_tolerance(host(got), orc.gemm_rows(a, sa, 1, b, sb, 2, np.arange(M)), f"M={M} with SMs taken")
