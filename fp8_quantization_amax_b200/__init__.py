@@ -26,7 +26,7 @@ __all__ = [
     "linear_act_workspace_bytes", "fp8_linear_dynamic", "fp8_quantize_mx", "fp8_dequantize_mx",
     "mx_blocked_scale_bytes", "fp8_quantize_mx_blocked", "fp8_gemm_mx", "fp8_pack_b_tiles",
     "fp8_gemm_blockscaled_packed", "fp8_scale_histogram", "fp8_count_underflow", "fp8_quantize_many",
-    "selftest_wait_timeout", "fp8_gemm_blockscaled_to_fp8",
+    "selftest_wait_timeout", "fp8_gemm_blockscaled_to_fp8", "check_decode_split", "check_tile_walk",
 ]
 
 E4M3, E5M2 = 0, 1
@@ -92,6 +92,8 @@ def lib() -> ctypes.CDLL:
             L.fp8q_selftest_wait_timeout.argtypes = [vp]
             L.fp8q_check_decode_split.argtypes = [i64, i64, i64, i32]
             L.fp8q_check_decode_split.restype = i32
+            L.fp8q_check_tile_walk.argtypes = [i64, i64, i64]
+            L.fp8q_check_tile_walk.restype = i32
             L.fp8_gemm_blockscaled_to_fp8.argtypes = [vp, vp, i32, vp, vp, i32, i64, i64, i64, vp, vp, vp]
             L.fp8_gemm_blockscaled_to_fp8.restype = i32
             L.fp8q_selftest_wait_timeout.restype = i32
@@ -509,6 +511,12 @@ def selftest_wait_timeout(device=None) -> None:
     barrier nothing completes gives up after its time limit and sets bit 0 of device_status()."""
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     _check("fp8q_selftest_wait_timeout", lib().fp8q_selftest_wait_timeout(_stream(dev)))
+
+
+def check_tile_walk(M: int, N: int, K: int) -> int:
+    """Host-only check of the prefill GEMMs' tile walk: 0 when every output tile is visited exactly
+    once (-1: not a prefill shape).  See fp8q_check_tile_walk in include/fp8q.h."""
+    return int(lib().fp8q_check_tile_walk(M, N, K))
 
 
 def check_decode_split(M: int, N: int, K: int, sms: int) -> int:

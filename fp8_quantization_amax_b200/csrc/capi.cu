@@ -57,6 +57,8 @@ fp8q_status fp8q_selftest_wait_timeout(fp8q_stream_t stream) {
   return from_cuda(fp8q::launch_selftest_wait((cudaStream_t)stream));
 }
 
+int fp8q_check_tile_walk(int64_t M, int64_t N, int64_t K) { return fp8q::check_tile_walk(M, N, K); }
+
 int fp8q_check_decode_split(int64_t M, int64_t N, int64_t K, int sms) {
   return fp8q::check_decode_split(M, N, K, sms);
 }

@@ -1221,6 +1221,27 @@ int check_decode_split(int64_t M, int64_t N, int64_t K, int sms) {
   return 0;
 }
 
+// The prefill kernels' tile walk, checked on the host with the kernels' own functions: every tile
+// of the M x N output visited once, every coordinate inside the matrix.
+int check_tile_walk(int64_t M, int64_t N, int64_t K) {
+  using namespace gemm;
+  if (M <= 64 || N <= 0 || K <= 0 || N % 128 != 0 || K % 128 != 0) return -1;
+  const int64_t m_tiles = (M + BM - 1) / BM, n_tiles = (N + BN - 1) / BN;
+  if (m_tiles * n_tiles > (int64_t(1) << 26)) return -1;
+  const int group_m = tile_group_m(M, K, (int)m_tiles);
+  if (group_m < 1 || group_m > m_tiles) return 1;
+  std::vector<uint8_t> seen((size_t)(m_tiles * n_tiles), 0);
+  for (int t = 0; t < (int)(m_tiles * n_tiles); ++t) {
+    int mt, nt;
+    tile_walk(t, (int)m_tiles, (int)n_tiles, group_m, &mt, &nt);
+    if (mt < 0 || mt >= m_tiles || nt < 0 || nt >= n_tiles) return 2;   // outside the matrix
+    uint8_t& v = seen[(size_t)nt * m_tiles + mt];
+    if (v) return 3;                                                      // visited twice
+    v = 1;
+  }
+  return 0;   // tiles visited = tiles in the matrix, none twice: each exactly once
+}
+
 // the prefill kernel (M > 64): C in bf16, or (q_codes non-null) quantized to E4M3 1x128 groups
 static cudaError_t launch_prefill(const uint8_t* A, const float* sA, int gA, const uint8_t* B, bool b_packed,
                                   const float* sB, int gB, int64_t M, int64_t N, int64_t K, uint16_t* C,

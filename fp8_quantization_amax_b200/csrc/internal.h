@@ -125,6 +125,8 @@ cudaError_t launch_pack_b_tiles(const uint8_t* B, int64_t N, int64_t K, uint8_t*
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 // host-only consistency check of the decode split (fp8q_check_decode_split)
 int check_decode_split(int64_t M, int64_t N, int64_t K, int sms);
+// host-only check of the prefill GEMMs' tile walk (fp8q_check_tile_walk)
+int check_tile_walk(int64_t M, int64_t N, int64_t K);
 
 // the same GEMM (prefill shapes, M > 64) with C quantized in the epilogue to E4M3 1x128 groups:
 // codes [M][N], scales [N/128][M]; cudaErrorNotSupported for decode shapes

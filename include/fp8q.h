@@ -134,6 +134,16 @@ FP8Q_API fp8q_status fp8q_selftest_wait_timeout(fp8q_stream_t stream);
  */
 FP8Q_API int fp8q_check_decode_split(int64_t M, int64_t N, int64_t K, int sms);
 
+/*
+ * Host-only self-check of the prefill GEMMs' persistent tile walk (no device work): for an
+ * M x N x K product with M > 64 (128 x 256 output tiles, in the block-scaled, per-tensor and
+ * MXFP8 kernels alike) walks tile indices 0 .. tiles-1 through the kernels' own walk function
+ * (bands of M tiles when A does not fit in L2) and checks that every output tile is visited
+ * exactly once and that every coordinate lies inside the matrix.  Returns 0 when it
+ * holds, a positive code for the first violation, or -1 for a shape that is not a prefill shape.
+ */
+FP8Q_API int fp8q_check_tile_walk(int64_t M, int64_t N, int64_t K);
+
 /* ---------------------------------------------------------------- sizes */
 
 /* Number of fp32 scales fp8_quantize writes for a [rows][cols] tensor; 0 on a bad argument. */
