@@ -341,3 +341,16 @@ def test_gemm_to_fp8_against_oracle_product(orc):
     ref = orc.gemm_rows(a, sa, 1, b, sb, 2, np.arange(M))
     bound = np.abs(ref) * (2.0 ** -4 + 2.0 ** -8 + ELEM) + s_full * 2.0 ** -9 + 1e-2 * 1e-2
     assert np.all(np.abs(got - ref) <= bound)
+
+
+@pytest.mark.parametrize("ga,gb", [(1, 2), (0, 0)])
+def test_gemm_banded_tile_walk_ragged(orc, ga, gb):
+    """A (8320 x 8192 codes, 68 MB) above the L2 budget: tiles walk in bands of 16 M tiles, the
+    last band is one M tile high (65 tiles) and N = 1408 leaves a half-filled 256-column tile.
+    One sampled row per M tile, both scale modes."""
+    M, N, K = 8320, 1408, 8192
+    assert fq.check_tile_walk(M, N, K) == 0
+    a, sa, b, sb = operands(orc, M, N, K, ga, gb, seed=23)
+    got = run_gpu(a, sa, b, sb, ga, gb)
+    rows = sample_rows(M, seed=23)
+    check_tolerance(got[rows], orc.gemm_rows(a, sa, ga, b, sb, gb, rows), f"banded walk gA={ga} gB={gb}")

@@ -160,3 +160,15 @@ def test_gemm_mx_config2_sampled(orc, M):
     got = run_gpu(orc, a, sa, b, sb, 0, 0)
     rows = sample_rows(M, seed=M)
     check_tolerance(got[rows], orc.gemm_mx_rows(a, sa, b, sb, rows), f"M={M} sampled")
+
+
+def test_gemm_mx_banded_tile_walk(orc):
+    """A (8192 x 8192 codes, 64 MB) above the L2 budget, so tiles walk in bands of 16 M tiles;
+    N = 1280 leaves a half-filled 256-column tile in every band.  One sampled row per M tile."""
+    M, N, K = 8192, 1280, 8192
+    assert fq.check_tile_walk(M, N, K) == 0
+    a, sa = orc.quantize_mx(synth.activations(seed=9, m=M, k=K), 0)
+    b, sb = orc.quantize_mx(synth.weight_8b(seed=9, n=N, k=K), 0)
+    got = run_gpu(orc, a, sa, b, sb, 0, 0)
+    rows = sample_rows(M, seed=9)
+    check_tolerance(got[rows], orc.gemm_mx_rows(a, sa, b, sb, rows), "banded walk")
