@@ -526,6 +526,14 @@ def supplementary(device, stream, peaks, flush, sampler):
                                                    "quantize_alone_us": round(ms_q1 * 1e3, 2)})
             add_clocks("linear_8b_m8192_dynamic")
             del act8
+            # the same layer as one cooperative launch (quantize phase, grid barrier, GEMM)
+            actf = torch.zeros(fq.linear_fused_workspace_bytes(m, W_SHAPE[1]), dtype=torch.uint8, device=device)
+            fq.fp8_linear_dynamic_fused(x8, wc, ws, out=cbuf, act_ws=actf)
+            ms_f = ctimed(lambda: fq.fp8_linear_dynamic_fused(x8, wc, ws, out=cbuf, act_ws=actf), 20, flush)
+            out["linear_8b_m8192_fused"] = gemm_entry(m, W_SHAPE[0], W_SHAPE[1], ms_f, a, sa, ws, cbuf)
+            out["linear_8b_m8192_fused"]["two_launch_us"] = round(ms_lin * 1e3, 2)
+            add_clocks("linear_8b_m8192_fused")
+            del actf
             # the same GEMM with C quantized to E4M3 1x128 groups in the epilogue, against the two
             # steps it replaces (bf16 C, then the 1x128 quantizer)
             qc = torch.empty((m, W_SHAPE[0]), dtype=torch.uint8, device=device)
@@ -641,6 +649,15 @@ def supplementary(device, stream, peaks, flush, sampler):
                                                                 "quantize_alone_us": round(ms_q1 * 1e3, 2)})
                     add_clocks("linear_70b_up_m16384_dynamic")
                     del act70
+                    actf = torch.zeros(fq.linear_fused_workspace_bytes(16384, b70.shape[1]), dtype=torch.uint8,
+                                       device=device)
+                    fq.fp8_linear_dynamic_fused(x70, b70, s70, out=c70, act_ws=actf)
+                    ms_f = ctimed(lambda: fq.fp8_linear_dynamic_fused(x70, b70, s70, out=c70, act_ws=actf), 20, flush)
+                    out["linear_70b_up_m16384_fused"] = gemm_entry(16384, b70.shape[0], b70.shape[1], ms_f, a70,
+                                                                   sa70, s70, c70)
+                    out["linear_70b_up_m16384_fused"]["two_launch_us"] = round(ms_lin * 1e3, 2)
+                    add_clocks("linear_70b_up_m16384_fused")
+                    del actf
                 del x70
                 if which == "up":
                     one = torch.ones(1, dtype=torch.float32, device=device)
@@ -901,6 +918,13 @@ def profile_target(name, reps):
             b, sb = fq.fp8_quantize(w, fq.E4M3, fq.BLOCK_128x128)
             c = torch.empty((a.shape[0], b.shape[0]), dtype=torch.bfloat16, device=device)
             fn = lambda: fq.fp8_gemm_blockscaled(a, sa, b, sb, out=c)  # noqa: E731
+        elif name == "linear_fused_8b_m8192":
+            x = dev_bf16(synth.activations(seed=1), device)
+            b, sb = fq.fp8_quantize(dev_bf16(synth.weight_8b(seed=1), device), fq.E4M3, fq.BLOCK_128x128)
+            c = torch.empty((x.shape[0], b.shape[0]), dtype=torch.bfloat16, device=device)
+            actf = torch.zeros(fq.linear_fused_workspace_bytes(x.shape[0], x.shape[1]), dtype=torch.uint8,
+                               device=device)
+            fn = lambda: fq.fp8_linear_dynamic_fused(x, b, sb, out=c, act_ws=actf)  # noqa: E731
         elif name == "gemm_mx_8b_m8192":
             a, sa = fq.fp8_quantize_mx_blocked(dev_bf16(synth.activations(seed=1), device))
             b, sb = fq.fp8_quantize_mx_blocked(dev_bf16(synth.weight_8b(seed=1), device))
@@ -949,7 +973,7 @@ def main():
     ap.add_argument("--skip-extras", action="store_true",
                     help="time the steps only: no e2e, CPU baseline or supplementary kernels (for profiling)")
     ap.add_argument("--profile-target", default=None,
-                    choices=["gemm_8b_m8192", "gemm_8b_m16", "gemm_mx_8b_m8192", "gemm_70b_up_m16384", "gemm_70b_up_m64", "kv_tok128", "kv_head",
+                    choices=["gemm_8b_m8192", "gemm_8b_m16", "linear_fused_8b_m8192", "gemm_mx_8b_m8192", "gemm_70b_up_m16384", "gemm_70b_up_m64", "kv_tok128", "kv_head",
                              "kv_delayed", "mx_8b", "dequant_8b"],
                     help="run one workload a few times and exit (a small target for ncu)")
     args = ap.parse_args()

@@ -23,7 +23,8 @@ __all__ = [
     "kv_workspace_bytes", "gemm_workspace_bytes", "scale_shape", "kv_scale_shape",
     "fp8_encode", "fp8_decode", "fp8_quantize", "fp8_dequantize", "fp8_kv_quantize",
     "fp8_kv_quantize_noalloc", "fp8_gemm_blockscaled", "fp8_quantize_delayed", "fp8_kv_quantize_delayed",
-    "linear_act_workspace_bytes", "fp8_linear_dynamic", "fp8_quantize_mx", "fp8_dequantize_mx",
+    "linear_act_workspace_bytes", "fp8_linear_dynamic", "linear_fused_workspace_bytes", "fp8_linear_dynamic_fused",
+    "fp8_quantize_mx", "fp8_dequantize_mx",
     "mx_blocked_scale_bytes", "fp8_quantize_mx_blocked", "fp8_gemm_mx", "fp8_pack_b_tiles",
     "fp8_gemm_blockscaled_packed", "fp8_scale_histogram", "fp8_count_underflow", "fp8_quantize_many",
     "selftest_wait_timeout", "fp8_gemm_blockscaled_to_fp8", "check_decode_split", "check_tile_walk",
@@ -103,6 +104,9 @@ def lib() -> ctypes.CDLL:
             L.fp8q_linear_act_workspace_bytes.argtypes = [i64, i64]
             L.fp8q_linear_act_workspace_bytes.restype = sz
             L.fp8_linear_dynamic.argtypes = [vp, i64, i64, i64, vp, vp, i32, vp, vp, sz, vp, sz, vp]
+            L.fp8q_linear_fused_workspace_bytes.argtypes = [i64, i64]
+            L.fp8q_linear_fused_workspace_bytes.restype = sz
+            L.fp8_linear_dynamic_fused.argtypes = [vp, i64, i64, i64, vp, vp, i32, vp, vp, sz, vp]
             L.fp8_encode.argtypes = [vp, i64, i32, vp, vp]
             L.fp8_decode.argtypes = [vp, i64, i32, vp, vp]
             L.fp8_quantize.argtypes = [vp, i64, i64, i32, i32, vp, vp, vp, sz, vp]
@@ -115,7 +119,8 @@ def lib() -> ctypes.CDLL:
                                                   vp, vp, sz, vp]
             for fn in ("fp8_encode", "fp8_decode", "fp8_quantize", "fp8_dequantize", "fp8_kv_quantize",
                        "fp8_gemm_blockscaled", "fp8_kv_quantize_noalloc", "fp8_quantize_delayed",
-                       "fp8_kv_quantize_delayed", "fp8_linear_dynamic", "fp8_quantize_mx", "fp8_dequantize_mx",
+                       "fp8_kv_quantize_delayed", "fp8_linear_dynamic", "fp8_linear_dynamic_fused",
+                       "fp8_quantize_mx", "fp8_dequantize_mx",
                        "fp8_quantize_mx_blocked", "fp8_gemm_mx", "fp8_pack_b_tiles",
                        "fp8_gemm_blockscaled_packed", "fp8_scale_histogram", "fp8_count_underflow",
                        "fp8_quantize_many"):
@@ -608,6 +613,37 @@ def fp8_linear_dynamic(x: torch.Tensor, b: torch.Tensor, sb: torch.Tensor, gb: i
     if st != 0 and cached:
         _gemm_ws.clear()
     _check("fp8_linear_dynamic", st)
+    return out
+
+
+def linear_fused_workspace_bytes(M: int, K: int) -> int:
+    return int(lib().fp8q_linear_fused_workspace_bytes(M, K))
+
+
+def fp8_linear_dynamic_fused(x: torch.Tensor, b: torch.Tensor, sb: torch.Tensor, gb: int = BLOCK_128x128,
+                             out: torch.Tensor | None = None, act_ws: torch.Tensor | None = None) -> torch.Tensor:
+    """fp8_linear_dynamic at prefill shapes (M > 64) as one cooperative launch that quantizes x
+    and then runs the GEMM on the codes; output bit-identical to fp8_linear_dynamic.  act_ws
+    (uint8, fp8q_linear_fused_workspace_bytes(M, K) bytes) starts with two grid-barrier words
+    (256 bytes) that must be zero before its first use; a buffer is allocated with them zeroed
+    when not given, and every call that completes leaves them ready for the next call of any
+    shape (the arrival count back at zero)."""
+    _dev(x, "x", torch.bfloat16)
+    _dev(b, "b", torch.uint8)
+    _dev(sb, "sb", torch.float32)
+    M, K = x.shape
+    N, K2 = b.shape
+    if K != K2:
+        raise ValueError("x and b disagree on K")
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if out is None else _dev(out, "out", torch.bfloat16)
+    nbytes = linear_fused_workspace_bytes(M, K)
+    if act_ws is None and nbytes > 0:
+        act_ws = torch.empty(nbytes, dtype=torch.uint8, device=x.device)
+        act_ws[:256].zero_()
+    st = lib().fp8_linear_dynamic_fused(_ptr(x), M, N, K, _ptr(b), _ptr(sb), gb, _ptr(out), _ptr(act_ws),
+                                        0 if act_ws is None else act_ws.numel() * act_ws.element_size(),
+                                        ctypes.c_void_p(_stream_handle(x.device)))
+    _check("fp8_linear_dynamic_fused", st)
     return out
 
 

@@ -402,6 +402,31 @@ fp8q_status fp8_linear_dynamic(const void* X, int64_t M, int64_t N, int64_t K, c
   return from_cuda(e);
 }
 
+size_t fp8q_linear_fused_workspace_bytes(int64_t M, int64_t K) {
+  if (M <= 64 || K <= 0 || K % 128 != 0 || checked_elems(M, K) < 0) return 0;
+  return fp8q::linear_fused_workspace_bytes(M, K);
+}
+
+fp8q_status fp8_linear_dynamic_fused(const void* X, int64_t M, int64_t N, int64_t K, const uint8_t* B, const float* sB,
+                                     fp8q_granularity gB, void* C, void* act_ws, size_t act_ws_bytes,
+                                     fp8q_stream_t stream) {
+  if (M < 0 || N < 0 || K < 0) return FP8Q_ERR_INVALID_ARGUMENT;
+  if (!(gB == FP8Q_BLOCK_128x128 || gB == FP8Q_PER_TENSOR)) return FP8Q_ERR_INVALID_ARGUMENT;
+  if (M == 0 || N == 0) return FP8Q_OK;
+  if (M <= 64) return FP8Q_ERR_UNSUPPORTED;   // decode shapes: fp8_linear_dynamic
+  if (N % 128 != 0 || K % 128 != 0 || K == 0) return FP8Q_ERR_UNSUPPORTED;
+  if (checked_elems(M, K) < 0 || checked_elems(N, K) < 0 || checked_elems(M, N) < 0) return FP8Q_ERR_UNSUPPORTED;
+  if (M > (int64_t(1) << 31) - 1 || N > (int64_t(1) << 31) - 1) return FP8Q_ERR_UNSUPPORTED;
+  if (!X || !B || !C || !sB || !aligned(X, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(sB, 4))
+    return FP8Q_ERR_INVALID_ARGUMENT;
+  if (!act_ws || act_ws_bytes < fp8q::linear_fused_workspace_bytes(M, K) || !aligned(act_ws, 256))
+    return FP8Q_ERR_WORKSPACE;
+  const cudaError_t e = fp8q::launch_linear_fused(static_cast<const uint16_t*>(X), B, sB, gB, M, N, K,
+                                                  static_cast<uint16_t*>(C), act_ws, (cudaStream_t)stream);
+  if (e == cudaErrorNotSupported || e == cudaErrorCooperativeLaunchTooLarge) return FP8Q_ERR_UNSUPPORTED;
+  return from_cuda(e);
+}
+
 fp8q_status fp8_gemm_mx(const uint8_t* A, const uint8_t* sA, fp8q_format fa, const uint8_t* B, const uint8_t* sB,
                         fp8q_format fb, int64_t M, int64_t N, int64_t K, void* C, fp8q_stream_t stream) {
   if (M < 0 || N < 0 || K < 0 || !valid_fmt(fa) || !valid_fmt(fb)) return FP8Q_ERR_INVALID_ARGUMENT;

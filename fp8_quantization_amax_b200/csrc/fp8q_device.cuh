@@ -226,6 +226,31 @@ __device__ __noinline__ uint2 quant8_slow(uint4 v, float d) {
   return make_uint2(c[0], c[1]);
 }
 
+// eight bf16 -> eight codes for a group of the slow path without a division (no call, for kernels
+// whose register budget a call would break).  A scale from a tiny amax (d < 2^-60) is scaled
+// with the elements by 2^100: both products are exact and normal, so x / d = (x 2^100) /
+// (d 2^100) and Markstein's step on the scaled pair is RN(x / d).  d = +inf gives x * 0 (the
+// signed zero for finite x, NaN for +-inf or NaN x) and d = NaN gives NaN, as x / d does.  The
+// scale of delayed scaling (d = 0) is not handled here.
+template <int FMT>
+__device__ __forceinline__ uint2 quant8_nodiv(uint4 v, float d) {
+  const bool tiny = d < 0x1.0p-60f;
+  const bool inf = d == __int_as_float(0x7F800000);
+  const float xs = tiny ? 0x1.0p100f : 1.0f;
+  const float ds = tiny ? d * 0x1.0p100f : d;
+  const float rs = inf ? 0.0f : __frcp_rn(ds);
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t c[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float x0 = bf16_lo(w[i]) * xs, x1 = bf16_hi(w[i]) * xs;
+    const float q0 = inf ? x0 * 0.0f : markstein_div(x0, ds, rs);
+    const float q1 = inf ? x1 * 0.0f : markstein_div(x1, ds, rs);
+    c[i] = cvt2<FMT>(q0, q1);
+  }
+  return make_uint2(__byte_perm(c[0], c[1], 0x5410), __byte_perm(c[2], c[3], 0x5410));
+}
+
 template <int FMT>
 __device__ __forceinline__ uint2 quant8(uint4 v, const GroupScale& g) {
   return g.fast ? quant8_fast<FMT>(v, g.d, g.r) : quant8_slow<FMT>(v, g.d);

@@ -81,6 +81,11 @@ struct Params {
   uint16_t* C;
   uint8_t* q_codes;   // non-null: the output is quantized (E4M3, 1x128 groups) instead of stored as bf16
   float* q_scales;    // [N/128][M]
+  // non-null: a first phase quantizes these bf16 activations [M][K] into the A codes and 1x128
+  // scales the GEMM then reads (xq_codes / sA), behind a grid barrier on gbar (cooperative launch)
+  const uint16_t* xq;
+  uint8_t* xq_codes;
+  uint32_t* gbar;     // [0] arrivals (zero between calls), [1] generation
   uint32_t* err;
 };
 
@@ -114,6 +119,89 @@ __device__ __forceinline__ void store_row_e4m3(PairFn pair, uint8_t* codes_row, 
   *scale = gs.s;
 }
 
+constexpr int kPhaseDepth = 16;
+
+// First phase of the fused linear layer: every warp of the grid quantizes 1x128 groups of the
+// bf16 activations (group g = row g / nkb, K block g % nkb) with the arithmetic of the stand-alone
+// 1x128 kernel; then the grid meets at a barrier (all CTAs are resident: the kernel is launched
+// cooperatively) so no A tile is loaded before every code and scale is written.  Returns false
+// if the barrier's wait gave up (error word set).
+__device__ __forceinline__ bool quantize_phase(const uint16_t* __restrict__ xq, uint8_t* __restrict__ xq_codes,
+                                             float* __restrict__ sA, uint32_t M, uint32_t K, uint32_t* gbar,
+                                             uint32_t* err) {
+  __shared__ uint32_t s_flag_bar;
+  const uint32_t nkb = K / 128u;
+  const uint32_t groups = M * nkb;   // < 2^31 (checked by the launcher)
+  // a half-warp per group, a lane per 16 bytes (8 elements): every load and store of a warp is
+  // 512 contiguous bytes of two groups of one row.  A warp's work item is a run of up to
+  // 2 * kPhaseDepth groups of one row, all loaded before the first is quantized.
+  const uint32_t lane = threadIdx.x & 31u, half = lane >> 4, hl = lane & 15u;
+  const uint32_t warps = gridDim.x * (blockDim.x >> 5);
+  const uint32_t runs = (nkb + 2u * kPhaseDepth - 1u) / (2u * kPhaseDepth);   // runs per row
+  const uint32_t items = M * runs;
+  for (uint32_t item = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); item < items; item += warps) {
+    const uint32_t m = item / runs, kb0 = (item - m * runs) * (2u * kPhaseDepth) + half;
+    const uint16_t* row = xq + (size_t)m * K + hl * 8;
+    uint8_t* crow = xq_codes + (size_t)m * K + hl * 8;
+    uint4 v[kPhaseDepth];
+#pragma unroll
+    for (int u = 0; u < kPhaseDepth; ++u) {
+      const uint32_t kb = kb0 + 2u * u;
+      v[u] = kb < nkb ? ld_stream_v4(row + (size_t)kb * 128) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < kPhaseDepth; ++u) {
+      const uint32_t kb = kb0 + 2u * u;
+      uint32_t mx = absmax_v4(0u, v[u]);
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) mx = absmax2(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+      const GroupScale gs = make_group_scale<kE4M3>(packed_amax_to_f32(mx));
+      const uint2 q = gs.fast ? quant8_fast<kE4M3>(v[u], gs.d, gs.r) : quant8_nodiv<kE4M3>(v[u], gs.d);
+      if (kb < nkb) {
+        st_v2(crow + (size_t)kb * 128, q);
+        if (hl == 0) sA[(size_t)kb * M + m] = gs.s;
+      }
+    }
+  }
+  // the codes and scales written above must be visible to every CTA's TMA loads and scale copies
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  __threadfence();
+  __syncthreads();
+  bool ok = true;
+  if (threadIdx.x == 0) {
+    uint32_t gen0;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(gen0) : "l"(gbar + 1) : "memory");
+    __threadfence();                                   // the generation is read before arriving
+    const uint32_t old = atomicAdd(gbar, 1u);
+    if (old >= gridDim.x) {
+      raise_device_error(err, kErrWorkspaceDirty);     // arrivals left from a call that did not finish
+      ok = false;
+    } else if (old == gridDim.x - 1) {
+      gbar[0] = 0;                                     // the last to arrive resets the count
+      __threadfence();
+      atomicAdd(gbar + 1, 1u);                         // and releases the others
+    } else {
+      const uint64_t t0 = globaltimer_ns();
+      for (;;) {
+        uint32_t gen;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(gen) : "l"(gbar + 1) : "memory");
+        if (gen != gen0) break;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          raise_device_error(err, kErrWaitTimeout);
+          ok = false;
+          break;
+        }
+        __nanosleep(256);
+      }
+    }
+    __threadfence();
+    s_flag_bar = ok ? 1u : 0u;
+  }
+  __syncthreads();
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  return s_flag_bar != 0;
+}
+
 __device__ __forceinline__ void tile_coords(int t, const Params& p, int* m0, int* n0) {
   int mt, nt;
   tile_walk(t, p.m_tiles, p.n_tiles, p.group_m, &mt, &nt);
@@ -121,7 +209,9 @@ __device__ __forceinline__ void tile_coords(int t, const Params& p, int* m0, int
   *n0 = nt * BN;
 }
 
-template <bool PROMOTE>
+// QPHASE: the fused linear layer's instantiation, whose first phase quantizes the activations
+// (quantize_phase); a separate kernel so the phase's registers do not weigh on the others
+template <bool PROMOTE, bool QPHASE = false>
 __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ CUtensorMap tA,
                                                       const __grid_constant__ CUtensorMap tB, Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -167,7 +257,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ CU
   const uint32_t tmem_base = *tmem_slot;
   allow_dependent_launch();
   grid_dependency_wait();
-  const int my_tiles = p.tiles > (int)blockIdx.x ? (p.tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+  bool phase_ok = true;
+  if constexpr (QPHASE)
+    phase_ok = quantize_phase(p.xq, p.xq_codes, const_cast<float*>(p.sA), (uint32_t)p.M, (uint32_t)p.K, p.gbar, p.err);
+  const int my_tiles = !phase_ok             ? 0
+                       : p.tiles > (int)blockIdx.x ? (p.tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x
+                                                   : 0;
 
   if (warp < kFirstEpiWarp) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
@@ -1253,7 +1348,7 @@ static cudaError_t launch_prefill(const uint8_t* A, const float* sA, int gA, con
   if (!make_tmap_2d(&mA, 1, A, (uint64_t)K, (uint64_t)M, (uint64_t)K, BK, BM, 1)) return cudaErrorInvalidValue;
   if (!b_packed && !make_tmap_2d(&mB, 1, B, (uint64_t)K, (uint64_t)N, (uint64_t)K, BK, BN, 1))
     return cudaErrorInvalidValue;
-  Params p;
+  Params p{};
   p.M = (int)M;
   p.N = (int)N;
   p.K = (int)K;
@@ -1308,6 +1403,64 @@ cudaError_t launch_gemm_to_fp8(const uint8_t* A, const float* sA, int gA, const 
 size_t linear_act_workspace_bytes(int64_t M, int64_t K) {
   const size_t codes = ((size_t)M * (size_t)K + 255) / 256 * 256;
   return codes + (size_t)((K + 127) / 128) * (size_t)M * sizeof(float);
+}
+
+// The fused linear layer (prefill shapes): one cooperative launch of the block-scaled GEMM whose
+// first phase quantizes X into act_ws (the two grid-barrier words in its first 256 bytes, then the
+// codes, then the 1x128 scales),
+// so the codes are read back from L2 by the second phase without a kernel boundary.
+size_t linear_fused_workspace_bytes(int64_t M, int64_t K) {
+  return (linear_act_workspace_bytes(M, K) + 255) / 256 * 256 + 256;
+}
+
+cudaError_t launch_linear_fused(const uint16_t* X, const uint8_t* B, const float* sB, int gB, int64_t M, int64_t N,
+                                int64_t K, uint16_t* C, void* act_ws, cudaStream_t st) {
+  using namespace gemm;
+  if (M <= 64 || N == 0) return M <= 64 ? cudaErrorNotSupported : cudaSuccess;
+  if (M * (K / BK) >= (int64_t(1) << 31)) return cudaErrorNotSupported;   // the phase's group index
+  // the barrier words first, at a place that does not depend on the shape, so one buffer serves
+  // calls of any shape; then the codes and the scales
+  uint32_t* gbar = static_cast<uint32_t*>(act_ws);
+  uint8_t* codes = static_cast<uint8_t*>(act_ws) + 256;
+  float* scales = reinterpret_cast<float*>(codes + ((size_t)M * (size_t)K + 255) / 256 * 256);
+  CUtensorMap mA, mB;
+  std::memset(&mA, 0, sizeof(mA));
+  std::memset(&mB, 0, sizeof(mB));
+  if (!make_tmap_2d(&mA, 1, codes, (uint64_t)K, (uint64_t)M, (uint64_t)K, BK, BM, 1)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&mB, 1, B, (uint64_t)K, (uint64_t)N, (uint64_t)K, BK, BN, 1)) return cudaErrorInvalidValue;
+  Params p{};
+  p.M = (int)M;
+  p.N = (int)N;
+  p.K = (int)K;
+  p.num_kb = (int)(K / BK);
+  p.m_tiles = (int)((M + BM - 1) / BM);
+  p.n_tiles = (int)((N + BN - 1) / BN);
+  p.tiles = p.m_tiles * p.n_tiles;
+  p.group_m = tile_group_m(M, K, p.m_tiles);
+  p.sA = scales;
+  p.sB = sB;
+  p.gA_group = 1;
+  p.gB_block = gB == 2;
+  p.C = C;
+  p.xq = X;
+  p.xq_codes = codes;
+  p.gbar = gbar;
+  p.err = device_error_word();
+  const cudaError_t ea = ensure_dynamic_smem((const void*)k_gemm<true, true>, kSmemBytes);
+  if (ea != cudaSuccess) return ea;
+  // every CTA must be resident for the grid barrier: a cooperative launch guarantees it (one CTA
+  // per SM here) or fails
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)std::max(1, std::min(p.tiles, device_sm_count())));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_gemm<true, true>, mA, mB, p);
 }
 
 cudaError_t launch_linear(const uint16_t* X, const uint8_t* B, const float* sB, int gB, int64_t M, int64_t N,

@@ -145,5 +145,9 @@ size_t linear_act_workspace_bytes(int64_t M, int64_t K);
 cudaError_t launch_linear(const uint16_t* X, const uint8_t* B, const float* sB, int gB, int64_t M, int64_t N,
                           int64_t K, uint16_t* C, void* act_ws, void* gemm_ws, size_t gemm_ws_bytes,
                           cudaStream_t st);
+// the same as one cooperative launch (M > 64): the quantizer as the GEMM kernel's first phase
+size_t linear_fused_workspace_bytes(int64_t M, int64_t K);
+cudaError_t launch_linear_fused(const uint16_t* X, const uint8_t* B, const float* sB, int gB, int64_t M, int64_t N,
+                                int64_t K, uint16_t* C, void* act_ws, cudaStream_t st);
 
 }  // namespace fp8q

@@ -453,6 +453,28 @@ FP8Q_API fp8q_status fp8_gemm_blockscaled_packed(const uint8_t *A, const float *
  * Requirements as for fp8_gemm_blockscaled: N % 128 == 0, K % 128 == 0.
  */
 FP8Q_API size_t fp8q_linear_act_workspace_bytes(int64_t M, int64_t K);
+
+/*
+ * The same linear layer at prefill shapes (M > 64; decode shapes return FP8Q_ERR_UNSUPPORTED) as
+ * ONE cooperative launch: the block-scaled GEMM kernel first quantizes X into act_ws (every
+ * block takes a share of the 1x128 groups, with the stand-alone quantizer's arithmetic), all
+ * blocks meet at a grid barrier, and the GEMM then reads the codes back, from L2 where they
+ * fit.  Output bit-identical to fp8_linear_dynamic.  The pages describe the quantizer and the
+ * GEMM as two steps ([W] "激活动态量化", "FP8 矩阵乘"); this is the fused form of the two.
+ *   act_ws   device, 256-byte aligned, at least fp8q_linear_fused_workspace_bytes(M, K) bytes:
+ *            two grid-barrier words (an arrival count and a generation) in its first 256 bytes,
+ *            then the codes [M][K] (rows of K bytes, the block padded to a multiple of 256
+ *            bytes), then the fp32 scales [K/128][M].  The first 256 bytes must be ZERO-FILLED
+ *            before the first use; every call that completes leaves the arrival count at zero,
+ *            so the buffer is reused as is, by calls of any shape it is large enough for.  After
+ *            a device error zero them again.  Calls sharing one act_ws must not overlap.
+ * Needs every SM free for the grid (a cooperative launch): FP8Q_ERR_UNSUPPORTED when the device
+ * cannot hold the grid at once.
+ */
+FP8Q_API size_t fp8q_linear_fused_workspace_bytes(int64_t M, int64_t K);
+FP8Q_API fp8q_status fp8_linear_dynamic_fused(const void *X, int64_t M, int64_t N, int64_t K, const uint8_t *B,
+                                              const float *sB, fp8q_granularity gB, void *C, void *act_ws,
+                                              size_t act_ws_bytes, fp8q_stream_t stream);
 FP8Q_API fp8q_status fp8_linear_dynamic(const void *X, int64_t M, int64_t N, int64_t K, const uint8_t *B,
                                         const float *sB, fp8q_granularity gB, void *C, void *act_ws,
                                         size_t act_ws_bytes, void *gemm_ws, size_t gemm_ws_bytes,

@@ -223,3 +223,22 @@ def test_gemm_to_fp8_rejects(L):
     assert L.fp8_gemm_blockscaled_to_fp8(a, a, 1, a, a, 2, 256, 256, 256, m, a, None) == 1    # codes alignment
     assert L.fp8_gemm_blockscaled_to_fp8(a, a, 3, a, a, 2, 256, 256, 256, a, a, None) == 1    # gA
     assert L.fp8_gemm_blockscaled_to_fp8(a, a, 1, a, a, 2, 256, 256, 256, a, None, None) == 1  # scales
+
+
+@host_only
+def test_linear_fused_rejects(L):
+    a, m = ALIGNED, MISALIGNED
+    ws = fq.linear_fused_workspace_bytes(256, 512)
+    # codes (M x K, to 256) + scales (K/128 x M floats, to 256) + 256 bytes of barrier words
+    assert ws == 256 * 512 + 4 * 256 * 4 + 256
+    assert fq.linear_fused_workspace_bytes(64, 512) == 0          # decode shapes: not this form
+    assert fq.linear_fused_workspace_bytes(300, 384) == (300 * 384 + 255) // 256 * 256 + (3 * 300 * 4 + 255) // 256 * 256 + 256
+    # (X, M, N, K, B, sB, gB, C, act_ws, act_ws_bytes, stream)
+    assert L.fp8_linear_dynamic_fused(a, 64, 256, 512, a, a, 2, a, a, 1 << 30, None) == 2      # decode shape
+    assert L.fp8_linear_dynamic_fused(a, 256, 200, 512, a, a, 2, a, a, 1 << 30, None) == 2     # N % 128
+    assert L.fp8_linear_dynamic_fused(a, 256, 256, 500, a, a, 2, a, a, 1 << 30, None) == 2     # K % 128
+    assert L.fp8_linear_dynamic_fused(a, 256, 256, 512, a, a, 1, a, a, 1 << 30, None) == 1     # gB
+    assert L.fp8_linear_dynamic_fused(m, 256, 256, 512, a, a, 2, a, a, 1 << 30, None) == 1     # X alignment
+    assert L.fp8_linear_dynamic_fused(a, 256, 256, 512, a, a, 2, a, a, ws - 1, None) == 3      # small act_ws
+    assert L.fp8_linear_dynamic_fused(a, 256, 256, 512, a, a, 2, a, P((1 << 20) + 16), ws, None) == 3  # not 256-aligned
+    assert L.fp8_linear_dynamic_fused(a, 0, 256, 512, a, a, 2, a, None, 0, None) == 0          # empty
