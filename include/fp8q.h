@@ -469,7 +469,9 @@ FP8Q_API size_t fp8q_linear_act_workspace_bytes(int64_t M, int64_t K);
  *            so the buffer is reused as is, by calls of any shape it is large enough for.  After
  *            a device error zero them again.  Calls sharing one act_ws must not overlap.
  * Needs every SM free for the grid (a cooperative launch): FP8Q_ERR_UNSUPPORTED when the device
- * cannot hold the grid at once.
+ * cannot hold the grid at once.  On the measured prefill shapes this form is slower than
+ * fp8_linear_dynamic (its quantize phase runs at the GEMM kernel's occupancy, one block of eight
+ * warps per SM), which remains the faster call.
  */
 FP8Q_API size_t fp8q_linear_fused_workspace_bytes(int64_t M, int64_t K);
 FP8Q_API fp8q_status fp8_linear_dynamic_fused(const void *X, int64_t M, int64_t N, int64_t K, const uint8_t *B,
