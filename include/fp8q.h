@@ -457,9 +457,9 @@ FP8Q_API size_t fp8q_linear_act_workspace_bytes(int64_t M, int64_t K);
 /*
  * The same linear layer at prefill shapes (M > 64; decode shapes return FP8Q_ERR_UNSUPPORTED) as
  * ONE cooperative launch: the block-scaled GEMM kernel first quantizes X into act_ws (every
- * block takes a share of the 1x128 groups, with the stand-alone quantizer's arithmetic), all
- * blocks meet at a grid barrier, and the GEMM then reads the codes back, from L2 where they
- * fit.  Output bit-identical to fp8_linear_dynamic.  The pages describe the quantizer and the
+ * warp of the grid takes a share of the 1x128 groups, with the stand-alone quantizer's
+ * arithmetic), all blocks meet at a grid barrier, and the GEMM then reads the codes back, from
+ * L2 where they fit.  Output bit-identical to fp8_linear_dynamic.  The pages describe the quantizer and the
  * GEMM as two steps ([W] "激活动态量化", "FP8 矩阵乘"); this is the fused form of the two.
  *   act_ws   device, 256-byte aligned, at least fp8q_linear_fused_workspace_bytes(M, K) bytes:
  *            two grid-barrier words (an arrival count and a generation) in its first 256 bytes,
@@ -470,7 +470,7 @@ FP8Q_API size_t fp8q_linear_act_workspace_bytes(int64_t M, int64_t K);
  *            a device error zero them again.  Calls sharing one act_ws must not overlap.
  * Needs every SM free for the grid (a cooperative launch): FP8Q_ERR_UNSUPPORTED when the device
  * cannot hold the grid at once.  On the measured prefill shapes this form is slower than
- * fp8_linear_dynamic (its quantize phase runs at the GEMM kernel's occupancy, one block of eight
+ * fp8_linear_dynamic (its quantize phase runs at the GEMM kernel's occupancy, one block of twelve
  * warps per SM), which remains the faster call.
  */
 FP8Q_API size_t fp8q_linear_fused_workspace_bytes(int64_t M, int64_t K);
